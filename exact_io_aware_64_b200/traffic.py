@@ -1,0 +1,57 @@
+"""Work and memory-traffic arithmetic used for reporting (FLOPs, bytes, score sizes).
+
+None of this runs on the data path; it turns shapes into the figures the benchmark
+divides by.
+"""
+from __future__ import annotations
+
+
+def score_entries(N: int) -> int:
+    """Entries of one head's N x N score matrix ("FlashAttention" page, "A concrete
+    example: 10,000 tokens")."""
+    return N * N
+
+
+def tile_entries(block: int) -> int:
+    """Score entries held on chip for one block x block tile (same example)."""
+    return block * block
+
+
+def materialised_score_bytes(N: int, heads: int = 1, bytes_per_entry: int = 2,
+                             passes: int = 1) -> int:
+    """HBM bytes that standard attention moves for its score matrix.
+
+    One pass is one write or one read of the N x N matrix for every head.  The
+    "FlashAttention" page's example counts write S, read S, write P, read P: four passes.
+    """
+    return passes * bytes_per_entry * score_entries(N) * heads
+
+
+def fwd_flops(B: int, H: int, N: int, d: int, causal: bool) -> float:
+    """Credited forward FLOPs: two N x N x d matrix products, 4 B H N^2 d, halved when
+    causal (only the lower triangle is needed)."""
+    f = 4.0 * B * H * N * N * d
+    return f / 2 if causal else f
+
+
+def bwd_flops(B: int, H: int, N: int, d: int, causal: bool) -> float:
+    """Credited backward FLOPs: five N x N x d products (dV, dP, dQ, dK and the score
+    recompute), 10 B H N^2 d, halved when causal."""
+    f = 10.0 * B * H * N * N * d
+    return f / 2 if causal else f
+
+
+def fwd_compulsory_bytes(B: int, H: int, N: int, d: int, elem_bytes: int = 2,
+                         lse: bool = True) -> int:
+    """Bytes the forward must move at least once: read Q, K, V, write O (and the fp32
+    LSE row statistics)."""
+    b = 4 * B * H * N * d * elem_bytes
+    if lse:
+        b += 4 * B * H * N
+    return b
+
+
+def bwd_compulsory_bytes(B: int, H: int, N: int, d: int, elem_bytes: int = 2) -> int:
+    """Bytes the backward must move at least once: read Q, K, V, O, dO, LSE; write dQ, dK,
+    dV; write and read D once (fp32)."""
+    return 8 * B * H * N * d * elem_bytes + 4 * B * H * N * 3
