@@ -1,0 +1,165 @@
+"""ctypes binding for libfa.so (include/fa.h).
+
+Argument marshalling only: it checks that tensors are CUDA, contiguous and of the right
+shape and dtype, allocates outputs with torch when the caller does not pass them, and
+hands raw pointers and the current CUDA stream to the C ABI.  Every step of the
+computation runs in the library's kernels; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfa.so")
+
+FA_OK = 0
+FA_ERR_INVALID_ARG = 1
+FA_ERR_UNSUPPORTED = 2
+FA_ERR_CUDA = 3
+FA_ERR_TIMEOUT = 4
+
+_lib = None
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_f = ctypes.c_float
+_sz = ctypes.c_size_t
+
+SIGNATURES = {
+    "fa_abi_version": ([], _i),
+    "fa_fwd": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp], _i),
+    "fa_fwd_f32": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp], _i),
+    "fa_bwd_workspace_bytes": ([_i, _i, _i, _i], _sz),
+    "fa_bwd": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _sz,
+                _vp], _i),
+    "fa_status_string": ([_i], ctypes.c_char_p),
+    "fa_last_error_message": ([], ctypes.c_char_p),
+    "fa_check_device_error": ([_vp], _i),
+}
+
+
+class FAError(RuntimeError):
+    def __init__(self, call: str, status: int, message: str):
+        super().__init__(f"{call} failed: {status_name(status)}: {message}")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """Load libfa.so (built in place by ``python -m exact_io_aware_64_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with python -m exact_io_aware_64_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def status_name(status: int) -> str:
+    return lib().fa_status_string(status).decode()
+
+
+def _check(call: str, status: int) -> None:
+    if status != FA_OK:
+        raise FAError(call, status, lib().fa_last_error_message().decode())
+
+
+def _stream_handle(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _check_bhnd(name: str, t: torch.Tensor, shape, dtype) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def fwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, scale: Optional[float] = None,
+        causal: bool = False, O: Optional[torch.Tensor] = None,
+        LSE: Optional[torch.Tensor] = None, want_lse: bool = True,
+        stream: Optional[torch.cuda.Stream] = None):
+    """Exact attention forward through ``fa_fwd`` (bf16) or ``fa_fwd_f32`` (float32).
+
+    Q, K, V: [B, H, N, d] CUDA tensors, contiguous, all bf16 or all float32.
+    Returns (O, LSE); LSE is None when ``want_lse`` is False and none is passed.
+    """
+    B, H, N, d = Q.shape
+    dtype = Q.dtype
+    if dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("Q, K, V must be bfloat16 or float32")
+    for name, t in (("Q", Q), ("K", K), ("V", V)):
+        _check_bhnd(name, t, (B, H, N, d), dtype)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if O is None:
+        O = torch.empty_like(Q)
+    _check_bhnd("O", O, (B, H, N, d), dtype)
+    if LSE is None and want_lse:
+        LSE = torch.empty((B, H, N), device=Q.device, dtype=torch.float32)
+    if LSE is not None:
+        _check_bhnd("LSE", LSE, (B, H, N), torch.float32)
+    fn = lib().fa_fwd if dtype == torch.bfloat16 else lib().fa_fwd_f32
+    with torch.cuda.device(Q.device):
+        st = fn(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), B, H, N, d, float(scale),
+                int(bool(causal)), _stream_handle(stream))
+    _check("fa_fwd" if dtype == torch.bfloat16 else "fa_fwd_f32", st)
+    return O, LSE
+
+
+def workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(lib().fa_bwd_workspace_bytes(B, H, N, d))
+
+
+def bwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, O: torch.Tensor,
+        dO: torch.Tensor, LSE: torch.Tensor, scale: Optional[float] = None,
+        causal: bool = False, dQ: Optional[torch.Tensor] = None,
+        dK: Optional[torch.Tensor] = None, dV: Optional[torch.Tensor] = None,
+        workspace: Optional[torch.Tensor] = None,
+        stream: Optional[torch.cuda.Stream] = None):
+    """Exact attention backward through ``fa_bwd`` (bf16).  Returns (dQ, dK, dV)."""
+    B, H, N, d = Q.shape
+    for name, t in (("Q", Q), ("K", K), ("V", V), ("O", O), ("dO", dO)):
+        _check_bhnd(name, t, (B, H, N, d), torch.bfloat16)
+    _check_bhnd("LSE", LSE, (B, H, N), torch.float32)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dQ = torch.empty_like(Q) if dQ is None else dQ
+    dK = torch.empty_like(K) if dK is None else dK
+    dV = torch.empty_like(V) if dV is None else dV
+    for name, t in (("dQ", dQ), ("dK", dK), ("dV", dV)):
+        _check_bhnd(name, t, (B, H, N, d), torch.bfloat16)
+    need = workspace_bytes(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), device=Q.device, dtype=torch.uint8)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    with torch.cuda.device(Q.device):
+        st = lib().fa_bwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _ptr(LSE), _ptr(dQ),
+                          _ptr(dK), _ptr(dV), B, H, N, d, float(scale), int(bool(causal)),
+                          _ptr(workspace), ws_bytes, _stream_handle(stream))
+    _check("fa_bwd", st)
+    return dQ, dK, dV
+
+
+def check_device_error(stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Synchronise the stream and raise FAError if a kernel reported a wait timeout."""
+    _check("fa_check_device_error", lib().fa_check_device_error(_stream_handle(stream)))

@@ -1,0 +1,298 @@
+// fa_api.cu -- the C ABI declared in include/fa.h: argument validation, TMA tensor-map
+// construction, kernel launches, status reporting.
+//
+// Everything here runs on the host.  Validation happens before any CUDA call, so a bad
+// argument is reported without touching the device.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime_api.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+#include "internal.h"
+
+// Set by kernels when a pipeline wait runs out of time (see sm100.cuh).
+__device__ unsigned int g_fa_device_error;
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+fa_status fail(fa_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  std::vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+fa_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(FA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// ------------------------------------------------------------------ per-device facts
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int num_sms = 0;
+  int cc_major = 0, cc_minor = 0;
+  unsigned int* err = nullptr;  // device address of g_fa_device_error
+};
+
+std::mutex g_dev_mutex;
+DeviceInfo g_dev[kMaxDevices];
+
+fa_status device_info(DeviceInfo* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(FA_ERR_CUDA, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    e = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (e == cudaSuccess) e = cudaGetSymbolAddress(reinterpret_cast<void**>(&d.err), g_fa_device_error);
+    if (e != cudaSuccess) return cuda_fail(e, "querying the device");
+    d.ready = true;
+  }
+  *out = d;
+  return FA_OK;
+}
+
+fa_status require_sm100(const DeviceInfo& d) {
+  if (d.cc_major != 10 || d.cc_minor != 0)
+    return fail(FA_ERR_UNSUPPORTED,
+                "the kernels are built for sm_100a (B200); this device is sm_%d%d",
+                d.cc_major, d.cc_minor);
+  return FA_OK;
+}
+
+// ------------------------------------------------------------------ tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// [BH][N][d] bf16 viewed as a 3-D tensor; boxes of 64 elements x 128 rows x 1 head with
+// the 128-byte swizzle that the tensor-core shared-memory descriptors expect.  Rows
+// past N inside a head read as zeros.
+fa_status make_tmap(CUtensorMap* tm, const void* ptr, int BH, int N, int d) {
+  auto fn = encode_fn();
+  if (!fn) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                           static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return FA_OK;
+}
+
+// ------------------------------------------------------------------ validation
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void* a, const void* b, size_t bytes) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + bytes && y < x + bytes;
+}
+
+// Checks shared by every call.  Sets *noop when there is nothing to compute.
+fa_status check_common(int B, int H, int N, int d, float scale, int causal, bool* noop) {
+  if (B < 0 || H < 0 || N < 0)
+    return fail(FA_ERR_INVALID_ARG, "sizes must be non-negative (B=%d H=%d N=%d)", B, H, N);
+  if (d != 64 && d != 128)
+    return fail(FA_ERR_UNSUPPORTED, "head dimension d=%d is not supported (64 or 128)", d);
+  if (!(std::isfinite(scale) && scale > 0.f))
+    return fail(FA_ERR_INVALID_ARG, "scale must be finite and positive");
+  if (causal != 0 && causal != 1) return fail(FA_ERR_INVALID_ARG, "causal must be 0 or 1");
+  const long long bh = static_cast<long long>(B) * H;
+  // work units and row indices are 32-bit on the device
+  if (bh > 0 && N > 0 && (bh > (1ll << 31) / ((N + 255) / 256) || bh * N >= (1ll << 31)))
+    return fail(FA_ERR_INVALID_ARG, "B*H*N = %lld rows is too large", bh * N);
+  *noop = (bh == 0 || N == 0);
+  return FA_OK;
+}
+
+fa_status check_ptr(const void* p, const char* name) {
+  if (p == nullptr) return fail(FA_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned16(p)) return fail(FA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return FA_OK;
+}
+
+#define FA_TRY(x)                      \
+  do {                                 \
+    fa_status _s = (x);                \
+    if (_s != FA_OK) return _s;        \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+int fa_abi_version(void) { return 1; }
+
+const char* fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+  }
+  return "FA_ERR_UNKNOWN";
+}
+
+const char* fa_last_error_message(void) { return g_last_error; }
+
+fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H,
+                 int N, int d, float scale, int causal, cudaStream_t stream) {
+  g_last_error[0] = '\0';
+  bool noop = false;
+  FA_TRY(check_common(B, H, N, d, scale, causal, &noop));
+  if (noop) return FA_OK;  // empty problem: the pointers are never used (may be NULL)
+  FA_TRY(check_ptr(Q, "Q"));
+  FA_TRY(check_ptr(K, "K"));
+  FA_TRY(check_ptr(V, "V"));
+  FA_TRY(check_ptr(O, "O"));
+  if (LSE != nullptr && (reinterpret_cast<uintptr_t>(LSE) & 3u))
+    return fail(FA_ERR_INVALID_ARG, "LSE is not 4-byte aligned");
+  const size_t bytes = static_cast<size_t>(B) * H * N * d * 2;
+  if (overlaps(O, Q, bytes) || overlaps(O, K, bytes) || overlaps(O, V, bytes))
+    return fail(FA_ERR_INVALID_ARG, "O overlaps an input");
+  DeviceInfo dev;
+  FA_TRY(device_info(&dev));
+  FA_TRY(require_sm100(dev));
+  const int BH = B * H;
+  CUtensorMap tmQ, tmK, tmV;
+  FA_TRY(make_tmap(&tmQ, Q, BH, N, d));
+  FA_TRY(make_tmap(&tmK, K, BH, N, d));
+  FA_TRY(make_tmap(&tmV, V, BH, N, d));
+  fa::Problem p{BH, N, d, scale, causal, dev.err};
+  cudaError_t e = fa::launch_fwd_sm100(tmQ, tmK, tmV, O, LSE, p, dev.num_sms, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "launching the forward kernel");
+  return FA_OK;
+}
+
+fa_status fa_fwd_f32(const float* Q, const float* K, const float* V, float* O, float* LSE,
+                     int B, int H, int N, int d, float scale, int causal,
+                     cudaStream_t stream) {
+  g_last_error[0] = '\0';
+  bool noop = false;
+  FA_TRY(check_common(B, H, N, d, scale, causal, &noop));
+  if (noop) return FA_OK;  // empty problem: the pointers are never used (may be NULL)
+  FA_TRY(check_ptr(Q, "Q"));
+  FA_TRY(check_ptr(K, "K"));
+  FA_TRY(check_ptr(V, "V"));
+  FA_TRY(check_ptr(O, "O"));
+  if (LSE != nullptr && (reinterpret_cast<uintptr_t>(LSE) & 3u))
+    return fail(FA_ERR_INVALID_ARG, "LSE is not 4-byte aligned");
+  const size_t bytes = static_cast<size_t>(B) * H * N * d * 4;
+  if (overlaps(O, Q, bytes) || overlaps(O, K, bytes) || overlaps(O, V, bytes))
+    return fail(FA_ERR_INVALID_ARG, "O overlaps an input");
+  DeviceInfo dev;
+  FA_TRY(device_info(&dev));
+  fa::Problem p{B * H, N, d, scale, causal, dev.err};
+  cudaError_t e = fa::launch_fwd_f32(Q, K, V, O, LSE, p, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "launching the float32 forward kernel");
+  return FA_OK;
+}
+
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
+  (void)d;
+  if (B <= 0 || H <= 0 || N <= 0) return 0;
+  const size_t raw = static_cast<size_t>(B) * H * N * sizeof(float);
+  return (raw + 255) / 256 * 256;
+}
+
+fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                 const float* LSE, void* dQ, void* dK, void* dV, int B, int H, int N, int d,
+                 float scale, int causal, void* workspace, size_t workspace_bytes,
+                 cudaStream_t stream) {
+  g_last_error[0] = '\0';
+  bool noop = false;
+  FA_TRY(check_common(B, H, N, d, scale, causal, &noop));
+  if (noop) return FA_OK;  // empty problem: the pointers are never used (may be NULL)
+  FA_TRY(check_ptr(Q, "Q"));
+  FA_TRY(check_ptr(K, "K"));
+  FA_TRY(check_ptr(V, "V"));
+  FA_TRY(check_ptr(O, "O"));
+  FA_TRY(check_ptr(dO, "dO"));
+  FA_TRY(check_ptr(LSE, "LSE"));
+  FA_TRY(check_ptr(dQ, "dQ"));
+  FA_TRY(check_ptr(dK, "dK"));
+  FA_TRY(check_ptr(dV, "dV"));
+  const size_t need = fa_bwd_workspace_bytes(B, H, N, d);
+  if (need > 0) {
+    FA_TRY(check_ptr(workspace, "workspace"));
+    if (workspace_bytes < need)
+      return fail(FA_ERR_INVALID_ARG, "workspace has %zu bytes, %zu needed", workspace_bytes,
+                  need);
+  }
+  const size_t bytes = static_cast<size_t>(B) * H * N * d * 2;
+  const void* ins[5] = {Q, K, V, O, dO};
+  void* outs[3] = {dQ, dK, dV};
+  for (void* o : outs) {
+    for (const void* in : ins)
+      if (overlaps(o, in, bytes)) return fail(FA_ERR_INVALID_ARG, "a gradient overlaps an input");
+    if (need > 0 && overlaps(o, workspace, need > bytes ? need : bytes))
+      return fail(FA_ERR_INVALID_ARG, "a gradient overlaps the workspace");
+  }
+  if (overlaps(dQ, dK, bytes) || overlaps(dQ, dV, bytes) || overlaps(dK, dV, bytes))
+    return fail(FA_ERR_INVALID_ARG, "gradients overlap each other");
+  DeviceInfo dev;
+  FA_TRY(device_info(&dev));
+  FA_TRY(require_sm100(dev));
+  const int BH = B * H;
+  CUtensorMap tmQ, tmK, tmV, tmdO;
+  FA_TRY(make_tmap(&tmQ, Q, BH, N, d));
+  FA_TRY(make_tmap(&tmK, K, BH, N, d));
+  FA_TRY(make_tmap(&tmV, V, BH, N, d));
+  FA_TRY(make_tmap(&tmdO, dO, BH, N, d));
+  fa::Problem p{BH, N, d, scale, causal, dev.err};
+  cudaError_t e = fa::launch_bwd_sm100(tmQ, tmK, tmV, tmdO, O, dO, LSE, dQ, dK, dV,
+                                       static_cast<float*>(workspace), p, dev.num_sms, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "launching the backward kernels");
+  return FA_OK;
+}
+
+fa_status fa_check_device_error(cudaStream_t stream) {
+  g_last_error[0] = '\0';
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  DeviceInfo dev;
+  FA_TRY(device_info(&dev));
+  unsigned int word = 0;
+  e = cudaMemcpy(&word, dev.err, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  if (word != 0) {
+    const unsigned int zero = 0;
+    e = cudaMemcpy(dev.err, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+    return fail(FA_ERR_TIMEOUT, "a kernel pipeline wait timed out (error word 0x%x)", word);
+  }
+  return FA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,115 @@
+// fwd_f32.cu -- forward attention in float32 on the CUDA cores.
+//
+// Same tiled online softmax as the tensor-core path ("FlashAttention, simplified", "The
+// trick"): per query row a running max m, running sum l and accumulator acc; each block
+// of 32 keys is scored, the max updated, acc and l rescaled by exp(m - m_new), and O =
+// acc / l at the end.  Every step is float32 (no TF32, no bf16 rounding).
+//
+// Mapping: a CTA of 128 threads owns 32 query rows of one (batch, head); four threads
+// share a row, each holding every fourth element of q and acc, and combine their partial
+// dot products with two shuffles.  The key and value blocks are staged in shared memory.
+#include <cmath>
+#include <cstdint>
+
+#include "internal.h"
+
+namespace fa {
+namespace {
+
+constexpr int kRows = 32;     // query rows per CTA
+constexpr int kKeys = 32;     // keys per shared-memory block
+constexpr int kThreads = 128; // 4 threads per row
+
+template <int D>
+__global__ void __launch_bounds__(kThreads)
+    fwd_f32_kernel(const float* __restrict__ Q, const float* __restrict__ K,
+                   const float* __restrict__ V, float* __restrict__ O,
+                   float* __restrict__ LSE, int N, float scale, int causal) {
+  constexpr int E = D / 4;  // elements of q / acc per thread
+  __shared__ float Ks[kKeys][D];
+  __shared__ float Vs[kKeys][D];
+
+  const int bh = blockIdx.y;
+  const int r = threadIdx.x / 4;  // row within the CTA
+  const int part = threadIdx.x % 4;
+  const int row = blockIdx.x * kRows + r;
+  const bool valid = row < N;
+  const size_t head = static_cast<size_t>(bh) * N * D;
+
+  float q[E], acc[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    q[e] = valid ? Q[head + static_cast<size_t>(row) * D + 4 * e + part] : 0.f;
+    acc[e] = 0.f;
+  }
+  float m = -INFINITY, l = 0.f;
+
+  const int last_row = min(N - 1, (blockIdx.x + 1) * kRows - 1);
+  const int key_end = causal ? last_row + 1 : N;
+  for (int k0 = 0; k0 < key_end; k0 += kKeys) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < kKeys * D; i += kThreads) {
+      const int kr = i / D, c = i % D;
+      const int key = k0 + kr;
+      const bool in = key < N;
+      Ks[kr][c] = in ? K[head + static_cast<size_t>(key) * D + c] : 0.f;
+      Vs[kr][c] = in ? V[head + static_cast<size_t>(key) * D + c] : 0.f;
+    }
+    __syncthreads();
+    float s[kKeys];
+    float tile_max = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < kKeys; ++j) {
+      float part_dot = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) part_dot = fmaf(q[e], Ks[j][4 * e + part], part_dot);
+      part_dot += __shfl_xor_sync(0xffffffffu, part_dot, 1);
+      part_dot += __shfl_xor_sync(0xffffffffu, part_dot, 2);
+      const int key = k0 + j;
+      const bool visible = key < N && (!causal || key <= row);
+      s[j] = visible ? part_dot * scale : -INFINITY;
+      tile_max = fmaxf(tile_max, s[j]);
+    }
+    const float m_new = fmaxf(m, tile_max);
+    if (m_new == -INFINITY) continue;  // nothing visible yet for this row
+    const float alpha = expf(m - m_new);
+    float psum = 0.f;
+#pragma unroll
+    for (int j = 0; j < kKeys; ++j) {
+      s[j] = expf(s[j] - m_new);
+      psum += s[j];
+    }
+    l = alpha * l + psum;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      float a = alpha * acc[e];
+#pragma unroll
+      for (int j = 0; j < kKeys; ++j) a = fmaf(s[j], Vs[j][4 * e + part], a);
+      acc[e] = a;
+    }
+    m = m_new;
+  }
+  if (!valid) return;
+  const float inv_l = 1.f / l;
+#pragma unroll
+  for (int e = 0; e < E; ++e) O[head + static_cast<size_t>(row) * D + 4 * e + part] = acc[e] * inv_l;
+  if (LSE != nullptr && part == 0) LSE[static_cast<size_t>(bh) * N + row] = m + logf(l);
+}
+
+template <int D>
+cudaError_t launch_d(const float* Q, const float* K, const float* V, float* O, float* LSE,
+                     const Problem& p, cudaStream_t stream) {
+  dim3 grid((p.N + kRows - 1) / kRows, p.BH);
+  fwd_f32_kernel<D><<<grid, kThreads, 0, stream>>>(Q, K, V, O, LSE, p.N, p.scale, p.causal);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_f32(const float* Q, const float* K, const float* V, float* O,
+                           float* LSE, const Problem& p, cudaStream_t stream) {
+  if (p.d == 64) return launch_d<64>(Q, K, V, O, LSE, p, stream);
+  return launch_d<128>(Q, K, V, O, LSE, p, stream);
+}
+
+}  // namespace fa

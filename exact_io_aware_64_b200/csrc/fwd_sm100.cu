@@ -1,0 +1,481 @@
+// fwd_sm100.cu -- forward attention on the sm_100a tensor cores.
+//
+// Method ("FlashAttention, simplified", "The trick"; "FlashAttention" page, "The
+// bottleneck is memory, not multiplication" and "A concrete example: 10,000 tokens"):
+// for a block of queries, walk the key/value blocks, form the 128 x 128 score tile on
+// chip, keep a running row max m and running sum l, rescale the accumulated output when
+// the max grows, add exp(S - m) V, and divide by l once at the end.  The N x N scores
+// never leave the SM.
+//
+// B200 mapping
+//   * One persistent CTA per SM walks a static list of work units; a unit is two
+//     128-row query tiles (Q0, Q1) of one (batch, head), so every K/V tile that TMA
+//     brings in is used by 256 query rows.
+//   * Warp roles (384 threads, three warpgroups): warps 0-3 own the softmax of Q0 (one
+//     thread per row, TMEM lane = row), warps 4-7 the softmax of Q1, warp 8 issues TMA
+//     loads, warp 9 issues tcgen05 MMAs from one thread, warps 10-11 only give up their
+//     registers.  The launch grants 168 registers a thread (384 x 168 = 64512); the
+//     control warpgroup drops to 56 and the two softmax warpgroups rise to 224, which
+//     uses exactly that pool (2 x 128 x 224 + 128 x 56 = 64512) and lets a softmax
+//     thread hold its whole 128-entry score row in registers.
+//   * TMEM (512 columns): S0 | S1 | O0 | O1.  The score tile S_t = Q_t K_j^T lands in
+//     TMEM as fp32; the softmax threads read their row, write the probabilities as bf16
+//     over the first 64 columns of the same S_t region, and the MMA O_t += P_t V_j
+//     takes P straight from TMEM (A operand) and V from shared memory.
+//   * The MMA issue order S0(0) S1(0) | PV0(0) S0(1) PV1(0) S1(1) | PV0(1) ... lets the
+//     tensor core work on one tile's products while the other tile's softmax runs.
+//   * The running max is kept in log2 units.  The output is rescaled only when a row's
+//     max grows by more than kRescaleThreshold (a factor 2^8); otherwise the older,
+//     smaller reference max stays in force, which is exact because l and O always use
+//     the same reference, and keeps every exponential below 2^8.
+//   * K/V tiles stream through a ring of shared-memory slots guarded by mbarriers
+//     (full: TMA transaction bytes; empty: tcgen05.commit from the MMA thread).
+//   * Causal: query tile q needs key tiles 0..q; only the diagonal tile and a ragged
+//     last key tile need element masks.  Rows past N (ragged last query tile) are
+//     computed on zero-filled Q and never stored.
+#include <cfloat>
+#include <cstdint>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace fa {
+namespace {
+
+using namespace sm100;
+
+constexpr int kBM = 128;  // query rows per tile
+constexpr int kBN = 128;  // key rows per tile
+constexpr int kThreads = 384;
+constexpr int kRegsLaunch = 168;   // 65536 / 384, rounded down to a multiple of 8
+constexpr int kRegsControl = 56;
+constexpr int kRegsSoftmax = 224;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kThreads * kRegsLaunch,
+              "register split exceeds the launch pool");
+constexpr int kWarpTMA = 8;
+constexpr int kWarpMMA = 9;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr uint32_t kTmemCols = 512;
+
+template <int D>
+struct FwdLayout {
+  static constexpr int kTileBytes = kBM * D * 2;  // one 128-row bf16 tile
+  static constexpr int kBoxBytes = 128 * 128;     // one 128-row x 64-col box
+  static constexpr int kStages = (D == 128) ? 4 : 8;
+  static constexpr int kQ0 = 0;
+  static constexpr int kQ1 = kTileBytes;
+  static constexpr int kRing = 2 * kTileBytes;
+  static constexpr int kBar = kRing + kStages * kTileBytes;
+  // barrier indices
+  static constexpr int kBarQFull = 0;                 // [2]
+  static constexpr int kBarQEmpty = 2;                // [2]
+  static constexpr int kBarKVFull = 4;                // [kStages]
+  static constexpr int kBarKVEmpty = 4 + kStages;     // [kStages]
+  static constexpr int kBarSFull = 4 + 2 * kStages;   // [2]
+  static constexpr int kBarPReady = 6 + 2 * kStages;  // [2]
+  static constexpr int kBarODone = 8 + 2 * kStages;   // [2]
+  static constexpr int kBarOFree = 10 + 2 * kStages;  // [2]
+  static constexpr int kBarDrain = 12 + 2 * kStages;  // [1]
+  static constexpr int kNumBars = 13 + 2 * kStages;
+  static constexpr int kMisc = kBar + kNumBars * 8;
+  static constexpr int kBytes = kMisc + 16;
+  static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024 bytes
+};
+
+struct FwdArgs {
+  unsigned int* err;  // library error word (wait timeouts)
+  __nv_bfloat16* O;
+  float* LSE;
+  int BH;
+  int N;
+  int causal;
+  int n_units;      // units per (batch, head) = ceil(N / 256)
+  int total_units;  // BH * n_units
+  float scale_log2;  // scale * log2(e)
+};
+
+struct UnitInfo {
+  int bh, u, n0, n1;
+};
+
+__device__ __forceinline__ UnitInfo unit_info(int w, const FwdArgs& a) {
+  UnitInfo r;
+  if (a.causal) {
+    // heaviest units (largest query index) first, all heads of one row-band together
+    r.u = a.n_units - 1 - w / a.BH;
+    r.bh = w % a.BH;
+  } else {
+    r.bh = w / a.n_units;
+    r.u = w % a.n_units;
+  }
+  const int n_kv = (a.N + kBN - 1) / kBN;
+  const int qt0 = 2 * r.u, qt1 = 2 * r.u + 1;
+  const bool valid1 = qt1 * kBM < a.N;
+  r.n0 = a.causal ? min(qt0 + 1, n_kv) : n_kv;
+  r.n1 = valid1 ? (a.causal ? min(qt1 + 1, n_kv) : n_kv) : 0;
+  return r;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
+                     const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const FwdArgs args) {
+  using L = FwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base = (raw_addr + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw_addr);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  auto bar = [&](int i) -> uint32_t { return base + L::kBar + 8 * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  auto wait = [&](uint32_t b, uint32_t parity) -> bool {
+    return mbar_wait(b, parity, abort_flag, args.err);
+  };
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(bar(L::kBarQFull + 0), 1);
+    mbar_init(bar(L::kBarQFull + 1), 1);
+    mbar_init(bar(L::kBarQEmpty + 0), 1);
+    mbar_init(bar(L::kBarQEmpty + 1), 1);
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(bar(L::kBarKVFull + s), 1);
+      mbar_init(bar(L::kBarKVEmpty + s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(L::kBarSFull + t), 1);
+      mbar_init(bar(L::kBarPReady + t), kBM);
+      mbar_init(bar(L::kBarODone + t), 1);
+      mbar_init(bar(L::kBarOFree + t), kBM);
+    }
+    mbar_init(bar(L::kBarDrain), 1);
+    fence_mbar_init();
+  }
+  if (warp == kWarpTMA && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == kWarpMMA) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS[2] = {tmem, tmem + 128};
+  const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
+
+  if (warp >= 8) regs_dec<kRegsControl>();
+  if (warp == kWarpTMA) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int q_uses[2] = {0, 0};
+      bool ok = true;
+      int issued[L::kStages];
+      uint32_t issued_phase[L::kStages];
+      for (int s = 0; s < L::kStages; ++s) issued[s] = 0, issued_phase[s] = 0;
+      for (int w = blockIdx.x; ok && w < args.total_units; w += gridDim.x) {
+        const UnitInfo ui = unit_info(w, args);
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (t == 1 && ui.n1 == 0) break;
+          if (q_uses[t] > 0)
+            ok = wait(bar(L::kBarQEmpty + t), (q_uses[t] - 1) & 1);
+          if (!ok) break;
+          const uint32_t qb = bar(L::kBarQFull + t);
+          mbar_arrive_expect_tx(qb, L::kTileBytes);
+          const uint32_t dst = base + (t == 0 ? L::kQ0 : L::kQ1);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(dst + c * L::kBoxBytes, &tmQ, qb, c * 64, (2 * ui.u + t) * kBM, ui.bh);
+          ++q_uses[t];
+        }
+        const int n = max(ui.n0, ui.n1);
+        for (int j = 0; ok && j < n; ++j) {
+          for (int kv = 0; kv < 2; ++kv) {  // K_j then V_j
+            ok = wait(bar(L::kBarKVEmpty + stage), phase ^ 1);
+            if (!ok) break;
+            const uint32_t fb = bar(L::kBarKVFull + stage);
+            mbar_arrive_expect_tx(fb, L::kTileBytes);
+            const uint32_t dst = base + L::kRing + stage * L::kTileBytes;
+            const CUtensorMap* tm = kv == 0 ? &tmK : &tmV;
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_3d(dst + c * L::kBoxBytes, tm, fb, c * 64, j * kBN, ui.bh);
+            issued[stage] = 1;
+            issued_phase[stage] = phase;
+            if (++stage == L::kStages) stage = 0, phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        // wind down: let every load already issued land before the CTA exits
+        for (int s = 0; s < L::kStages; ++s)
+          if (issued[s]) mbar_wait_drain(bar(L::kBarKVFull + s), issued_phase[s], args.err);
+        for (int t = 0; t < 2; ++t)
+          if (q_uses[t] > 0)
+            mbar_wait_drain(bar(L::kBarQFull + t), (q_uses[t] - 1) & 1, args.err);
+      }
+    }
+  } else if (warp == kWarpMMA) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(kBN, false);
+      constexpr uint32_t idPV = idesc_bf16_f32(D, true);
+      int stage = 0;
+      uint32_t phase = 0;
+      int uses[2] = {0, 0};
+      int p_count[2] = {0, 0};
+      bool ok = true;
+      auto next_slot = [&](int& slot) -> bool {
+        slot = stage;
+        const bool r = wait(bar(L::kBarKVFull + stage), phase);
+        if (++stage == L::kStages) stage = 0, phase ^= 1;
+        return r;
+      };
+      // Descriptors differ only in their start-address field (low 14 bits, address >> 4),
+      // so each K step adds its byte offset >> 4 to a base descriptor.
+      const uint64_t dQ0 = desc_kmajor(base + L::kQ0);
+      const uint64_t dQ1 = desc_kmajor(base + L::kQ1);
+      const uint64_t dRingK = desc_kmajor(base + L::kRing);
+      const uint64_t dRingV = desc_mnmajor(base + L::kRing, L::kBoxBytes);
+      auto issue_s = [&](int t, int kslot) {
+        const uint64_t da = t == 0 ? dQ0 : dQ1;
+        const uint64_t db = dRingK + static_cast<uint64_t>((kslot * L::kTileBytes) >> 4);
+#pragma unroll 1
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk / 4) * L::kBoxBytes + (kk % 4) * 32) >> 4;
+          mma_ss(tS[t], da + off, db + off, idS, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar(L::kBarSFull + t));
+      };
+      auto issue_pv = [&](int t, int vslot, bool accumulate) {
+        const uint64_t db = dRingV + static_cast<uint64_t>((vslot * L::kTileBytes) >> 4);
+#pragma unroll 1
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          mma_ts(tO[t], tS[t] + kk * 8, db + static_cast<uint64_t>((kk * 2048) >> 4), idPV,
+                 (accumulate || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(bar(L::kBarODone + t));
+      };
+      for (int w = blockIdx.x; ok && w < args.total_units; w += gridDim.x) {
+        const UnitInfo ui = unit_info(w, args);
+        const int nt[2] = {ui.n0, ui.n1};
+        const int n = max(ui.n0, ui.n1);
+        for (int t = 0; t < 2 && ok; ++t)
+          if (nt[t] > 0) ok = wait(bar(L::kBarQFull + t), uses[t] & 1);
+        if (!ok) break;
+        int kslot;
+        ok = next_slot(kslot);
+        if (!ok) break;
+        tc_fence_after();
+        for (int t = 0; t < 2; ++t) {
+          if (nt[t] > 0) {
+            issue_s(t, kslot);
+            if (nt[t] == 1) mma_commit(bar(L::kBarQEmpty + t));
+          }
+        }
+        mma_commit(bar(L::kBarKVEmpty + kslot));
+        for (int j = 0; ok && j < n; ++j) {
+          int vslot, knext = -1;
+          ok = next_slot(vslot);
+          if (ok && j + 1 < n) ok = next_slot(knext);
+          if (!ok) break;
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (j >= nt[t]) continue;
+            if (j == 0 && uses[t] > 0)
+              ok = wait(bar(L::kBarOFree + t), (uses[t] - 1) & 1);
+            if (ok) ok = wait(bar(L::kBarPReady + t), p_count[t] & 1);
+            if (!ok) break;
+            ++p_count[t];
+            tc_fence_after();
+            issue_pv(t, vslot, j > 0);
+            if (j + 1 < nt[t]) {
+              issue_s(t, knext);
+              if (j + 2 == nt[t]) mma_commit(bar(L::kBarQEmpty + t));
+            }
+          }
+          if (!ok) break;
+          mma_commit(bar(L::kBarKVEmpty + vslot));
+          if (knext >= 0) mma_commit(bar(L::kBarKVEmpty + knext));
+        }
+        for (int t = 0; t < 2; ++t)
+          if (nt[t] > 0) ++uses[t];
+      }
+      // drain: every MMA issued has completed before TMEM is released
+      mma_commit(bar(L::kBarDrain));
+      mbar_wait_drain(bar(L::kBarDrain), 0, args.err);
+    }
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ softmax, tile t
+    regs_inc<kRegsSoftmax>();
+    const int t = warp / 4;
+    const int row = (warp % 4) * 32 + lane;        // row within the tile = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>((warp % 4) * 32) << 16;
+    const uint32_t tSrow = tS[t] + lane_off;
+    const uint32_t tOrow = tO[t] + lane_off;
+    int s_count = 0, o_count = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; ok && w < args.total_units; w += gridDim.x) {
+      const UnitInfo ui = unit_info(w, args);
+      const int n_t = t == 0 ? ui.n0 : ui.n1;
+      if (n_t == 0) continue;
+      const int qt = 2 * ui.u + t;
+      const int q_row = qt * kBM + row;
+      float m = -INFINITY;  // running max, log2 units (scaled logits * log2 e)
+      float l = 0.f;
+      for (int j = 0; j < n_t; ++j) {
+        ok = wait(bar(L::kBarSFull + t), s_count & 1);
+        if (!ok) break;
+        ++s_count;
+        tc_fence_after();
+        uint32_t sr[kBN];
+#pragma unroll
+        for (int c = 0; c < kBN / 32; ++c) tmem_ld32(tSrow + c * 32, &sr[c * 32]);
+        tmem_wait_ld();
+        float s[kBN];
+#pragma unroll
+        for (int c = 0; c < kBN; ++c) s[c] = __uint_as_float(sr[c]);
+        const int kv0 = j * kBN;
+        const bool need_mask = (kv0 + kBN > args.N) || (args.causal && j == qt);
+        if (need_mask) {
+          const int lim = args.causal ? min(args.N, q_row + 1) : args.N;
+#pragma unroll
+          for (int c = 0; c < kBN; ++c)
+            if (kv0 + c >= lim) s[c] = -INFINITY;
+        }
+        float mx = s[0];
+#pragma unroll
+        for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, s[c]);
+        const float m_tile = mx * args.scale_log2;
+        float alpha = 1.f;
+        bool rescale = false;
+        if (m_tile > m + kRescaleThreshold || m == -INFINITY) {
+          const float m_new = fmaxf(m, m_tile);
+          alpha = (m == -INFINITY) ? 0.f : ex2_approx(m - m_new);
+          m = m_new;
+          rescale = true;
+        }
+        if (__any_sync(0xffffffffu, rescale && j > 0)) {
+          // O_t holds the sum through key tile j-1: wait for that product, then scale
+          ok = wait(bar(L::kBarODone + t), (o_count + j - 1) & 1);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tOrow + c * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+              v[k] = __float_as_uint(__uint_as_float(v[k]) * alpha);
+            tmem_st32(tOrow + c * 32, v);
+          }
+        }
+        l *= alpha;
+        const float mref = (m == -INFINITY) ? 0.f : m;
+        uint32_t pk[kBN / 2];
+        float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+        for (int c = 0; c < kBN / 2; ++c) {
+          const float p0 = ex2_approx(fmaf(s[2 * c], args.scale_log2, -mref));
+          const float p1 = ex2_approx(fmaf(s[2 * c + 1], args.scale_log2, -mref));
+          ls0 += p0;
+          ls1 += p1;
+          pk[c] = pack_bf16x2(p0, p1);
+        }
+        l += ls0 + ls1;
+        tmem_st32(tSrow, &pk[0]);
+        tmem_st32(tSrow + 32, &pk[32]);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(L::kBarPReady + t));
+      }
+      if (!ok) break;
+      // epilogue: O = acc / l, LSE = (m + log2 l) * ln 2
+      ok = wait(bar(L::kBarODone + t), (o_count + n_t - 1) & 1);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      o_count += n_t;
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+      const int bh = ui.bh;
+      __nv_bfloat16* orow = args.O + (static_cast<size_t>(bh) * args.N + q_row) * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tOrow + c * 32, v);
+        tmem_wait_ld();
+        if (q_row < args.N) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k)
+            pk[k] = pack_bf16x2(__uint_as_float(v[2 * k]) * inv_l,
+                                __uint_as_float(v[2 * k + 1]) * inv_l);
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(L::kBarOFree + t));
+      if (args.LSE != nullptr && q_row < args.N)
+        args.LSE[static_cast<size_t>(bh) * args.N + q_row] =
+            (m + __log2f(l)) * 0.69314718055994531f;
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMMA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int D>
+cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                     void* O, float* LSE, const Problem& p, int num_sms, cudaStream_t stream) {
+  using L = FwdLayout<D>;
+  FwdArgs a;
+  a.err = p.err;
+  a.O = static_cast<__nv_bfloat16*>(O);
+  a.LSE = LSE;
+  a.BH = p.BH;
+  a.N = p.N;
+  a.causal = p.causal;
+  a.n_units = (p.N + 2 * kBM - 1) / (2 * kBM);
+  a.total_units = p.BH * a.n_units;
+  a.scale_log2 = p.scale * 1.4426950408889634f;
+  // The register split inside the kernel assumes exactly kRegsLaunch registers a thread
+  // at launch; with fewer, the softmax warpgroups' increase could never be granted.
+  cudaFuncAttributes fattr;
+  cudaError_t e = cudaFuncGetAttributes(&fattr, fwd_sm100_kernel<D>);
+  if (e != cudaSuccess) return e;
+  if (fattr.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
+  e = cudaFuncSetAttribute(fwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           L::kAlloc);
+  if (e != cudaSuccess) return e;
+  const int grid = a.total_units < num_sms ? a.total_units : num_sms;
+  fwd_sm100_kernel<D><<<grid, kThreads, L::kAlloc, stream>>>(tmQ, tmK, tmV, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_sm100(const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                             const CUtensorMap& tmV, void* O, float* LSE, const Problem& p,
+                             int num_sms, cudaStream_t stream) {
+  if (p.d == 64) return launch_d<64>(tmQ, tmK, tmV, O, LSE, p, num_sms, stream);
+  return launch_d<128>(tmQ, tmK, tmV, O, LSE, p, num_sms, stream);
+}
+
+}  // namespace fa

@@ -1,0 +1,37 @@
+// internal.h -- launch interfaces shared between the API layer (fa_api.cu) and the
+// kernel translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime_api.h>
+#include <cstddef>
+
+namespace fa {
+
+// Problem shared by every kernel: [B*H, N, d] tensors, contiguous.
+struct Problem {
+  int BH;
+  int N;
+  int d;
+  float scale;
+  int causal;
+  unsigned int* err;  // device address of the library's error word
+};
+
+// Forward, bf16, tcgen05.  Tensor maps describe Q, K, V as 3-D [BH][N][d] bf16 with
+// 64 x 128 x 1 boxes and the 128-byte swizzle.
+cudaError_t launch_fwd_sm100(const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                             const CUtensorMap& tmV, void* O, float* LSE, const Problem& p,
+                             int num_sms, cudaStream_t stream);
+
+// Forward, float32 on the CUDA cores.
+cudaError_t launch_fwd_f32(const float* Q, const float* K, const float* V, float* O,
+                           float* LSE, const Problem& p, cudaStream_t stream);
+
+// Backward, bf16: D = rowsum(dO * O), then dK/dV, then dQ.
+cudaError_t launch_bwd_sm100(const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                             const CUtensorMap& tmV, const CUtensorMap& tmdO, const void* O,
+                             const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                             float* Dbuf, const Problem& p, int num_sms, cudaStream_t stream);
+
+}  // namespace fa

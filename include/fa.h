@@ -1,0 +1,136 @@
+/*
+ * fa.h -- C ABI of libfa.so: exact scaled dot-product attention, computed tile by tile
+ * with an online softmax so that the N x N score matrix never reaches device memory.
+ *
+ * What the calls compute
+ *   Forward ("FlashAttention" page, introduction and "The bottleneck is memory, not
+ *   multiplication"; "FlashAttention, simplified", "The trick"):
+ *       S  = scale * Q K^T            (per batch b and head h, N x N)
+ *       S_ij = -inf where causal and j > i   (query i sees keys 0..i)
+ *       O  = softmax_rows(S) V
+ *       LSE_i = log(sum_j exp(S_ij))  (natural log, of the scaled and masked logits)
+ *   The result is the plain definition above; only the order of floating-point
+ *   operations differs (tiles of 128 keys, running max and running sum, one final
+ *   division).
+ *   Backward ("What FlashAttention actually buys", "Why the distinction matters
+ *   downstream": the backward recomputes the score tiles instead of storing them):
+ *       P = exp(S - LSE), dV = P^T dO, dP = dO V^T, D_i = sum_k dO_ik O_ik,
+ *       dS = P * (dP - D), dQ = scale dS K, dK = scale dS^T Q.
+ *
+ * Layout and types
+ *   Q, K, V, O, dO, dQ, dK, dV: [B, H, N, d] contiguous row-major (d fastest).  bf16 in
+ *   the bf16 calls (__nv_bfloat16, passed as void*), float in the _f32 calls.
+ *   LSE: [B, H, N] float32.  All pointers are device pointers.
+ *   Arithmetic: bf16 inputs, float32 accumulation and softmax statistics; the bf16 calls
+ *   round the probabilities (and dS in the backward) to bf16 before the second matrix
+ *   product.  The _f32 calls compute in float32 throughout.
+ *
+ * Ownership and asynchrony
+ *   The caller allocates and owns every buffer.  The library allocates no device memory
+ *   and keeps no per-call state; it reads the device's SM count once per device.  Each
+ *   call validates its arguments on the host, enqueues kernels on `stream` and returns;
+ *   the results are ready when `stream` reaches that point.  A return of FA_OK says the
+ *   launch was accepted; errors raised while the kernels run are reported by
+ *   fa_check_device_error().
+ *
+ * Errors
+ *   FA_ERR_INVALID_ARG  null or misaligned pointer (16-byte alignment is required),
+ *                       negative size, B*H*N too large, non-finite or non-positive
+ *                       scale, causal not 0/1, workspace too small, O aliasing an input.
+ *   FA_ERR_UNSUPPORTED  head dimension other than 64 or 128.
+ *   FA_ERR_CUDA         a CUDA runtime call failed (launch error, no device, ...).
+ *   FA_ERR_TIMEOUT      a kernel gave up waiting on one of its own pipeline barriers
+ *                       (reported by fa_check_device_error; the outputs are invalid).
+ *   On any error the outputs are unspecified.  fa_last_error_message() gives detail for
+ *   the calling thread's most recent failed call.
+ *
+ * N == 0 (or B*H == 0) is valid and does nothing; the pointers are then not checked
+ * (empty tensors may have NULL data pointers).
+ */
+#ifndef FA_H
+#define FA_H
+
+#include <stddef.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,
+  FA_ERR_UNSUPPORTED = 2,
+  FA_ERR_CUDA = 3,
+  FA_ERR_TIMEOUT = 4
+} fa_status;
+
+/* Version of this ABI; bumped when a signature changes. */
+FA_API int fa_abi_version(void);
+
+/*
+ * Forward pass, bf16 in and out ("FlashAttention, simplified", "The trick").
+ *   Q, K, V  in : [B,H,N,d] bf16
+ *   O        out: [B,H,N,d] bf16; must not overlap Q, K or V
+ *   LSE      out: [B,H,N] float32 natural-log log-sum-exp per query row; may be NULL
+ *   d in {64, 128}; scale > 0 and finite (usually 1/sqrt(d)); causal in {0, 1}
+ * Kernel: persistent, one CTA per SM, tensor cores (tcgen05) with TMEM accumulators.
+ */
+FA_API fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                 int B, int H, int N, int d, float scale, int causal, cudaStream_t stream);
+
+/*
+ * Forward pass with float32 inputs and outputs, computed in float32 on the CUDA cores
+ * (same definition and arguments as fa_fwd).
+ */
+FA_API fa_status fa_fwd_f32(const float* Q, const float* K, const float* V, float* O, float* LSE,
+                     int B, int H, int N, int d, float scale, int causal,
+                     cudaStream_t stream);
+
+/*
+ * Bytes of scratch that fa_bwd needs for given sizes: one float32 per query row for
+ * D_i = sum_k dO_ik O_ik, rounded up to 256 bytes.  Grows as B*H*N, never as N^2.
+ */
+FA_API size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
+
+/*
+ * Backward pass, bf16 ("What FlashAttention actually buys", "Why the distinction
+ * matters downstream": the score tiles are recomputed from Q, K and the saved LSE).
+ *   Q, K, V, O, dO in : [B,H,N,d] bf16 (O is the forward output)
+ *   LSE            in : [B,H,N] float32 from fa_fwd with the same scale and causal
+ *   dQ, dK, dV     out: [B,H,N,d] bf16; must not overlap the inputs
+ *   workspace         : caller-owned device scratch of at least
+ *                       fa_bwd_workspace_bytes(B,H,N,d) bytes, 16-byte aligned; its
+ *                       contents on entry do not matter and are overwritten
+ * Three kernels on `stream`: D = rowsum(dO * O); dK and dV per key block; dQ per query
+ * block.  No atomics: the result is the same bits on every run.
+ */
+FA_API fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O,
+                 const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                 int B, int H, int N, int d, float scale, int causal,
+                 void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Static text for a status code ("FA_OK", ...). */
+FA_API const char* fa_status_string(fa_status status);
+
+/* Detail of the calling thread's last failed call (empty string if none). */
+FA_API const char* fa_last_error_message(void);
+
+/*
+ * Synchronises `stream`, then reports and clears the device-side error word that the
+ * kernels set when a pipeline wait exceeds its time limit (FA_ERR_TIMEOUT), or
+ * FA_ERR_CUDA if the stream itself reports an error.
+ */
+FA_API fa_status fa_check_device_error(cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H */

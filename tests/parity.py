@@ -1,0 +1,46 @@
+"""Comparison helpers for the parity tests (CUDA path vs the fp64 oracle)."""
+import numpy as np
+import torch
+
+# Tolerances of the bf16 path (bf16 in/out, fp32 accumulation) and the fp32 path.
+BF16_MAX_ABS = 2e-2
+BF16_REL_L2 = 5e-3
+F32_MAX_ABS = 1e-4
+# LSE is float32 from float32 scores; this bound is ours (nothing fixes one for it).
+LSE_MAX_ABS = 1e-3
+
+
+def to64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def errors(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.isfinite(got).all(), "non-finite values in the CUDA result"
+    diff = got - ref
+    max_abs = float(np.abs(diff).max()) if diff.size else 0.0
+    denom = float(np.linalg.norm(ref))
+    rel_l2 = float(np.linalg.norm(diff) / denom) if denom > 0 else float(np.linalg.norm(diff))
+    return max_abs, rel_l2
+
+
+def assert_bf16_close(got, ref, what=""):
+    max_abs, rel_l2 = errors(got, ref)
+    ref_max = float(np.abs(np.asarray(ref)).max()) if np.size(ref) else 0.0
+    assert max_abs <= BF16_MAX_ABS and rel_l2 <= BF16_REL_L2, (
+        f"{what}: max_abs={max_abs:.3e} rel_l2={rel_l2:.3e} (max |ref|={ref_max:.3g})")
+    return max_abs, rel_l2
+
+
+def assert_f32_close(got, ref, what=""):
+    max_abs, rel_l2 = errors(got, ref)
+    assert max_abs <= F32_MAX_ABS, f"{what}: max_abs={max_abs:.3e} rel_l2={rel_l2:.3e}"
+    return max_abs, rel_l2
+
+
+def assert_lse_close(got, ref, what=""):
+    max_abs, _ = errors(got, ref)
+    assert max_abs <= LSE_MAX_ABS, f"{what}: LSE max_abs={max_abs:.3e}"
+    return max_abs

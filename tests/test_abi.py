@@ -1,0 +1,126 @@
+"""The C ABI: the library loads, exports every function include/fa.h declares, and its
+host-side validation rejects bad arguments before touching a device (runs without a
+GPU: no call here reaches a kernel)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_io_aware_64_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    inc = os.path.join(ROOT, "include")
+    for fn in os.listdir(inc):
+        if not fn.endswith(".h"):
+            continue
+        text = open(os.path.join(inc, fn)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^[A-Za-z_][\w\s\*]*?\b(fa_\w+)\s*\(", text, flags=re.M):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return binding.lib()
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for required in ("fa_fwd", "fa_bwd", "fa_fwd_f32", "fa_bwd_workspace_bytes",
+                     "fa_status_string", "fa_check_device_error"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+    # the binding's signature table covers the same set
+    assert set(binding.SIGNATURES) == set(_declared_functions())
+
+
+def test_status_strings(lib):
+    assert binding.status_name(0) == "FA_OK"
+    assert binding.status_name(1) == "FA_ERR_INVALID_ARG"
+    assert binding.status_name(2) == "FA_ERR_UNSUPPORTED"
+    assert binding.status_name(3) == "FA_ERR_CUDA"
+    assert binding.status_name(4) == "FA_ERR_TIMEOUT"
+    assert lib.fa_abi_version() == 1
+
+
+def test_workspace_is_linear_in_rows(lib):
+    assert binding.workspace_bytes(2, 16, 8192, 128) == 2 * 16 * 8192 * 4
+    assert binding.workspace_bytes(1, 1, 1, 64) == 256          # rounded up to 256 bytes
+    assert binding.workspace_bytes(0, 4, 128, 64) == 0
+    # O(B*H*N), never O(N^2): the backward stores no score tile
+    assert binding.workspace_bytes(1, 1, 32768, 128) == 32768 * 4
+
+
+# Fake, 16-byte aligned addresses: validation must fail (or finish) before any use.
+A, B_, C, D_, E = 0x100000, 0x200000, 0x300000, 0x400000, 0x500000
+
+
+def _fwd(lib, q=A, k=B_, v=C, o=D_, lse=E, B=1, H=1, N=16, d=64, scale=0.125, causal=0):
+    st = lib.fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, None)
+    return st, lib.fa_last_error_message().decode()
+
+
+def test_fwd_validation(lib):
+    assert _fwd(lib, q=0)[0] == binding.FA_ERR_INVALID_ARG
+    assert _fwd(lib, o=0)[0] == binding.FA_ERR_INVALID_ARG
+    assert _fwd(lib, k=B_ + 8)[0] == binding.FA_ERR_INVALID_ARG      # misaligned
+    assert _fwd(lib, d=96)[0] == binding.FA_ERR_UNSUPPORTED
+    assert _fwd(lib, d=256)[0] == binding.FA_ERR_UNSUPPORTED
+    assert _fwd(lib, N=-1)[0] == binding.FA_ERR_INVALID_ARG
+    assert _fwd(lib, scale=0.0)[0] == binding.FA_ERR_INVALID_ARG
+    assert _fwd(lib, scale=float("nan"))[0] == binding.FA_ERR_INVALID_ARG
+    assert _fwd(lib, scale=float("inf"))[0] == binding.FA_ERR_INVALID_ARG
+    assert _fwd(lib, causal=2)[0] == binding.FA_ERR_INVALID_ARG
+    assert _fwd(lib, o=A + 16)[0] == binding.FA_ERR_INVALID_ARG       # O overlaps Q
+    assert _fwd(lib, lse=E + 2)[0] == binding.FA_ERR_INVALID_ARG      # LSE misaligned
+    st, msg = _fwd(lib, d=96)
+    assert "d=96" in msg
+    huge = _fwd(lib, B=1 << 15, H=1 << 15, N=1 << 12)
+    assert huge[0] == binding.FA_ERR_INVALID_ARG
+
+
+def test_empty_problems_are_noops(lib):
+    # N = 0 or B*H = 0: nothing to do, no device needed
+    assert _fwd(lib, N=0)[0] == binding.FA_OK
+    assert _fwd(lib, B=0)[0] == binding.FA_OK
+    assert lib.fa_fwd_f32(A, B_, C, D_, E, 1, 3, 0, 128, 0.1, 1, None) == binding.FA_OK
+
+
+def test_bwd_validation(lib):
+    F, G, H_, I, J = 0x600000, 0x700000, 0x800000, 0x900000, 0xA00000
+    args = [A, B_, C, D_, E, F, G, H_, I, 1, 2, 64, 128, 0.1, 1, J, 1 << 20, None]
+
+    def call(**kw):
+        a = list(args)
+        names = ["Q", "K", "V", "O", "dO", "LSE", "dQ", "dK", "dV", "B", "H", "N", "d",
+                 "scale", "causal", "ws", "ws_bytes", "stream"]
+        for k, v in kw.items():
+            a[names.index(k)] = v
+        return lib.fa_bwd(*a)
+
+    assert call(B=0) == binding.FA_OK                      # empty: no-op
+    assert lib.fa_fwd(0, 0, 0, 0, 0, 1, 1, 0, 64, 0.1, 0, None) == binding.FA_OK
+    assert call(LSE=0) == binding.FA_ERR_INVALID_ARG        # LSE required
+    assert call(ws=0) == binding.FA_ERR_INVALID_ARG
+    assert call(ws_bytes=100) == binding.FA_ERR_INVALID_ARG
+    assert call(d=80) == binding.FA_ERR_UNSUPPORTED
+    assert call(dQ=A) == binding.FA_ERR_INVALID_ARG         # gradient overlaps an input
+    assert call(dK=G) == binding.FA_ERR_INVALID_ARG         # gradients overlap
+    assert call(ws=H_) == binding.FA_ERR_INVALID_ARG        # workspace overlaps dK
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(binding, "_lib", None)
+    monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        binding.lib()
