@@ -130,17 +130,24 @@ def attention_head_tiled(Q, K, V, scale: float, causal: bool, block_q: int, bloc
     return O, LSE
 
 
-def attention_bwd_head(Q, K, V, dO, scale: float, causal: bool):
+def attention_bwd_head(Q, K, V, dO, scale: float, causal: bool, O_given=None):
     """Analytic gradients of O = softmax(scale Q K^T [masked]) V for one head.
 
     Returns (dQ, dK, dV, D) where D_i = sum_k dO_ik O_ik.  Masked entries have P = 0 and
     so contribute nothing to any gradient.
+
+    By default D uses the exact O.  A backward pass that is handed the forward's output
+    (as the recompute-based backward is) forms D from that stored O instead; pass it as
+    ``O_given`` to get exactly that computation.  With O_given equal to the exact O the
+    two agree.
     """
     Q = _f64(Q)
     K = _f64(K)
     V = _f64(V)
     dO = _f64(dO)
     O, _, P = attention_head(Q, K, V, scale, causal)
+    if O_given is not None:
+        O = _f64(O_given)
     dV = P.T @ dO
     dP = dO @ V.T
     D = (dO * O).sum(axis=1)

@@ -305,6 +305,25 @@ def pin_batched_backward(A):
                                                           V[b, h]), rtol=1e-6, atol=1e-8)
 
 
+def pin_backward_with_given_output(A):
+    """The stored-output variant: with the exact O it equals the default; with another
+    O it forms D from that O, and only dQ and dK move (dV = P^T dO does not use D)."""
+    rng = _rng(13)
+    N, d, scale = 6, 3, 0.9
+    Q, K, V, dO = (rng.standard_normal((N, d)) for _ in range(4))
+    for causal in (False, True):
+        base = A.attention_bwd_head(Q, K, V, dO, scale, causal)
+        O = A.attention_head(Q, K, V, scale, causal)[0]
+        same = A.attention_bwd_head(Q, K, V, dO, scale, causal, O_given=O)
+        for x, y in zip(base, same):
+            np.testing.assert_allclose(x, y, rtol=0, atol=1e-14)
+        Ob = O + 0.01 * rng.standard_normal(O.shape)
+        got = A.attention_bwd_head(Q, K, V, dO, scale, causal, O_given=Ob)
+        np.testing.assert_allclose(got[3], (dO * Ob).sum(1), rtol=0, atol=1e-14)
+        np.testing.assert_allclose(got[2], base[2], rtol=0, atol=1e-14)
+        assert np.abs(got[0] - base[0]).max() > 1e-6
+
+
 PINS = [
     pin_golden_forward,
     pin_golden_backward,
@@ -320,6 +339,7 @@ PINS = [
     pin_finite_differences,
     pin_dq_rows_finite_differences,
     pin_batched_backward,
+    pin_backward_with_given_output,
 ]
 
 
@@ -355,6 +375,7 @@ MUTANTS = [
     ("attention_bwd_head", "dQ = scale * (dS @ K)", "dQ = (dS @ K)"),
     ("attention_bwd_head", "dK = scale * (dS.T @ Q)", "dK = scale * (dS @ Q)"),
     ("attention_bwd_head", "dK = scale * (dS.T @ Q)", "dK = (dS.T @ Q)"),
+    ("attention_bwd_head", "        O = _f64(O_given)", "        O = O"),
     ("attention_bwd_dq_rows", "dQ = scale * (dS @ K)", "dQ = (dS @ K)"),
     ("attention_bwd_dq_rows", "D = (dO_rows * O).sum(axis=1)", "D = (dO_rows * dO_rows).sum(axis=1)"),
     ("attention_fwd", "O[b, h], LSE[b, h], _ = attention_head(Q[b, h], np.asarray(K)[b, h],",
