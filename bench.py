@@ -1,0 +1,390 @@
+"""Benchmark of the hot path: exact attention forward (fa_fwd) then backward (fa_bwd).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = fa_fwd + fa_bwd on one batch of synthetic inputs already resident in device
+memory (the default workload is B=2, H=16, N=8192, d=128, causal, bf16).  The value is
+credited TFLOP/s: forward 4*B*H*N^2*d plus backward 10*B*H*N^2*d, halved for causal, per
+second of device time, summed over ranks.  Under torchrun every rank runs the same
+workload on its own GPU (replicas of independent heads: weak scaling, no data-path
+collective); the time is the max over ranks.
+
+Rank 0 prints one JSON line.  Besides the contract keys it carries:
+  roofline      the dominant kernel's achieved TFLOP/s against the measured bf16 peak
+  cpu_baseline  the fp64 oracle timed on this host on a bounded sample (rank 0, N=1)
+  e2e           the same metric with host buffers: pinned host -> device copies of the
+                inputs, fa_fwd, fa_bwd and device -> host copies of the results, all
+                inside the timed region
+  clocks        SM clocks and throttle reasons sampled during the timed region
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from exact_io_aware_64_b200 import inputs as fa_inputs  # noqa: E402
+from exact_io_aware_64_b200 import traffic  # noqa: E402
+
+DEFAULT_WORKLOAD = "n8192_d128_causal_bwd"
+METRIC = "attention TFLOP/s (fwd, bwd) vs N and % of B200 dense BF16 peak, 1 GPU"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def library_digest() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "exact_io_aware_64_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    current kernel sources; otherwise None."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel)
+    if not e or e.get("source_digest") != library_digest():
+        return None
+    return e.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        self.file.flush()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.file.seek(0)
+        rows = [r.strip().split(", ") for r in self.file.read().strip().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        sm, smax, power, reasons = [], None, [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                smax = float(r[2])
+                power.append(float(r[3]))
+            except ValueError:
+                continue
+            for name, val in zip(names, r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(name)
+        loaded = [s for s, p in zip(sm, power) if p > 200.0] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def step_flops(w) -> float:
+    return traffic.fwd_flops(w.B, w.H, w.N, w.d, w.causal) + \
+        traffic.bwd_flops(w.B, w.H, w.N, w.d, w.causal)
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+def time_oracle(w, max_seconds: float = 20.0):
+    """The fp64 oracle, as it stands, on a bounded sample of the workload: the forward
+    and backward of whole heads (b, h) = (0, 0), (0, 1), ... until about max_seconds of
+    CPU work.  Returns (TFLOP/s credited, threads, sample description, seconds)."""
+    import numpy as np
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((i.get("num_threads", 1) for i in threadpool_info()
+                       if i.get("user_api") == "blas"), default=1)
+    except Exception:
+        threads = os.cpu_count() or 1
+    ins = fa_inputs.make_inputs(1, 1, w.N, w.d, w.seed, sigma_qk=w.sigma_qk,
+                                sigma_v=w.sigma_v, with_dO=True)
+    Q, K, V, dO = (ins[n][0, 0].double().numpy() for n in ("Q", "K", "V", "dO"))
+    heads = 0
+    t0 = time.perf_counter()
+    while True:
+        oracle.attention_head(Q, K, V, w.scale, w.causal)
+        oracle.attention_bwd_head(Q, K, V, dO, w.scale, w.causal)
+        heads += 1
+        el = time.perf_counter() - t0
+        if el > max_seconds / 2 or heads >= 4:
+            break
+    flops = heads * (traffic.fwd_flops(1, 1, w.N, w.d, w.causal) +
+                     traffic.bwd_flops(1, 1, w.N, w.d, w.causal))
+    sample = (f"fp64 oracle forward+backward of {heads} whole head(s) of the workload "
+              f"(N={w.N}, d={w.d}, causal={w.causal}); credited FLOPs per second")
+    return flops / el / 1e12, int(threads), sample, el
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    per_step = []
+    value = threads = sample = None
+    for i in range(args.warmup + args.steps):
+        v, threads, sample, el = time_oracle(w, max_seconds=args.ref_seconds)
+        if i >= args.warmup:
+            per_step.append((v, el))
+    value = statistics.median(v for v, _ in per_step)
+    ms = statistics.median(el for _, el in per_step) * 1e3
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                   "causal": w.causal, "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_gpu(args, w):
+    from exact_io_aware_64_b200 import binding
+    rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    B, H, N, d = w.B, w.H, w.N, w.d
+    with_bwd = not args.fwd_only
+    ins = fa_inputs.make_inputs(B, H, N, d, w.seed + 101 * rank, sigma_qk=w.sigma_qk,
+                                sigma_v=w.sigma_v, with_dO=True, device=str(dev))
+    q, k, v, do = ins["Q"], ins["K"], ins["V"], ins["dO"]
+    O = torch.empty_like(q)
+    LSE = torch.empty((B, H, N), device=dev, dtype=torch.float32)
+    dQ, dK, dV = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(max(binding.workspace_bytes(B, H, N, d), 1), device=dev,
+                     dtype=torch.uint8)
+    stream = torch.cuda.current_stream(dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    def step(marks=None):
+        if marks is not None:
+            marks[0].record(stream)
+        binding.fwd(q, k, v, scale=w.scale, causal=w.causal, O=O, LSE=LSE)
+        if marks is not None:
+            marks[1].record(stream)
+        if with_bwd:
+            binding.bwd(q, k, v, O, do, LSE, scale=w.scale, causal=w.causal, dQ=dQ, dK=dK,
+                        dV=dV, workspace=ws)
+        if marks is not None:
+            marks[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    binding.check_device_error()
+    marks = [[ev(), ev(), ev()] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        start, end = ev(), ev()
+        start.record(stream)
+        for i in range(args.steps):
+            step(marks[i])
+        end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    binding.check_device_error()
+    ms_local = start.elapsed_time(end) / args.steps
+    ms = max_over_ranks(ms_local, world)
+    fwd_ms = statistics.mean(m[0].elapsed_time(m[1]) for m in marks)
+    bwd_ms = statistics.mean(m[1].elapsed_time(m[2]) for m in marks) if with_bwd else 0.0
+    f_fwd = traffic.fwd_flops(B, H, N, d, w.causal)
+    f_bwd = traffic.bwd_flops(B, H, N, d, w.causal) if with_bwd else 0.0
+    value = world * (f_fwd + f_bwd) / (ms * 1e-3) / 1e12
+
+    # ---- end to end through the public API with host buffers
+    pin = lambda t: t.detach().to("cpu").pin_memory()  # noqa: E731
+    hq, hk, hv, hdo = pin(q), pin(k), pin(v), pin(do)
+    hO = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
+    hL = torch.empty(LSE.shape, dtype=LSE.dtype, pin_memory=True)
+    hdQ, hdK, hdV = (torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for _ in range(3))
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
+    outs = [(O, hO), (LSE, hL)] + ([(dQ, hdQ), (dK, hdK), (dV, hdV)] if with_bwd else [])
+    d2h = sum(dt.numel() * dt.element_size() for dt, _ in outs)
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        do.copy_(hdo, non_blocking=True)
+        step()
+        for dt, ht in outs:
+            ht.copy_(dt, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = ev(), ev()
+    e0.record(stream)
+    e2e_steps = max(2, min(args.steps, 10))
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+    e2e_value = world * (f_fwd + f_bwd) / (e2e_ms * 1e-3) / 1e12
+
+    if rank != 0:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return 0
+
+    peaks, peak_src = load_peaks()
+    # dominant kernel: the forward kernel or the backward call, whichever takes longer
+    if with_bwd and bwd_ms > fwd_ms:
+        dom_name, dom_ms, dom_flops = "fa_bwd (3 kernels)", bwd_ms, f_bwd
+        dom_key = "bwd"
+    else:
+        dom_name, dom_ms, dom_flops = "fwd_sm100_kernel", fwd_ms, f_fwd
+        dom_key = "fwd_sm100_kernel"
+    peak = peaks.get("bf16_tflops_sustained" if args.sustained_peak else "bf16_tflops")
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": B, "H": H, "N": N, "d": d, "causal": w.causal,
+                   "step": "fa_fwd + fa_bwd" if with_bwd else "fa_fwd",
+                   "l2": "inputs larger than L2 (no flush)",
+                   "parallelism": f"replicas x{world} (independent heads per GPU)"},
+        "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+        "fwd_tflops": f_fwd / (fwd_ms * 1e-3) / 1e12,
+        "bwd_tflops": (f_bwd / (bwd_ms * 1e-3) / 1e12) if with_bwd else None,
+        "roofline": {"kernel": dom_name, "bound": "tensor", "achieved": achieved,
+                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": f"{peak_src} "
+                                    f"{'sustained' if args.sustained_peak else 'burst'} bf16",
+                     "traffic": recorded_traffic(dom_key)},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": args.steps * (1 + (3 if with_bwd else 0)),
+        "clocks": clocks.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        v_cpu, threads, sample, _ = time_oracle(w, max_seconds=args.ref_seconds)
+        line["cpu_baseline"] = {"value": v_cpu, "unit": "TFLOP/s", "cores": threads,
+                                "kind": "oracle", "sample": sample}
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(fa_inputs.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--fwd-only", action="store_true")
+    ap.add_argument("--sustained-peak", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-seconds", type=float, default=20.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    w = fa_inputs.WORKLOADS[args.workload]
+    if w.dtype != "bf16":
+        ap.error("the benchmark runs the bf16 path")
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,15 +1,770 @@
-// bwd_sm100.cu -- backward attention (under construction: row statistic D only).
+// bwd_sm100.cu -- backward attention on the sm_100a tensor cores.
+//
+// Method ("What FlashAttention actually buys", "Why the distinction matters downstream":
+// the backward recomputes score tiles instead of storing the N x N matrix).  With the
+// forward's per-row log-sum-exp L, every probability tile is rebuilt on chip as
+// P = exp(scale Q K^T - L); the gradients are the textbook ones
+//     dV = P^T dO,  dP = dO V^T,  D_i = sum_k dO_ik O_ik,  dS = P * (dP - D),
+//     dQ = scale dS K,  dK = scale dS^T Q.
+//
+// Three kernels, no atomics (bitwise reproducible):
+//   1. bwd_prep: D = rowsum(dO * O) and L2 = L * log2(e), both stored padded to whole
+//      128-row tiles in the caller's workspace (rows past N: D = 0, L2 = +inf, so their
+//      probabilities are exactly 0) so that TMA can stream them.
+//   2. bwd_dkdv: one work unit per (batch*head, 128-row key tile j).  K_j and V_j stay in
+//      shared memory while the query tiles i stream past; the tile products are taken
+//      transposed so that the key row is the TMEM lane:
+//          S^T = K_j Q_i^T,  dP^T = V_j dO_i^T             (SS MMAs into TMEM)
+//          P^T = exp2(S^T * scale*log2e - L2_i)            (one thread per key row)
+//          dS^T = P^T * (dP^T - D_i)
+//          dV_j += P^T dO_i,  dK_j += dS^T Q_i             (TS MMAs, P^T/dS^T from TMEM)
+//      TMEM: dV | dK | S^T (P^T over its first 64 columns) | dP^T (dS^T likewise).
+//   3. bwd_dq: one work unit per (batch*head, 128-row query tile i); key/value tiles
+//      stream past:  S = Q_i K_j^T, dP = dO_i V_j^T, P, dS as above, dQ_i += dS K_j.
+//      TMEM: dQ | S | dP (dS over its first 64 columns).
+//
+// Both tensor-core kernels are persistent (one CTA per SM) with 256 threads: warps 0-3
+// are the element-wise warps (thread = TMEM lane = tile row; up to 255 registers, so a
+// whole 128-entry probability row stays in registers), warp 4 issues TMA loads, warp 5
+// issues the MMAs from one thread, warps 6-7 are idle.  The MMA order is chosen so the
+// tensor core works on one product while the element-wise warps build the next operand
+// (dK/dV: S^T(i) dP^T(i) | dV(i) S^T(i+1) | dK(i) dP^T(i+1) | ...;
+//  dQ: S(j) dP(j) | S(j+1) | dQ(j) dP(j+1) | S(j+2) | ...).
+// Causal work units are ordered heaviest first.
 #include <cstdint>
 
 #include "internal.h"
 #include "sm100.cuh"
 
 namespace fa {
+namespace {
 
-cudaError_t launch_bwd_sm100(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                             const CUtensorMap&, const void*, const void*, const float*, void*,
-                             void*, void*, float*, const Problem&, int, cudaStream_t) {
-  return cudaErrorNotSupported;
+using namespace sm100;
+
+constexpr int kTile = 128;        // rows per query / key tile
+constexpr int kThreads = 256;
+constexpr int kWarpTMA = 4;
+constexpr int kWarpMMA = 5;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kLog2e = 1.4426950408889634f;
+
+__host__ __device__ constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+// ------------------------------------------------------------------ 1. preparation
+// D[bh][r] = sum_k dO[bh][r][k] * O[bh][r][k];  L2[bh][r] = LSE[bh][r] * log2(e).
+// Padded rows r in [N, Npad): D = 0, L2 = +inf.  One warp per row, 16-byte loads.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __restrict__ O,
+                                                       const __nv_bfloat16* __restrict__ dO,
+                                                       const float* __restrict__ LSE,
+                                                       float* __restrict__ Dout,
+                                                       float* __restrict__ L2out, int BH,
+                                                       int N, int Npad) {
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (row >= static_cast<long long>(BH) * Npad) return;
+  const int bh = static_cast<int>(row / Npad);
+  const int r = static_cast<int>(row % Npad);
+  float acc = 0.f;
+  if (r < N) {
+    const size_t base = (static_cast<size_t>(bh) * N + r) * D;
+    constexpr int kVec = 8;  // bf16 per 16-byte load
+    for (int c = lane * kVec; c < D; c += 32 * kVec) {
+      const uint4 a = *reinterpret_cast<const uint4*>(O + base + c);
+      const uint4 b = *reinterpret_cast<const uint4*>(dO + base + c);
+      const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
+      const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 fa = __bfloat1622float2(pa[k]);
+        const float2 fb = __bfloat1622float2(pb[k]);
+        acc = fmaf(fa.x, fb.x, acc);
+        acc = fmaf(fa.y, fb.y, acc);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  }
+  if (lane == 0) {
+    const size_t out = static_cast<size_t>(bh) * Npad + r;
+    Dout[out] = acc;
+    L2out[out] = r < N ? LSE[static_cast<size_t>(bh) * N + r] * kLog2e : INFINITY;
+  }
+}
+
+struct BwdArgs {
+  unsigned int* err;
+  __nv_bfloat16* dQ;
+  __nv_bfloat16* dK;
+  __nv_bfloat16* dV;
+  const float* Dpad;   // [BH][Npad]
+  const float* L2pad;  // [BH][Npad]
+  int BH;
+  int N;
+  int Npad;
+  int n_tiles;      // ceil(N / 128)
+  int total_units;  // BH * n_tiles
+  int causal;
+  float scale;
+  float scale_log2;
+};
+
+// Convert 32 fp32 accumulator columns (times `mul`) to bf16 and store them to a row.
+__device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t* v, float mul) {
+  uint32_t pk[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k)
+    pk[k] = pack_bf16x2(__uint_as_float(v[2 * k]) * mul, __uint_as_float(v[2 * k + 1]) * mul);
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) d[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+}
+
+// ------------------------------------------------------------------ 2. dK, dV
+template <int D>
+struct DkdvLayout {
+  static constexpr int kTileBytes = kTile * D * 2;
+  static constexpr int kBoxBytes = 128 * 128;
+  static constexpr int kStages = 2;
+  static constexpr int kK = 0;
+  static constexpr int kV = kTileBytes;
+  static constexpr int kStage0 = 2 * kTileBytes;
+  // per stage: Q tile, dO tile, L2 row (512 B), D row (512 B)
+  static constexpr int kStageQ = 0;
+  static constexpr int kStageDO = kTileBytes;
+  static constexpr int kStageL = 2 * kTileBytes;
+  static constexpr int kStageD = 2 * kTileBytes + 512;
+  static constexpr int kStageBytes = 2 * kTileBytes + 1024;
+  static constexpr int kBar = kStage0 + kStages * kStageBytes;
+  static constexpr int kBarKVFull = 0, kBarKVEmpty = 1;
+  static constexpr int kBarQFull = 2;                 // [kStages]
+  static constexpr int kBarQEmpty = 2 + kStages;      // [kStages]
+  static constexpr int kBarSFull = 2 + 2 * kStages;
+  static constexpr int kBarDPFull = 3 + 2 * kStages;
+  static constexpr int kBarPReady = 4 + 2 * kStages;
+  static constexpr int kBarDSReady = 5 + 2 * kStages;
+  static constexpr int kBarAccFull = 6 + 2 * kStages;
+  static constexpr int kBarAccFree = 7 + 2 * kStages;
+  static constexpr int kBarDrain = 8 + 2 * kStages;
+  static constexpr int kNumBars = 9 + 2 * kStages;
+  static constexpr int kMisc = kBar + kNumBars * 8;
+  static constexpr int kAlloc = kMisc + 16 + 1024;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                    const __grid_constant__ CUtensorMap tmL2, const __grid_constant__ CUtensorMap tmD,
+                    const BwdArgs args) {
+  using L = DkdvLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base = (raw_addr + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw_addr);
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  auto bar = [&](int i) -> uint32_t { return base + L::kBar + 8 * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  auto wait = [&](uint32_t b, uint32_t parity) -> bool {
+    return mbar_wait(b, parity, abort_flag, args.err);
+  };
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(bar(L::kBarKVFull), 1);
+    mbar_init(bar(L::kBarKVEmpty), 1);
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(bar(L::kBarQFull + s), 1);
+      mbar_init(bar(L::kBarQEmpty + s), 1 + kTile);  // MMA commit + element-wise threads
+    }
+    mbar_init(bar(L::kBarSFull), 1);
+    mbar_init(bar(L::kBarDPFull), 1);
+    mbar_init(bar(L::kBarPReady), kTile);
+    mbar_init(bar(L::kBarDSReady), kTile);
+    mbar_init(bar(L::kBarAccFull), 1);
+    mbar_init(bar(L::kBarAccFree), kTile);
+    mbar_init(bar(L::kBarDrain), 1);
+    fence_mbar_init();
+  }
+  if (warp == kWarpMMA) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tdV = tmem, tdK = tmem + D, tS = tmem + 2 * D, tdP = tmem + 2 * D + 128;
+
+  auto unit = [&](int w, int& bh, int& j, int& i0) {
+    if (args.causal) {
+      j = w / args.BH;  // key tile 0 meets every query tile: heaviest first
+      bh = w % args.BH;
+      i0 = j;
+    } else {
+      bh = w / args.n_tiles;
+      j = w % args.n_tiles;
+      i0 = 0;
+    }
+  };
+
+  if (warp == kWarpTMA) {
+    if (lane == 0) {
+      int stage = 0, units = 0, kv_loads = 0;
+      uint32_t phase = 0;
+      int issued[L::kStages] = {};
+      uint32_t issued_phase[L::kStages] = {};
+      bool ok = true;
+      for (int w = blockIdx.x; ok && w < args.total_units; w += gridDim.x, ++units) {
+        int bh, j, i0;
+        unit(w, bh, j, i0);
+        if (units > 0) ok = wait(bar(L::kBarKVEmpty), (units - 1) & 1);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar(L::kBarKVFull), 2 * L::kTileBytes);
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_3d(base + L::kK + c * L::kBoxBytes, &tmK, bar(L::kBarKVFull), c * 64, j * kTile, bh);
+          tma_load_3d(base + L::kV + c * L::kBoxBytes, &tmV, bar(L::kBarKVFull), c * 64, j * kTile, bh);
+        }
+        ++kv_loads;
+        for (int i = i0; ok && i < args.n_tiles; ++i) {
+          ok = wait(bar(L::kBarQEmpty + stage), phase ^ 1);
+          if (!ok) break;
+          const uint32_t fb = bar(L::kBarQFull + stage);
+          const uint32_t sb = base + L::kStage0 + stage * L::kStageBytes;
+          mbar_arrive_expect_tx(fb, 2 * L::kTileBytes + 1024);
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_3d(sb + L::kStageQ + c * L::kBoxBytes, &tmQ, fb, c * 64, i * kTile, bh);
+            tma_load_3d(sb + L::kStageDO + c * L::kBoxBytes, &tmdO, fb, c * 64, i * kTile, bh);
+          }
+          tma_load_3d(sb + L::kStageL, &tmL2, fb, i * kTile, bh, 0);
+          tma_load_3d(sb + L::kStageD, &tmD, fb, i * kTile, bh, 0);
+          issued[stage] = 1;
+          issued_phase[stage] = phase;
+          if (++stage == L::kStages) stage = 0, phase ^= 1;
+        }
+      }
+      if (!ok) {
+        // let the loads already issued land before the CTA exits
+        for (int s = 0; s < L::kStages; ++s)
+          if (issued[s]) mbar_wait_drain(bar(L::kBarQFull + s), issued_phase[s], args.err);
+        if (kv_loads > 0) mbar_wait_drain(bar(L::kBarKVFull), (kv_loads - 1) & 1, args.err);
+      }
+    }
+  } else if (warp == kWarpMMA) {
+    if (lane == 0) {
+      constexpr uint32_t idSS = idesc_bf16_f32(kTile, false);
+      constexpr uint32_t idTS = idesc_bf16_f32(D, true);
+      const uint64_t dK0 = desc_kmajor(base + L::kK);
+      const uint64_t dV0 = desc_kmajor(base + L::kV);
+      int stage = 0, units = 0, p_cnt = 0, ds_cnt = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      auto stage_base = [&](int s) { return base + L::kStage0 + s * L::kStageBytes; };
+      // S^T = K Q^T or dP^T = V dO^T: both operands K-major, K extent = D
+      auto issue_ss = [&](uint32_t dtm, uint64_t da, uint32_t b_saddr, uint32_t done_bar) {
+        const uint64_t db = desc_kmajor(b_saddr);
+#pragma unroll 1
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk / 4) * L::kBoxBytes + (kk % 4) * 32) >> 4;
+          mma_ss(dtm, da + off, db + off, idSS, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(done_bar);
+      };
+      // acc += A(TMEM, 128 x 128 bf16) * B(smem tile, 128 rows x D, MN-major)
+      auto issue_ts = [&](uint32_t acc, uint32_t a_tmem, uint32_t b_saddr, bool accumulate) {
+        const uint64_t db = desc_mnmajor(b_saddr, L::kBoxBytes);
+#pragma unroll 1
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          mma_ts(acc, a_tmem + kk * 8, db + static_cast<uint64_t>((kk * 2048) >> 4), idTS,
+                 (accumulate || kk > 0) ? 1u : 0u);
+      };
+      for (int w = blockIdx.x; ok && w < args.total_units; w += gridDim.x, ++units) {
+        int bh, j, i0;
+        unit(w, bh, j, i0);
+        const int m = args.n_tiles - i0;
+        ok = wait(bar(L::kBarKVFull), units & 1);
+        if (ok) ok = wait(bar(L::kBarQFull + stage), phase);
+        if (!ok) break;
+        tc_fence_after();
+        int cur = stage;
+        if (++stage == L::kStages) stage = 0, phase ^= 1;
+        issue_ss(tS, dK0, stage_base(cur) + L::kStageQ, bar(L::kBarSFull));
+        issue_ss(tdP, dV0, stage_base(cur) + L::kStageDO, bar(L::kBarDPFull));
+        for (int t = 0; t < m; ++t) {
+          ok = wait(bar(L::kBarPReady), p_cnt & 1);
+          if (ok && t == 0 && units > 0) ok = wait(bar(L::kBarAccFree), (units - 1) & 1);
+          if (!ok) break;
+          ++p_cnt;
+          tc_fence_after();
+          issue_ts(tdV, tS, stage_base(cur) + L::kStageDO, t > 0);  // dV += P^T dO
+          int nxt = -1;
+          if (t + 1 < m) {
+            ok = wait(bar(L::kBarQFull + stage), phase);
+            if (!ok) break;
+            nxt = stage;
+            if (++stage == L::kStages) stage = 0, phase ^= 1;
+            tc_fence_after();
+            issue_ss(tS, dK0, stage_base(nxt) + L::kStageQ, bar(L::kBarSFull));
+          }
+          ok = wait(bar(L::kBarDSReady), ds_cnt & 1);
+          if (!ok) break;
+          ++ds_cnt;
+          tc_fence_after();
+          issue_ts(tdK, tdP, stage_base(cur) + L::kStageQ, t > 0);  // dK += dS^T Q
+          mma_commit(bar(L::kBarQEmpty + cur));
+          if (nxt >= 0) {
+            issue_ss(tdP, dV0, stage_base(nxt) + L::kStageDO, bar(L::kBarDPFull));
+            cur = nxt;
+          }
+        }
+        if (!ok) break;
+        mma_commit(bar(L::kBarKVEmpty));
+        mma_commit(bar(L::kBarAccFull));
+      }
+      mma_commit(bar(L::kBarDrain));
+      mbar_wait_drain(bar(L::kBarDrain), 0, args.err);
+    }
+  } else if (warp < 4) {
+    const int row = warp * 32 + lane;  // key row within the tile = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    int stage = 0, units = 0, s_cnt = 0, dp_cnt = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; ok && w < args.total_units; w += gridDim.x, ++units) {
+      int bh, j, i0;
+      unit(w, bh, j, i0);
+      for (int i = i0; i < args.n_tiles; ++i) {
+        const uint8_t* sb = smem + L::kStage0 + stage * L::kStageBytes;
+        const float* sL = reinterpret_cast<const float*>(sb + L::kStageL);
+        const float* sD = reinterpret_cast<const float*>(sb + L::kStageD);
+        ok = wait(bar(L::kBarQFull + stage), phase);
+        if (ok) ok = wait(bar(L::kBarSFull), s_cnt & 1);
+        if (!ok) break;
+        ++s_cnt;
+        tc_fence_after();
+        float p[kTile];
+        {
+          uint32_t r[kTile];
+#pragma unroll
+          for (int c = 0; c < kTile / 32; ++c) tmem_ld32(tS + lane_off + c * 32, &r[c * 32]);
+          tmem_wait_ld();
+          const bool diag = args.causal && i == j;
+#pragma unroll
+          for (int c = 0; c < kTile; ++c) {
+            float e = ex2_approx(fmaf(__uint_as_float(r[c]), args.scale_log2, -sL[c]));
+            if (diag && c < row) e = 0.f;  // query i*128+c before key j*128+row
+            p[c] = e;
+          }
+        }
+        {
+          uint32_t pk[kTile / 2];
+#pragma unroll
+          for (int c = 0; c < kTile / 2; ++c) pk[c] = pack_bf16x2(p[2 * c], p[2 * c + 1]);
+          tmem_st32(tS + lane_off, &pk[0]);
+          tmem_st32(tS + lane_off + 32, &pk[32]);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(L::kBarPReady));
+        ok = wait(bar(L::kBarDPFull), dp_cnt & 1);
+        if (!ok) break;
+        ++dp_cnt;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < kTile / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tdP + lane_off + c * 32, r);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const int c0 = c * 32 + 2 * k;
+            const float ds0 = p[c0] * (__uint_as_float(r[2 * k]) - sD[c0]);
+            const float ds1 = p[c0 + 1] * (__uint_as_float(r[2 * k + 1]) - sD[c0 + 1]);
+            pk[k] = pack_bf16x2(ds0, ds1);
+          }
+          tmem_st16(tdP + lane_off + c * 16, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(L::kBarDSReady));
+        mbar_arrive(bar(L::kBarQEmpty + stage));  // done with this stage's L2 and D rows
+        if (++stage == L::kStages) stage = 0, phase ^= 1;
+      }
+      if (!ok) break;
+      // epilogue: dV and scale * dK for this key row
+      ok = wait(bar(L::kBarAccFull), units & 1);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const int kv_row = j * kTile + row;
+      const size_t off = (static_cast<size_t>(bh) * args.N + kv_row) * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tdV + lane_off + c * 32, v);
+        tmem_wait_ld();
+        if (kv_row < args.N) store_row32(args.dV + off + c * 32, v, 1.f);
+        tmem_ld32(tdK + lane_off + c * 32, v);
+        tmem_wait_ld();
+        if (kv_row < args.N) store_row32(args.dK + off + c * 32, v, args.scale);
+      }
+      tc_fence_before();
+      mbar_arrive(bar(L::kBarAccFree));
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMMA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ 3. dQ
+template <int D>
+struct DqLayout {
+  static constexpr int kTileBytes = kTile * D * 2;
+  static constexpr int kBoxBytes = 128 * 128;
+  static constexpr int kStages = 2;
+  static constexpr int kQ = 0;
+  static constexpr int kDO = kTileBytes;
+  static constexpr int kStage0 = 2 * kTileBytes;
+  static constexpr int kStageK = 0;
+  static constexpr int kStageV = kTileBytes;
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kBar = kStage0 + kStages * kStageBytes;
+  static constexpr int kBarQFull = 0, kBarQEmpty = 1;
+  static constexpr int kBarKVFull = 2;              // [kStages]
+  static constexpr int kBarKVEmpty = 2 + kStages;   // [kStages]
+  static constexpr int kBarSFull = 2 + 2 * kStages;
+  static constexpr int kBarSFree = 3 + 2 * kStages;
+  static constexpr int kBarDPFull = 4 + 2 * kStages;
+  static constexpr int kBarDSReady = 5 + 2 * kStages;
+  static constexpr int kBarAccFull = 6 + 2 * kStages;
+  static constexpr int kBarAccFree = 7 + 2 * kStages;
+  static constexpr int kBarDrain = 8 + 2 * kStages;
+  static constexpr int kNumBars = 9 + 2 * kStages;
+  static constexpr int kMisc = kBar + kNumBars * 8;
+  static constexpr int kAlloc = kMisc + 16 + 1024;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                  const BwdArgs args) {
+  using L = DqLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base = (raw_addr + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw_addr);
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  auto bar = [&](int i) -> uint32_t { return base + L::kBar + 8 * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  auto wait = [&](uint32_t b, uint32_t parity) -> bool {
+    return mbar_wait(b, parity, abort_flag, args.err);
+  };
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(bar(L::kBarQFull), 1);
+    mbar_init(bar(L::kBarQEmpty), 1);
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(bar(L::kBarKVFull + s), 1);
+      mbar_init(bar(L::kBarKVEmpty + s), 1);
+    }
+    mbar_init(bar(L::kBarSFull), 1);
+    mbar_init(bar(L::kBarSFree), kTile);
+    mbar_init(bar(L::kBarDPFull), 1);
+    mbar_init(bar(L::kBarDSReady), kTile);
+    mbar_init(bar(L::kBarAccFull), 1);
+    mbar_init(bar(L::kBarAccFree), kTile);
+    mbar_init(bar(L::kBarDrain), 1);
+    fence_mbar_init();
+  }
+  if (warp == kWarpMMA) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tdQ = tmem, tS = tmem + 128, tdP = tmem + 256;
+
+  auto unit = [&](int w, int& bh, int& i, int& m) {
+    if (args.causal) {
+      i = args.n_tiles - 1 - w / args.BH;  // last query tile meets every key tile
+      bh = w % args.BH;
+      m = i + 1;
+    } else {
+      bh = w / args.n_tiles;
+      i = w % args.n_tiles;
+      m = args.n_tiles;
+    }
+  };
+
+  if (warp == kWarpTMA) {
+    if (lane == 0) {
+      int stage = 0, units = 0, q_loads = 0;
+      uint32_t phase = 0;
+      int issued[L::kStages] = {};
+      uint32_t issued_phase[L::kStages] = {};
+      bool ok = true;
+      for (int w = blockIdx.x; ok && w < args.total_units; w += gridDim.x, ++units) {
+        int bh, i, m;
+        unit(w, bh, i, m);
+        if (units > 0) ok = wait(bar(L::kBarQEmpty), (units - 1) & 1);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar(L::kBarQFull), 2 * L::kTileBytes);
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_3d(base + L::kQ + c * L::kBoxBytes, &tmQ, bar(L::kBarQFull), c * 64, i * kTile, bh);
+          tma_load_3d(base + L::kDO + c * L::kBoxBytes, &tmdO, bar(L::kBarQFull), c * 64, i * kTile, bh);
+        }
+        ++q_loads;
+        for (int j = 0; ok && j < m; ++j) {
+          ok = wait(bar(L::kBarKVEmpty + stage), phase ^ 1);
+          if (!ok) break;
+          const uint32_t fb = bar(L::kBarKVFull + stage);
+          const uint32_t sb = base + L::kStage0 + stage * L::kStageBytes;
+          mbar_arrive_expect_tx(fb, 2 * L::kTileBytes);
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_3d(sb + L::kStageK + c * L::kBoxBytes, &tmK, fb, c * 64, j * kTile, bh);
+            tma_load_3d(sb + L::kStageV + c * L::kBoxBytes, &tmV, fb, c * 64, j * kTile, bh);
+          }
+          issued[stage] = 1;
+          issued_phase[stage] = phase;
+          if (++stage == L::kStages) stage = 0, phase ^= 1;
+        }
+      }
+      if (!ok) {
+        for (int s = 0; s < L::kStages; ++s)
+          if (issued[s]) mbar_wait_drain(bar(L::kBarKVFull + s), issued_phase[s], args.err);
+        if (q_loads > 0) mbar_wait_drain(bar(L::kBarQFull), (q_loads - 1) & 1, args.err);
+      }
+    }
+  } else if (warp == kWarpMMA) {
+    if (lane == 0) {
+      constexpr uint32_t idSS = idesc_bf16_f32(kTile, false);
+      constexpr uint32_t idTS = idesc_bf16_f32(D, true);
+      const uint64_t dQd = desc_kmajor(base + L::kQ);
+      const uint64_t ddO = desc_kmajor(base + L::kDO);
+      int stage = 0, units = 0, sfree_cnt = 0, ds_cnt = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      auto stage_base = [&](int s) { return base + L::kStage0 + s * L::kStageBytes; };
+      auto issue_ss = [&](uint32_t dtm, uint64_t da, uint32_t b_saddr, uint32_t done_bar) {
+        const uint64_t db = desc_kmajor(b_saddr);
+#pragma unroll 1
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk / 4) * L::kBoxBytes + (kk % 4) * 32) >> 4;
+          mma_ss(dtm, da + off, db + off, idSS, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(done_bar);
+      };
+      for (int w = blockIdx.x; ok && w < args.total_units; w += gridDim.x, ++units) {
+        int bh, i, m;
+        unit(w, bh, i, m);
+        ok = wait(bar(L::kBarQFull), units & 1);
+        if (ok) ok = wait(bar(L::kBarKVFull + stage), phase);
+        if (!ok) break;
+        tc_fence_after();
+        int cur = stage;
+        if (++stage == L::kStages) stage = 0, phase ^= 1;
+        issue_ss(tS, dQd, stage_base(cur) + L::kStageK, bar(L::kBarSFull));
+        issue_ss(tdP, ddO, stage_base(cur) + L::kStageV, bar(L::kBarDPFull));
+        for (int t = 0; t < m; ++t) {
+          int nxt = -1;
+          if (t + 1 < m) {
+            ok = wait(bar(L::kBarKVFull + stage), phase);
+            if (ok) ok = wait(bar(L::kBarSFree), sfree_cnt & 1);
+            if (!ok) break;
+            ++sfree_cnt;
+            nxt = stage;
+            if (++stage == L::kStages) stage = 0, phase ^= 1;
+            tc_fence_after();
+            issue_ss(tS, dQd, stage_base(nxt) + L::kStageK, bar(L::kBarSFull));
+          }
+          ok = wait(bar(L::kBarDSReady), ds_cnt & 1);
+          if (ok && t == 0 && units > 0) ok = wait(bar(L::kBarAccFree), (units - 1) & 1);
+          if (!ok) break;
+          ++ds_cnt;
+          tc_fence_after();
+          // dQ += dS K_j: A = dS (TMEM), B = K_j (128 key rows x D, MN-major)
+          const uint64_t db = desc_mnmajor(stage_base(cur) + L::kStageK, L::kBoxBytes);
+#pragma unroll 1
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            mma_ts(tdQ, tdP + kk * 8, db + static_cast<uint64_t>((kk * 2048) >> 4), idTS,
+                   (t > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar(L::kBarKVEmpty + cur));
+          if (nxt >= 0) {
+            issue_ss(tdP, ddO, stage_base(nxt) + L::kStageV, bar(L::kBarDPFull));
+            cur = nxt;
+          }
+        }
+        if (!ok) break;
+        // the last unit's S tile was read by the element-wise warps: consume that signal
+        ok = wait(bar(L::kBarSFree), sfree_cnt & 1);
+        if (!ok) break;
+        ++sfree_cnt;
+        mma_commit(bar(L::kBarQEmpty));
+        mma_commit(bar(L::kBarAccFull));
+      }
+      mma_commit(bar(L::kBarDrain));
+      mbar_wait_drain(bar(L::kBarDrain), 0, args.err);
+    }
+  } else if (warp < 4) {
+    const int row = warp * 32 + lane;  // query row within the tile = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    int units = 0, s_cnt = 0, dp_cnt = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; ok && w < args.total_units; w += gridDim.x, ++units) {
+      int bh, i, m;
+      unit(w, bh, i, m);
+      const int q_row = i * kTile + row;
+      const size_t prow = static_cast<size_t>(bh) * args.Npad + q_row;  // q_row < Npad
+      const float l2 = args.L2pad[prow];
+      const float drow = args.Dpad[prow];
+      for (int j = 0; j < m; ++j) {
+        ok = wait(bar(L::kBarSFull), s_cnt & 1);
+        if (!ok) break;
+        ++s_cnt;
+        tc_fence_after();
+        float p[kTile];
+        {
+          uint32_t r[kTile];
+#pragma unroll
+          for (int c = 0; c < kTile / 32; ++c) tmem_ld32(tS + lane_off + c * 32, &r[c * 32]);
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(bar(L::kBarSFree));
+          const int kv0 = j * kTile;
+          const bool need_mask = (kv0 + kTile > args.N) || (args.causal && j == i);
+          const int lim = args.causal ? min(args.N, q_row + 1) : args.N;
+#pragma unroll
+          for (int c = 0; c < kTile; ++c) {
+            float e = ex2_approx(fmaf(__uint_as_float(r[c]), args.scale_log2, -l2));
+            if (need_mask && kv0 + c >= lim) e = 0.f;
+            p[c] = e;
+          }
+        }
+        ok = wait(bar(L::kBarDPFull), dp_cnt & 1);
+        if (!ok) break;
+        ++dp_cnt;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < kTile / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tdP + lane_off + c * 32, r);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const int c0 = c * 32 + 2 * k;
+            pk[k] = pack_bf16x2(p[c0] * (__uint_as_float(r[2 * k]) - drow),
+                                p[c0 + 1] * (__uint_as_float(r[2 * k + 1]) - drow));
+          }
+          tmem_st16(tdP + lane_off + c * 16, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(L::kBarDSReady));
+      }
+      if (!ok) break;
+      ok = wait(bar(L::kBarAccFull), units & 1);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const size_t off = (static_cast<size_t>(bh) * args.N + q_row) * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tdQ + lane_off + c * 32, v);
+        tmem_wait_ld();
+        if (q_row < args.N) store_row32(args.dQ + off + c * 32, v, args.scale);
+      }
+      tc_fence_before();
+      mbar_arrive(bar(L::kBarAccFree));
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMMA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+template <int D>
+cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                     const CUtensorMap& tmdO, const CUtensorMap& tmL2, const CUtensorMap& tmD,
+                     const void* O, const void* dO, const float* LSE, void* dQ, void* dK,
+                     void* dV, float* ws, const Problem& p, int num_sms, cudaStream_t stream) {
+  BwdArgs a;
+  a.err = p.err;
+  a.dQ = static_cast<__nv_bfloat16*>(dQ);
+  a.dK = static_cast<__nv_bfloat16*>(dK);
+  a.dV = static_cast<__nv_bfloat16*>(dV);
+  a.BH = p.BH;
+  a.N = p.N;
+  a.n_tiles = (p.N + kTile - 1) / kTile;
+  a.Npad = a.n_tiles * kTile;
+  a.total_units = p.BH * a.n_tiles;
+  a.causal = p.causal;
+  a.scale = p.scale;
+  a.scale_log2 = p.scale * kLog2e;
+  float* Dpad = ws;
+  float* L2pad = ws + static_cast<size_t>(p.BH) * a.Npad;
+  a.Dpad = Dpad;
+  a.L2pad = L2pad;
+
+  const long long rows = static_cast<long long>(p.BH) * a.Npad;
+  bwd_prep_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO), LSE, Dpad,
+      L2pad, p.BH, p.N, a.Npad);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+
+  const int grid = a.total_units < num_sms ? a.total_units : num_sms;
+  e = cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           DkdvLayout<D>::kAlloc);
+  if (e != cudaSuccess) return e;
+  bwd_dkdv_kernel<D><<<grid, kThreads, DkdvLayout<D>::kAlloc, stream>>>(tmQ, tmK, tmV, tmdO,
+                                                                         tmL2, tmD, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           DqLayout<D>::kAlloc);
+  if (e != cudaSuccess) return e;
+  bwd_dq_kernel<D><<<grid, kThreads, DqLayout<D>::kAlloc, stream>>>(tmQ, tmK, tmV, tmdO, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int bwd_padded_rows(int N) { return round_up(N, kTile); }
+
+cudaError_t launch_bwd_sm100(const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                             const CUtensorMap& tmV, const CUtensorMap& tmdO,
+                             const CUtensorMap& tmL2, const CUtensorMap& tmD, const void* O,
+                             const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                             float* workspace, const Problem& p, int num_sms,
+                             cudaStream_t stream) {
+  if (p.d == 64)
+    return launch_d<64>(tmQ, tmK, tmV, tmdO, tmL2, tmD, O, dO, LSE, dQ, dK, dV, workspace, p,
+                        num_sms, stream);
+  return launch_d<128>(tmQ, tmK, tmV, tmdO, tmL2, tmD, O, dO, LSE, dQ, dK, dV, workspace, p,
+                       num_sms, stream);
 }
 
 }  // namespace fa

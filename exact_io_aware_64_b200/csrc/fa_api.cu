@@ -110,13 +110,33 @@ fa_status make_tmap(CUtensorMap* tm, const void* ptr, int BH, int N, int d) {
   return FA_OK;
 }
 
+// [BH][rows] float32 (a per-row statistic padded to whole tiles) viewed as a 3-D tensor
+// [1][BH][rows] with boxes of 128 rows, no swizzle.
+fa_status make_row_tmap(CUtensorMap* tm, const float* ptr, int BH, int rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(BH), 1};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(rows) * 4,
+                           static_cast<cuuint64_t>(rows) * static_cast<cuuint64_t>(BH) * 4};
+  cuuint32_t box[3] = {128, 1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return FA_OK;
+}
+
 // ------------------------------------------------------------------ validation
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-bool overlaps(const void* a, const void* b, size_t bytes) {
+// [a, a + a_bytes) and [b, b + b_bytes) share a byte
+bool overlaps(const void* a, size_t a_bytes, const void* b, size_t b_bytes) {
   const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
-  return x < y + bytes && y < x + bytes;
+  return x < y + b_bytes && y < x + a_bytes;
 }
+
+bool overlaps(const void* a, const void* b, size_t bytes) { return overlaps(a, bytes, b, bytes); }
 
 // Checks shared by every call.  Sets *noop when there is nothing to compute.
 fa_status check_common(int B, int H, int N, int d, float scale, int causal, bool* noop) {
@@ -222,7 +242,8 @@ fa_status fa_fwd_f32(const float* Q, const float* K, const float* V, float* O, f
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
   (void)d;
   if (B <= 0 || H <= 0 || N <= 0) return 0;
-  const size_t raw = static_cast<size_t>(B) * H * N * sizeof(float);
+  // D and LSE*log2(e), one float each per row, rows padded to whole 128-row tiles
+  const size_t raw = 2 * static_cast<size_t>(B) * H * fa::bwd_padded_rows(N) * sizeof(float);
   return (raw + 255) / 256 * 256;
 }
 
@@ -256,7 +277,7 @@ fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, con
   for (void* o : outs) {
     for (const void* in : ins)
       if (overlaps(o, in, bytes)) return fail(FA_ERR_INVALID_ARG, "a gradient overlaps an input");
-    if (need > 0 && overlaps(o, workspace, need > bytes ? need : bytes))
+    if (need > 0 && overlaps(o, bytes, workspace, need))
       return fail(FA_ERR_INVALID_ARG, "a gradient overlaps the workspace");
   }
   if (overlaps(dQ, dK, bytes) || overlaps(dQ, dV, bytes) || overlaps(dK, dV, bytes))
@@ -265,14 +286,18 @@ fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, con
   FA_TRY(device_info(&dev));
   FA_TRY(require_sm100(dev));
   const int BH = B * H;
-  CUtensorMap tmQ, tmK, tmV, tmdO;
+  CUtensorMap tmQ, tmK, tmV, tmdO, tmL2, tmD;
   FA_TRY(make_tmap(&tmQ, Q, BH, N, d));
   FA_TRY(make_tmap(&tmK, K, BH, N, d));
   FA_TRY(make_tmap(&tmV, V, BH, N, d));
   FA_TRY(make_tmap(&tmdO, dO, BH, N, d));
+  const int Npad = fa::bwd_padded_rows(N);
+  float* ws = static_cast<float*>(workspace);
+  FA_TRY(make_row_tmap(&tmD, ws, BH, Npad));
+  FA_TRY(make_row_tmap(&tmL2, ws + static_cast<size_t>(BH) * Npad, BH, Npad));
   fa::Problem p{BH, N, d, scale, causal, dev.err};
-  cudaError_t e = fa::launch_bwd_sm100(tmQ, tmK, tmV, tmdO, O, dO, LSE, dQ, dK, dV,
-                                       static_cast<float*>(workspace), p, dev.num_sms, stream);
+  cudaError_t e = fa::launch_bwd_sm100(tmQ, tmK, tmV, tmdO, tmL2, tmD, O, dO, LSE, dQ, dK, dV,
+                                       ws, p, dev.num_sms, stream);
   if (e != cudaSuccess) return cuda_fail(e, "launching the backward kernels");
   return FA_OK;
 }

@@ -94,8 +94,9 @@ FA_API fa_status fa_fwd_f32(const float* Q, const float* K, const float* V, floa
                      cudaStream_t stream);
 
 /*
- * Bytes of scratch that fa_bwd needs for given sizes: one float32 per query row for
- * D_i = sum_k dO_ik O_ik, rounded up to 256 bytes.  Grows as B*H*N, never as N^2.
+ * Bytes of scratch that fa_bwd needs for given sizes: two float32 per query row
+ * (D_i = sum_k dO_ik O_ik and LSE_i * log2(e)), rows padded to a multiple of 128,
+ * rounded up to 256 bytes: 8 * B * H * ceil(N/128) * 128.  Grows as B*H*N, never as N^2.
  */
 FA_API size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
 

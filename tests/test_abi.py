@@ -54,11 +54,13 @@ def test_status_strings(lib):
 
 
 def test_workspace_is_linear_in_rows(lib):
-    assert binding.workspace_bytes(2, 16, 8192, 128) == 2 * 16 * 8192 * 4
-    assert binding.workspace_bytes(1, 1, 1, 64) == 256          # rounded up to 256 bytes
+    # two float32 per row (D and LSE*log2e), rows padded to whole 128-row tiles
+    assert binding.workspace_bytes(2, 16, 8192, 128) == 2 * 2 * 16 * 8192 * 4
+    assert binding.workspace_bytes(1, 1, 1, 64) == 2 * 128 * 4
+    assert binding.workspace_bytes(1, 32, 10000, 128) == 2 * 32 * 10112 * 4
     assert binding.workspace_bytes(0, 4, 128, 64) == 0
     # O(B*H*N), never O(N^2): the backward stores no score tile
-    assert binding.workspace_bytes(1, 1, 32768, 128) == 32768 * 4
+    assert binding.workspace_bytes(1, 1, 32768, 128) == 2 * 32768 * 4
 
 
 # Fake, 16-byte aligned addresses: validation must fail (or finish) before any use.
@@ -117,6 +119,9 @@ def test_bwd_validation(lib):
     assert call(dQ=A) == binding.FA_ERR_INVALID_ARG         # gradient overlaps an input
     assert call(dK=G) == binding.FA_ERR_INVALID_ARG         # gradients overlap
     assert call(ws=H_) == binding.FA_ERR_INVALID_ARG        # workspace overlaps dK
+    # a workspace right after a small gradient does not overlap it
+    small = [A, B_, C, D_, E, F, G, H_, I, 1, 1, 1, 64, 0.1, 0, I + 128, 1024, None]
+    assert lib.fa_bwd(*small) != binding.FA_ERR_INVALID_ARG
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

@@ -1,0 +1,123 @@
+"""Backward parity: fa_bwd through the C ABI against the analytic fp64 oracle.
+
+The CUDA forward provides O and LSE (as a user would run it); the oracle recomputes
+everything from Q, K, V, dO in float64.  Small problems are compared in full; the named
+workload (B=2, H=16, N=8192, d=128, causal) in full on two seeded (batch, head) pairs and
+on a seeded subset of dQ rows in every head.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_io_aware_64_b200 import binding, inputs
+from parity import BF16_MAX_ABS, assert_bf16_close, errors, to64
+
+pytestmark = pytest.mark.gpu
+
+
+def _fwd_bwd(ins, scale, causal):
+    q, k, v, do = (ins[n].cuda() for n in ("Q", "K", "V", "dO"))
+    O, LSE = binding.fwd(q, k, v, scale=scale, causal=causal)
+    dQ, dK, dV = binding.bwd(q, k, v, O, do, LSE, scale=scale, causal=causal)
+    binding.check_device_error()
+    return dQ, dK, dV, O
+
+
+def _check_head(ins, grads, b, h, scale, causal, what=""):
+    """Against the exact gradient, within the bf16 tolerance."""
+    Q, K, V, dO = (to64(ins[n][b, h]) for n in ("Q", "K", "V", "dO"))
+    rQ, rK, rV, _ = oracle.attention_bwd_head(Q, K, V, dO, scale, causal)
+    for got, ref, name in zip(grads, (rQ, rK, rV), ("dQ", "dK", "dV")):
+        assert_bf16_close(to64(got[b, h]), ref, f"{what} {name} b={b} h={h} causal={causal}")
+
+
+def _check_head_given_O(ins, grads, O, b, h, scale, causal, what=""):
+    """Against the gradient formed with the bf16 forward output that fa_bwd was handed
+    (D = rowsum(dO * O)).  For a handful of keys the bf16 rounding of O alone moves dQ by
+    about 1% relative L2 (the difference dP - D is then small), so tiny problems are
+    held to the bf16 tolerance on this reference, and to the max-abs bound against the
+    exact gradient."""
+    Q, K, V, dO = (to64(ins[n][b, h]) for n in ("Q", "K", "V", "dO"))
+    exact = oracle.attention_bwd_head(Q, K, V, dO, scale, causal)
+    given = oracle.attention_bwd_head(Q, K, V, dO, scale, causal, O_given=to64(O[b, h]))
+    for k, name in enumerate(("dQ", "dK", "dV")):
+        got = to64(grads[k][b, h])
+        assert_bf16_close(got, given[k], f"{what} {name} b={b} h={h} causal={causal}")
+        max_abs, _ = errors(got, exact[k])
+        assert max_abs <= BF16_MAX_ABS, f"{what} {name} vs exact: max_abs={max_abs:.3e}"
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("N", [1, 2, 100, 128, 129, 256, 300, 513])
+def test_bwd_full_small(N, d, causal):
+    ins = inputs.make_inputs(1, 3, N, d, seed=2000 + N, with_dO=True)
+    scale = 1.0 / np.sqrt(d)
+    *grads, O = _fwd_bwd(ins, scale, causal)
+    for h in range(3):
+        _check_head_given_O(ins, grads, O, 0, h, scale, causal, f"N={N} d={d}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_many_units_per_cta(causal):
+    # 2 * 40 heads * 8 tiles = 640 units per kernel > 148 SMs
+    B, H, N, d = 2, 40, 1000, 64
+    ins = inputs.make_inputs(B, H, N, d, seed=31, with_dO=True)
+    *grads, _ = _fwd_bwd(ins, 0.125, causal)
+    for b, h in ((0, 0), (1, 39), (0, 17)):
+        _check_head(ins, grads, b, h, 0.125, causal, "many units")
+
+
+def test_workload_n8192_backward():
+    w = inputs.WORKLOADS["n8192_d128_causal_bwd"]
+    ins = inputs.make_workload_inputs(w)
+    *grads, _ = _fwd_bwd(ins, w.scale, w.causal)
+    rng = np.random.default_rng(1234)
+    pairs = {(int(rng.integers(w.B)), int(rng.integers(w.H))) for _ in range(2)}
+    for b, h in sorted(pairs):
+        _check_head(ins, grads, b, h, w.scale, w.causal, w.name)
+    dQ = to64(grads[0])
+    rows = np.array(inputs.sample_rows(w.N, 256, seed=99))
+    for b in range(w.B):
+        for h in range(w.H):
+            Q, K, V, dO = (to64(ins[n][b, h]) for n in ("Q", "K", "V", "dO"))
+            rQ, _ = oracle.attention_bwd_dq_rows(Q[rows], K, V, dO[rows], w.scale, w.causal,
+                                                 rows)
+            assert_bf16_close(dQ[b, h, rows], rQ, f"{w.name} dQ rows b={b} h={h}")
+
+
+def test_bwd_deterministic_and_in_bounds():
+    B, H, N, d = 1, 6, 777, 128
+    ins = inputs.make_inputs(B, H, N, d, seed=8, with_dO=True)
+    q, k, v, do = (ins[n].cuda() for n in ("Q", "K", "V", "dO"))
+    O, LSE = binding.fwd(q, k, v, causal=True)
+    guard = 4096
+    n = B * H * N * d
+    bufs = [torch.full((2 * guard + n,), 5.0, device="cuda", dtype=torch.bfloat16)
+            for _ in range(3)]
+    views = [b[guard:guard + n].view(B, H, N, d) for b in bufs]
+    ws_bytes = binding.workspace_bytes(B, H, N, d)
+    wsbuf = torch.full((ws_bytes + 2 * guard,), 0xAB, device="cuda", dtype=torch.uint8)
+    ws = wsbuf[guard:guard + ws_bytes]
+    outs = []
+    for _ in range(2):
+        binding.bwd(q, k, v, O, do, LSE, causal=True, dQ=views[0], dK=views[1], dV=views[2],
+                    workspace=ws)
+        binding.check_device_error()
+        outs.append([t.clone() for t in views])
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
+    for b in bufs:
+        assert bool((b[:guard] == 5.0).all()) and bool((b[-guard:] == 5.0).all())
+    assert bool((wsbuf[:guard] == 0xAB).all()) and bool((wsbuf[-guard:] == 0xAB).all())
+
+
+def test_bwd_rejects_small_workspace():
+    ins = inputs.make_inputs(1, 2, 256, 64, seed=1, with_dO=True)
+    q, k, v, do = (ins[n].cuda() for n in ("Q", "K", "V", "dO"))
+    O, LSE = binding.fwd(q, k, v)
+    small = torch.empty(64, device="cuda", dtype=torch.uint8)
+    with pytest.raises(binding.FAError) as e:
+        binding.bwd(q, k, v, O, do, LSE, workspace=small)
+    assert e.value.status == binding.FA_ERR_INVALID_ARG
