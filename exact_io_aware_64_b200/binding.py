@@ -37,6 +37,9 @@ SIGNATURES = {
     "fa_bwd_workspace_bytes": ([_i, _i, _i, _i], _sz),
     "fa_bwd": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _sz,
                 _vp], _i),
+    "fa_bwd_noalloc": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i,
+                        _vp], _i),
+    "fa_bwd_noalloc_max_scratch_bytes": ([], _sz),
     "fa_status_string": ([_i], ctypes.c_char_p),
     "fa_last_error_message": ([], ctypes.c_char_p),
     "fa_check_device_error": ([_vp], _i),
@@ -157,6 +160,33 @@ def bwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, O: torch.Tensor,
                           _ptr(dK), _ptr(dV), B, H, N, d, float(scale), int(bool(causal)),
                           _ptr(workspace), ws_bytes, _stream_handle(stream))
     _check("fa_bwd", st)
+    return dQ, dK, dV
+
+
+def bwd_noalloc(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, O: torch.Tensor,
+                dO: torch.Tensor, LSE: torch.Tensor, scale: Optional[float] = None,
+                causal: bool = False, dQ: Optional[torch.Tensor] = None,
+                dK: Optional[torch.Tensor] = None, dV: Optional[torch.Tensor] = None,
+                stream: Optional[torch.cuda.Stream] = None):
+    """Backward through ``fa_bwd_noalloc``: the library's fixed scratch replaces the
+    workspace, for callers that cannot allocate device memory.  Outputs may be passed in
+    so that nothing is allocated here either.  Returns (dQ, dK, dV)."""
+    B, H, N, d = Q.shape
+    for name, t in (("Q", Q), ("K", K), ("V", V), ("O", O), ("dO", dO)):
+        _check_bhnd(name, t, (B, H, N, d), torch.bfloat16)
+    _check_bhnd("LSE", LSE, (B, H, N), torch.float32)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dQ = torch.empty_like(Q) if dQ is None else dQ
+    dK = torch.empty_like(K) if dK is None else dK
+    dV = torch.empty_like(V) if dV is None else dV
+    for name, t in (("dQ", dQ), ("dK", dK), ("dV", dV)):
+        _check_bhnd(name, t, (B, H, N, d), torch.bfloat16)
+    with torch.cuda.device(Q.device):
+        st = lib().fa_bwd_noalloc(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _ptr(LSE),
+                                  _ptr(dQ), _ptr(dK), _ptr(dV), B, H, N, d, float(scale),
+                                  int(bool(causal)), _stream_handle(stream))
+    _check("fa_bwd_noalloc", st)
     return dQ, dK, dV
 
 

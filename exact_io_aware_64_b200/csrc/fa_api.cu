@@ -321,3 +321,79 @@ fa_status fa_check_device_error(cudaStream_t stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------
+// fa_bwd_noalloc: the backward pass for callers that cannot allocate device memory.
+//
+// Some callers have no way to hand fa_bwd a workspace: a plugin whose host API gives it
+// no allocator, code that runs inside a framework step whose memory plan is frozen, or
+// a latency-sensitive loop that must not enter cudaMalloc (which can synchronise the
+// device).  For them the library keeps its own scratch: the array below, a fixed
+// kNoAllocScratchBytes of device memory that every GPU which loads libfa.so holds until
+// the process exits.  The caller still provides every input and output.
+//
+// In host code `g_fa_bwd_scratch` names a host-side stand-in, not device memory, so it
+// is never passed to a kernel directly.  The first fa_bwd_noalloc call on a device looks
+// up the array's device address with cudaGetSymbolAddress while that device is current
+// and caches it; that first call should therefore come before any stream capture.
+//
+// Every call shares the one array.  fa_bwd fully rewrites the part it uses (D and
+// LSE*log2(e) for every padded row) before reading it, so nothing needs clearing between
+// calls, but two calls whose kernels overlap on the GPU (different streams, or another
+// thread) race on the array and give wrong gradients: serialise them.
+// ---------------------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 8u << 20;  // 8 MiB: B*H*ceil(N/128)*128 <= 2^20
+static __device__ __align__(256) unsigned char g_fa_bwd_scratch[kNoAllocScratchBytes];
+
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[kMaxDevices] = {};
+
+fa_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(FA_ERR_CUDA, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_fa_bwd_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(g_fa_bwd_scratch)");
+    g_scratch_addr[dev] = ptr;
+  }
+  *out = g_scratch_addr[dev];
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t fa_bwd_noalloc_max_scratch_bytes(void) { return kNoAllocScratchBytes; }
+
+fa_status fa_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O,
+                         const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                         int B, int H, int N, int d, float scale, int causal,
+                         cudaStream_t stream) {
+  g_last_error[0] = '\0';
+  if (B > 0 && H > 0 && N > 0) {
+    const size_t need = fa_bwd_workspace_bytes(B, H, N, d);
+    if (need > kNoAllocScratchBytes)
+      return fail(FA_ERR_INVALID_ARG,
+                  "fa_bwd_noalloc: B=%d H=%d N=%d needs %zu bytes of scratch, more than the "
+                  "library's fixed %zu (B*H*ceil(N/128)*128 must be at most %zu); use fa_bwd "
+                  "with a workspace",
+                  B, H, N, need, kNoAllocScratchBytes, kNoAllocScratchBytes / 8);
+  }
+  void* scratch = nullptr;
+  bool noop = false;
+  fa_status st = check_common(B, H, N, d, scale, causal, &noop);
+  if (st != FA_OK || noop) return st;
+  st = noalloc_scratch(&scratch);
+  if (st != FA_OK) return st;
+  return fa_bwd(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, scale, causal, scratch,
+                kNoAllocScratchBytes, stream);
+}
+
+}  // extern "C"

@@ -117,6 +117,32 @@ FA_API fa_status fa_bwd(const void* Q, const void* K, const void* V, const void*
                  int B, int H, int N, int d, float scale, int causal,
                  void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/*
+ * fa_bwd for callers that cannot allocate device memory (no counterpart on the pages:
+ * it is a property of this library, not of the method).  Same arguments and result as
+ * fa_bwd, without the workspace: the scratch is a fixed array inside the library,
+ * fa_bwd_noalloc_max_scratch_bytes() bytes (8 MiB) of device memory that every GPU which
+ * loads the library keeps until the process exits.
+ *   Who needs it: a caller with no allocator to draw on (a plugin host that passes only
+ *   tensors), code inside a framework step whose memory plan is fixed, or a loop that
+ *   must not enter cudaMalloc because it can synchronise the device.
+ *   Limit: fa_bwd_workspace_bytes(B,H,N,d) must not exceed that size, i.e.
+ *   B*H*ceil(N/128)*128 <= 2^20 rows; larger problems get FA_ERR_INVALID_ARG.
+ *   Set-up: the first call on a device looks up the array's device address and caches
+ *   it (no allocation); make that first call before any stream capture.
+ *   Sharing: all calls use the same array.  Each call rewrites what it reads, so no
+ *   clearing is needed, but calls whose kernels overlap on the GPU race on the array:
+ *   serialise them (one stream, or synchronise between streams and threads).
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ */
+FA_API fa_status fa_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O,
+                                const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                                int B, int H, int N, int d, float scale, int causal,
+                                cudaStream_t stream);
+
+/* Size of the fixed scratch array behind fa_bwd_noalloc, in bytes. */
+FA_API size_t fa_bwd_noalloc_max_scratch_bytes(void);
+
 /* Static text for a status code ("FA_OK", ...). */
 FA_API const char* fa_status_string(fa_status status);
 
