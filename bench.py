@@ -248,21 +248,26 @@ def run_gpu(args, w):
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
 
     def step(marks=None):
-        if marks is not None:
-            marks[0].record(stream)
-        binding.fwd(q, k, v, scale=w.scale, causal=w.causal, O=O, LSE=LSE)
-        if marks is not None:
-            marks[1].record(stream)
+        # marks: [fwd before, fwd after, bwd before, prep done, dkdv done, dq done], recorded
+        # by the library at its kernel boundaries (fa_trace_events)
+        if marks is None:
+            binding.fwd(q, k, v, scale=w.scale, causal=w.causal, O=O, LSE=LSE)
+        else:
+            with binding.trace_kernels(marks[0:2]):
+                binding.fwd(q, k, v, scale=w.scale, causal=w.causal, O=O, LSE=LSE)
         if with_bwd:
-            binding.bwd(q, k, v, O, do, LSE, scale=w.scale, causal=w.causal, dQ=dQ, dK=dK,
-                        dV=dV, workspace=ws)
-        if marks is not None:
-            marks[2].record(stream)
+            if marks is None:
+                binding.bwd(q, k, v, O, do, LSE, scale=w.scale, causal=w.causal, dQ=dQ, dK=dK,
+                            dV=dV, workspace=ws)
+            else:
+                with binding.trace_kernels(marks[2:6]):
+                    binding.bwd(q, k, v, O, do, LSE, scale=w.scale, causal=w.causal, dQ=dQ,
+                                dK=dK, dV=dV, workspace=ws)
 
     for _ in range(args.warmup):
         step()
     binding.check_device_error()
-    marks = [[ev(), ev(), ev()] for _ in range(args.steps)]
+    marks = [[ev() for _ in range(6)] for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
@@ -276,10 +281,27 @@ def run_gpu(args, w):
     binding.check_device_error()
     ms_local = start.elapsed_time(end) / args.steps
     ms = max_over_ranks(ms_local, world)
-    fwd_ms = statistics.mean(m[0].elapsed_time(m[1]) for m in marks)
-    bwd_ms = statistics.mean(m[1].elapsed_time(m[2]) for m in marks) if with_bwd else 0.0
+    def span(a, b):
+        return statistics.mean(m[a].elapsed_time(m[b]) for m in marks)
+
+    fwd_ms = span(0, 1)
+    bwd_ms = span(2, 5) if with_bwd else 0.0
     f_fwd = traffic.fwd_flops(B, H, N, d, w.causal)
     f_bwd = traffic.bwd_flops(B, H, N, d, w.causal) if with_bwd else 0.0
+    # per kernel: mean launch time and algorithmic work (FLOPs credited to that kernel,
+    # or bytes for the bandwidth-bound preparation)
+    kernels = {"fwd_sm100_kernel": {"ms": fwd_ms, "flops": f_fwd}}
+    if with_bwd:
+        half = 0.5 if w.causal else 1.0
+        kernels["bwd_prep_kernel"] = {"ms": span(2, 3),
+                                      "bytes": traffic.bwd_prep_bytes(B, H, N, d)}
+        kernels["bwd_dkdv_kernel"] = {"ms": span(3, 4), "flops": 8.0 * B * H * N * N * d * half}
+        kernels["bwd_dq_kernel"] = {"ms": span(4, 5), "flops": 2.0 * B * H * N * N * d * half}
+    for kinfo in kernels.values():
+        if "flops" in kinfo:
+            kinfo["tflops"] = kinfo["flops"] / (kinfo["ms"] * 1e-3) / 1e12
+        else:
+            kinfo["gbs"] = kinfo["bytes"] / (kinfo["ms"] * 1e-3) / 1e9
     value = world * (f_fwd + f_bwd) / (ms * 1e-3) / 1e12
 
     # ---- end to end through the public API with host buffers
@@ -322,15 +344,11 @@ def run_gpu(args, w):
         return 0
 
     peaks, peak_src = load_peaks()
-    # dominant kernel: the forward kernel or the backward call, whichever takes longer
-    if with_bwd and bwd_ms > fwd_ms:
-        dom_name, dom_ms, dom_flops = "fa_bwd (3 kernels)", bwd_ms, f_bwd
-        dom_key = "bwd"
-    else:
-        dom_name, dom_ms, dom_flops = "fwd_sm100_kernel", fwd_ms, f_fwd
-        dom_key = "fwd_sm100_kernel"
+    # dominant kernel: the one with the longest mean launch time
+    dom_name = max(kernels, key=lambda k: kernels[k]["ms"])
+    dom = kernels[dom_name]
     peak = peaks.get("bf16_tflops_sustained" if args.sustained_peak else "bf16_tflops")
-    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    achieved = dom["tflops"]
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -347,7 +365,8 @@ def run_gpu(args, w):
                      "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": f"{peak_src} "
                                     f"{'sustained' if args.sustained_peak else 'burst'} bf16",
-                     "traffic": recorded_traffic(dom_key)},
+                     "traffic": recorded_traffic(dom_name)},
+        "kernels": kernels,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": args.steps * (1 + (3 if with_bwd else 0)),

@@ -40,6 +40,7 @@ SIGNATURES = {
     "fa_bwd_noalloc": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i,
                         _vp], _i),
     "fa_bwd_noalloc_max_scratch_bytes": ([], _sz),
+    "fa_trace_events": ([ctypes.POINTER(_vp), _i], _i),
     "fa_status_string": ([_i], ctypes.c_char_p),
     "fa_last_error_message": ([], ctypes.c_char_p),
     "fa_check_device_error": ([_vp], _i),
@@ -188,6 +189,25 @@ def bwd_noalloc(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, O: torch.Tens
                                   int(bool(causal)), _stream_handle(stream))
     _check("fa_bwd_noalloc", st)
     return dQ, dK, dV
+
+
+class trace_kernels:
+    """Context manager: record the given torch.cuda.Events at kernel boundaries of the
+    library calls made inside it (fa_trace_events).  events[0] before the first kernel
+    of each call, events[k] after its k-th kernel."""
+
+    def __init__(self, events):
+        for e in events:
+            e.record()  # make sure the underlying cudaEvent_t exists
+        self._arr = (_vp * len(events))(*[e.cuda_event for e in events])
+        self._n = len(events)
+
+    def __enter__(self):
+        _check("fa_trace_events", lib().fa_trace_events(self._arr, self._n))
+        return self
+
+    def __exit__(self, *exc):
+        lib().fa_trace_events(None, 0)
 
 
 def check_device_error(stream: Optional[torch.cuda.Stream] = None) -> None:

@@ -23,10 +23,12 @@
 //      stream past:  S = Q_i K_j^T, dP = dO_i V_j^T, P, dS as above, dQ_i += dS K_j.
 //      TMEM: dQ | S | dP (dS over its first 64 columns).
 //
-// Both tensor-core kernels are persistent (one CTA per SM) with 256 threads: warps 0-3
-// are the element-wise warps (thread = TMEM lane = tile row; up to 255 registers, so a
-// whole 128-entry probability row stays in registers), warp 4 issues TMA loads, warp 5
-// issues the MMAs from one thread, warps 6-7 are idle.  The MMA order is chosen so the
+// Both tensor-core kernels are persistent (one CTA per SM) with 384 threads: warps 0-7
+// are two element-wise warpgroups that split every 128 x 128 tile by columns (group g
+// owns columns 64g..64g+63; thread = TMEM lane = tile row), warp 8 issues TMA loads,
+// warp 9 issues the MMAs from one thread, warps 10-11 only give up their registers.  Each group writes its bf16 half-row of P or
+// dS over the first 32 columns of its own 64-column half, so the two groups never touch
+// each other's TMEM, and the MMA reads the bf16 operand as two 32-column pieces.  The MMA order is chosen so the
 // tensor core works on one product while the element-wise warps build the next operand
 // (dK/dV: S^T(i) dP^T(i) | dV(i) S^T(i+1) | dK(i) dP^T(i+1) | ...;
 //  dQ: S(j) dP(j) | S(j+1) | dQ(j) dP(j+1) | S(j+2) | ...).
@@ -42,9 +44,26 @@ namespace {
 using namespace sm100;
 
 constexpr int kTile = 128;        // rows per query / key tile
-constexpr int kThreads = 256;
-constexpr int kWarpTMA = 4;
-constexpr int kWarpMMA = 5;
+constexpr int kGroups = 2;        // element-wise warpgroups, splitting a tile's columns
+constexpr int kCols = kTile / kGroups;
+constexpr int kEw = kGroups * 128;  // element-wise threads
+constexpr int kThreads = kEw + 128;  // + a control warpgroup: TMA warp, MMA warp, 2 idle
+constexpr int kWarpTMA = kEw / 32;
+constexpr int kWarpMMA = kWarpTMA + 1;
+// 12 warps put 3 on each SM sub-partition, so the launch grants 168 registers a thread
+// (3 x 32 x 168 <= 16384 per sub-partition).  The control warpgroup drops to 104 and the
+// element-wise warpgroups rise to 200: 2 x 128 x 200 + 128 x 104 = 384 x 168.
+constexpr int kRegsLaunch = 168;
+constexpr int kRegsControl = 104;
+constexpr int kRegsEw = 200;
+static_assert(kGroups * 128 * kRegsEw + 128 * kRegsControl <= kThreads * kRegsLaunch,
+              "register split exceeds the launch pool");
+
+// TMEM column of the k-th 16-wide K step of a bf16 operand written as two 32-column
+// pieces at `base` and `base + 64` (one per element-wise group).
+__device__ __forceinline__ uint32_t split_operand_col(uint32_t base, int kk) {
+  return base + (kk / 4) * 64 + (kk % 4) * 8;
+}
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -177,14 +196,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(L::kBarKVEmpty), 1);
     for (int s = 0; s < L::kStages; ++s) {
       mbar_init(bar(L::kBarQFull + s), 1);
-      mbar_init(bar(L::kBarQEmpty + s), 1 + kTile);  // MMA commit + element-wise threads
+      mbar_init(bar(L::kBarQEmpty + s), 1 + kEw / 32);  // MMA commit + element-wise warps
     }
     mbar_init(bar(L::kBarSFull), 1);
     mbar_init(bar(L::kBarDPFull), 1);
-    mbar_init(bar(L::kBarPReady), kTile);
-    mbar_init(bar(L::kBarDSReady), kTile);
+    mbar_init(bar(L::kBarPReady), kEw / 32);
+    mbar_init(bar(L::kBarDSReady), kEw / 32);
     mbar_init(bar(L::kBarAccFull), 1);
-    mbar_init(bar(L::kBarAccFree), kTile);
+    mbar_init(bar(L::kBarAccFree), kEw / 32);
     mbar_init(bar(L::kBarDrain), 1);
     fence_mbar_init();
   }
@@ -210,6 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   };
 
+  if (warp >= kWarpTMA) regs_dec<kRegsControl>();
   if (warp == kWarpTMA) {
     if (lane == 0) {
       int stage = 0, units = 0, kv_loads = 0;
@@ -262,10 +282,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       bool ok = true;
       auto stage_base = [&](int s) { return base + L::kStage0 + s * L::kStageBytes; };
-      // S^T = K Q^T or dP^T = V dO^T: both operands K-major, K extent = D
+      // S^T = K Q^T or dP^T = V dO^T: both operands K-major, K extent = D.  The K-step
+      // loops are fully unrolled so that the single issuing thread keeps up with the
+      // tensor pipe (64 cycles per 128 x 128 x 16 MMA).
       auto issue_ss = [&](uint32_t dtm, uint64_t da, uint32_t b_saddr, uint32_t done_bar) {
         const uint64_t db = desc_kmajor(b_saddr);
-#pragma unroll 1
+#pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = ((kk / 4) * L::kBoxBytes + (kk % 4) * 32) >> 4;
           mma_ss(dtm, da + off, db + off, idSS, kk > 0 ? 1u : 0u);
@@ -275,10 +297,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // acc += A(TMEM, 128 x 128 bf16) * B(smem tile, 128 rows x D, MN-major)
       auto issue_ts = [&](uint32_t acc, uint32_t a_tmem, uint32_t b_saddr, bool accumulate) {
         const uint64_t db = desc_mnmajor(b_saddr, L::kBoxBytes);
-#pragma unroll 1
+#pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ts(acc, a_tmem + kk * 8, db + static_cast<uint64_t>((kk * 2048) >> 4), idTS,
-                 (accumulate || kk > 0) ? 1u : 0u);
+          mma_ts(acc, split_operand_col(a_tmem, kk), db + static_cast<uint64_t>((kk * 2048) >> 4),
+                 idTS, (accumulate || kk > 0) ? 1u : 0u);
       };
       for (int w = blockIdx.x; ok && w < args.total_units; w += gridDim.x, ++units) {
         int bh, j, i0;
@@ -326,9 +348,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(bar(L::kBarDrain));
       mbar_wait_drain(bar(L::kBarDrain), 0, args.err);
     }
-  } else if (warp < 4) {
-    const int row = warp * 32 + lane;  // key row within the tile = TMEM lane
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+  } else if (warp < kWarpTMA) {
+    regs_inc<kRegsEw>();
+    const int g = warp / 4;            // column group
+    const int col0 = g * kCols;        // first tile column of this group
+    const int row = (warp % 4) * 32 + lane;  // key row within the tile = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>((warp % 4) * 32) << 16;
     int stage = 0, units = 0, s_cnt = 0, dp_cnt = 0;
     uint32_t phase = 0;
     bool ok = true;
@@ -337,45 +362,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       unit(w, bh, j, i0);
       for (int i = i0; i < args.n_tiles; ++i) {
         const uint8_t* sb = smem + L::kStage0 + stage * L::kStageBytes;
-        const float* sL = reinterpret_cast<const float*>(sb + L::kStageL);
-        const float* sD = reinterpret_cast<const float*>(sb + L::kStageD);
+        const float* sL = reinterpret_cast<const float*>(sb + L::kStageL) + col0;
+        const float* sD = reinterpret_cast<const float*>(sb + L::kStageD) + col0;
         ok = wait(bar(L::kBarQFull + stage), phase);
         if (ok) ok = wait(bar(L::kBarSFull), s_cnt & 1);
         if (!ok) break;
         ++s_cnt;
         tc_fence_after();
-        float p[kTile];
+        float p[kCols];
         {
-          uint32_t r[kTile];
+          uint32_t r[kCols];
 #pragma unroll
-          for (int c = 0; c < kTile / 32; ++c) tmem_ld32(tS + lane_off + c * 32, &r[c * 32]);
+          for (int c = 0; c < kCols / 32; ++c)
+            tmem_ld32(tS + lane_off + col0 + c * 32, &r[c * 32]);
           tmem_wait_ld();
           const bool diag = args.causal && i == j;
 #pragma unroll
-          for (int c = 0; c < kTile; ++c) {
+          for (int c = 0; c < kCols; ++c) {
             float e = ex2_approx(fmaf(__uint_as_float(r[c]), args.scale_log2, -sL[c]));
-            if (diag && c < row) e = 0.f;  // query i*128+c before key j*128+row
+            if (diag && col0 + c < row) e = 0.f;  // query i*128+col0+c before key j*128+row
             p[c] = e;
           }
         }
         {
-          uint32_t pk[kTile / 2];
+          uint32_t pk[kCols / 2];
 #pragma unroll
-          for (int c = 0; c < kTile / 2; ++c) pk[c] = pack_bf16x2(p[2 * c], p[2 * c + 1]);
-          tmem_st32(tS + lane_off, &pk[0]);
-          tmem_st32(tS + lane_off + 32, &pk[32]);
+          for (int c = 0; c < kCols / 2; ++c) pk[c] = pack_bf16x2(p[2 * c], p[2 * c + 1]);
+          tmem_st32(tS + lane_off + col0, pk);
         }
         tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar(L::kBarPReady));
+        warp_arrive(bar(L::kBarPReady));
         ok = wait(bar(L::kBarDPFull), dp_cnt & 1);
         if (!ok) break;
         ++dp_cnt;
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < kTile / 32; ++c) {
+        for (int c = 0; c < kCols / 32; ++c) {
           uint32_t r[32];
-          tmem_ld32(tdP + lane_off + c * 32, r);
+          tmem_ld32(tdP + lane_off + col0 + c * 32, r);
           tmem_wait_ld();
           uint32_t pk[16];
 #pragma unroll
@@ -385,16 +409,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float ds1 = p[c0 + 1] * (__uint_as_float(r[2 * k + 1]) - sD[c0 + 1]);
             pk[k] = pack_bf16x2(ds0, ds1);
           }
-          tmem_st16(tdP + lane_off + c * 16, pk);
+          // dS for columns c*32.. lands on columns this group has already read
+          tmem_st16(tdP + lane_off + col0 + c * 16, pk);
         }
         tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar(L::kBarDSReady));
-        mbar_arrive(bar(L::kBarQEmpty + stage));  // done with this stage's L2 and D rows
+        warp_arrive(bar(L::kBarDSReady));
+        if (lane == 0) mbar_arrive(bar(L::kBarQEmpty + stage));  // done with its L2, D rows
         if (++stage == L::kStages) stage = 0, phase ^= 1;
       }
       if (!ok) break;
-      // epilogue: dV and scale * dK for this key row
+      // epilogue: dV and scale * dK for this key row; group g writes columns of its half
       ok = wait(bar(L::kBarAccFull), units & 1);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
@@ -402,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int kv_row = j * kTile + row;
       const size_t off = (static_cast<size_t>(bh) * args.N + kv_row) * D;
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = g * (D / 64); c < (g + 1) * (D / 64); ++c) {
         uint32_t v[32];
         tmem_ld32(tdV + lane_off + c * 32, v);
         tmem_wait_ld();
@@ -411,8 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         if (kv_row < args.N) store_row32(args.dK + off + c * 32, v, args.scale);
       }
-      tc_fence_before();
-      mbar_arrive(bar(L::kBarAccFree));
+      warp_arrive(bar(L::kBarAccFree));
     }
   }
 
@@ -481,11 +504,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(L::kBarKVEmpty + s), 1);
     }
     mbar_init(bar(L::kBarSFull), 1);
-    mbar_init(bar(L::kBarSFree), kTile);
+    mbar_init(bar(L::kBarSFree), kEw / 32);
     mbar_init(bar(L::kBarDPFull), 1);
-    mbar_init(bar(L::kBarDSReady), kTile);
+    mbar_init(bar(L::kBarDSReady), kEw / 32);
     mbar_init(bar(L::kBarAccFull), 1);
-    mbar_init(bar(L::kBarAccFree), kTile);
+    mbar_init(bar(L::kBarAccFree), kEw / 32);
     mbar_init(bar(L::kBarDrain), 1);
     fence_mbar_init();
   }
@@ -511,6 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   };
 
+  if (warp >= kWarpTMA) regs_dec<kRegsControl>();
   if (warp == kWarpTMA) {
     if (lane == 0) {
       int stage = 0, units = 0, q_loads = 0;
@@ -562,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto stage_base = [&](int s) { return base + L::kStage0 + s * L::kStageBytes; };
       auto issue_ss = [&](uint32_t dtm, uint64_t da, uint32_t b_saddr, uint32_t done_bar) {
         const uint64_t db = desc_kmajor(b_saddr);
-#pragma unroll 1
+#pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = ((kk / 4) * L::kBoxBytes + (kk % 4) * 32) >> 4;
           mma_ss(dtm, da + off, db + off, idSS, kk > 0 ? 1u : 0u);
@@ -599,10 +623,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           // dQ += dS K_j: A = dS (TMEM), B = K_j (128 key rows x D, MN-major)
           const uint64_t db = desc_mnmajor(stage_base(cur) + L::kStageK, L::kBoxBytes);
-#pragma unroll 1
+#pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
-            mma_ts(tdQ, tdP + kk * 8, db + static_cast<uint64_t>((kk * 2048) >> 4), idTS,
-                   (t > 0 || kk > 0) ? 1u : 0u);
+            mma_ts(tdQ, split_operand_col(tdP, kk), db + static_cast<uint64_t>((kk * 2048) >> 4),
+                   idTS, (t > 0 || kk > 0) ? 1u : 0u);
           mma_commit(bar(L::kBarKVEmpty + cur));
           if (nxt >= 0) {
             issue_ss(tdP, ddO, stage_base(nxt) + L::kStageV, bar(L::kBarDPFull));
@@ -620,9 +644,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(bar(L::kBarDrain));
       mbar_wait_drain(bar(L::kBarDrain), 0, args.err);
     }
-  } else if (warp < 4) {
-    const int row = warp * 32 + lane;  // query row within the tile = TMEM lane
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+  } else if (warp < kWarpTMA) {
+    regs_inc<kRegsEw>();
+    const int g = warp / 4;            // column group
+    const int col0 = g * kCols;        // first tile column (key) of this group
+    const int row = (warp % 4) * 32 + lane;  // query row within the tile = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>((warp % 4) * 32) << 16;
     int units = 0, s_cnt = 0, dp_cnt = 0;
     bool ok = true;
     for (int w = blockIdx.x; ok && w < args.total_units; w += gridDim.x, ++units) {
@@ -637,19 +664,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         ++s_cnt;
         tc_fence_after();
-        float p[kTile];
+        float p[kCols];
         {
-          uint32_t r[kTile];
+          uint32_t r[kCols];
 #pragma unroll
-          for (int c = 0; c < kTile / 32; ++c) tmem_ld32(tS + lane_off + c * 32, &r[c * 32]);
+          for (int c = 0; c < kCols / 32; ++c)
+            tmem_ld32(tS + lane_off + col0 + c * 32, &r[c * 32]);
           tmem_wait_ld();
-          tc_fence_before();
-          mbar_arrive(bar(L::kBarSFree));
-          const int kv0 = j * kTile;
-          const bool need_mask = (kv0 + kTile > args.N) || (args.causal && j == i);
+          warp_arrive(bar(L::kBarSFree));
+          const int kv0 = j * kTile + col0;
+          const bool need_mask = (kv0 + kCols > args.N) || (args.causal && j == i);
           const int lim = args.causal ? min(args.N, q_row + 1) : args.N;
 #pragma unroll
-          for (int c = 0; c < kTile; ++c) {
+          for (int c = 0; c < kCols; ++c) {
             float e = ex2_approx(fmaf(__uint_as_float(r[c]), args.scale_log2, -l2));
             if (need_mask && kv0 + c >= lim) e = 0.f;
             p[c] = e;
@@ -660,9 +687,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++dp_cnt;
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < kTile / 32; ++c) {
+        for (int c = 0; c < kCols / 32; ++c) {
           uint32_t r[32];
-          tmem_ld32(tdP + lane_off + c * 32, r);
+          tmem_ld32(tdP + lane_off + col0 + c * 32, r);
           tmem_wait_ld();
           uint32_t pk[16];
 #pragma unroll
@@ -671,11 +698,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             pk[k] = pack_bf16x2(p[c0] * (__uint_as_float(r[2 * k]) - drow),
                                 p[c0 + 1] * (__uint_as_float(r[2 * k + 1]) - drow));
           }
-          tmem_st16(tdP + lane_off + c * 16, pk);
+          tmem_st16(tdP + lane_off + col0 + c * 16, pk);
         }
         tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar(L::kBarDSReady));
+        warp_arrive(bar(L::kBarDSReady));
       }
       if (!ok) break;
       ok = wait(bar(L::kBarAccFull), units & 1);
@@ -684,14 +710,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const size_t off = (static_cast<size_t>(bh) * args.N + q_row) * D;
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = g * (D / 64); c < (g + 1) * (D / 64); ++c) {
         uint32_t v[32];
         tmem_ld32(tdQ + lane_off + c * 32, v);
         tmem_wait_ld();
         if (q_row < args.N) store_row32(args.dQ + off + c * 32, v, args.scale);
       }
-      tc_fence_before();
-      mbar_arrive(bar(L::kBarAccFree));
+      warp_arrive(bar(L::kBarAccFree));
     }
   }
 
@@ -729,25 +754,36 @@ cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUten
   a.L2pad = L2pad;
 
   const long long rows = static_cast<long long>(p.BH) * a.Npad;
+  cudaError_t e = trace_mark(p, 0, stream);
+  if (e != cudaSuccess) return e;
   bwd_prep_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO), LSE, Dpad,
       L2pad, p.BH, p.N, a.Npad);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = trace_mark(p, 1, stream)) != cudaSuccess) return e;
 
   const int grid = a.total_units < num_sms ? a.total_units : num_sms;
+  // the in-kernel register split assumes exactly kRegsLaunch registers a thread at launch
+  cudaFuncAttributes fattr;
+  e = cudaFuncGetAttributes(&fattr, bwd_dkdv_kernel<D>);
+  if (e != cudaSuccess) return e;
+  if (fattr.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
+  e = cudaFuncGetAttributes(&fattr, bwd_dq_kernel<D>);
+  if (e != cudaSuccess) return e;
+  if (fattr.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
   e = cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            DkdvLayout<D>::kAlloc);
   if (e != cudaSuccess) return e;
   bwd_dkdv_kernel<D><<<grid, kThreads, DkdvLayout<D>::kAlloc, stream>>>(tmQ, tmK, tmV, tmdO,
                                                                          tmL2, tmD, a);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = trace_mark(p, 2, stream)) != cudaSuccess) return e;
   e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            DqLayout<D>::kAlloc);
   if (e != cudaSuccess) return e;
   bwd_dq_kernel<D><<<grid, kThreads, DqLayout<D>::kAlloc, stream>>>(tmQ, tmK, tmV, tmdO, a);
-  return cudaGetLastError();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  return trace_mark(p, 3, stream);
 }
 
 }  // namespace

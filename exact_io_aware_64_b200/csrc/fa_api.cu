@@ -23,6 +23,9 @@ __device__ unsigned int g_fa_device_error;
 namespace {
 
 thread_local char g_last_error[512] = "";
+constexpr int kMaxTrace = 8;
+thread_local cudaEvent_t g_trace[kMaxTrace] = {};
+thread_local int g_n_trace = 0;
 
 fa_status fail(fa_status s, const char* fmt, ...) {
   va_list ap;
@@ -186,6 +189,16 @@ const char* fa_status_string(fa_status s) {
 
 const char* fa_last_error_message(void) { return g_last_error; }
 
+fa_status fa_trace_events(cudaEvent_t* events, int n) {
+  g_last_error[0] = '\0';
+  if (n < 0 || n > kMaxTrace || (n > 0 && events == nullptr))
+    return fail(FA_ERR_INVALID_ARG, "fa_trace_events: n=%d (0..%d, events non-NULL)", n,
+                kMaxTrace);
+  for (int k = 0; k < n; ++k) g_trace[k] = events[k];
+  g_n_trace = n;
+  return FA_OK;
+}
+
 fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H,
                  int N, int d, float scale, int causal, cudaStream_t stream) {
   g_last_error[0] = '\0';
@@ -209,7 +222,7 @@ fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
   FA_TRY(make_tmap(&tmQ, Q, BH, N, d));
   FA_TRY(make_tmap(&tmK, K, BH, N, d));
   FA_TRY(make_tmap(&tmV, V, BH, N, d));
-  fa::Problem p{BH, N, d, scale, causal, dev.err};
+  fa::Problem p{BH, N, d, scale, causal, dev.err, g_n_trace ? g_trace : nullptr, g_n_trace};
   cudaError_t e = fa::launch_fwd_sm100(tmQ, tmK, tmV, O, LSE, p, dev.num_sms, stream);
   if (e != cudaSuccess) return cuda_fail(e, "launching the forward kernel");
   return FA_OK;
@@ -233,7 +246,8 @@ fa_status fa_fwd_f32(const float* Q, const float* K, const float* V, float* O, f
     return fail(FA_ERR_INVALID_ARG, "O overlaps an input");
   DeviceInfo dev;
   FA_TRY(device_info(&dev));
-  fa::Problem p{B * H, N, d, scale, causal, dev.err};
+  fa::Problem p{B * H, N, d, scale, causal, dev.err, g_n_trace ? g_trace : nullptr,
+                g_n_trace};
   cudaError_t e = fa::launch_fwd_f32(Q, K, V, O, LSE, p, stream);
   if (e != cudaSuccess) return cuda_fail(e, "launching the float32 forward kernel");
   return FA_OK;
@@ -295,7 +309,7 @@ fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, con
   float* ws = static_cast<float*>(workspace);
   FA_TRY(make_row_tmap(&tmD, ws, BH, Npad));
   FA_TRY(make_row_tmap(&tmL2, ws + static_cast<size_t>(BH) * Npad, BH, Npad));
-  fa::Problem p{BH, N, d, scale, causal, dev.err};
+  fa::Problem p{BH, N, d, scale, causal, dev.err, g_n_trace ? g_trace : nullptr, g_n_trace};
   cudaError_t e = fa::launch_bwd_sm100(tmQ, tmK, tmV, tmdO, tmL2, tmD, O, dO, LSE, dQ, dK, dV,
                                        ws, p, dev.num_sms, stream);
   if (e != cudaSuccess) return cuda_fail(e, "launching the backward kernels");

@@ -100,8 +100,11 @@ template <int D>
 cudaError_t launch_d(const float* Q, const float* K, const float* V, float* O, float* LSE,
                      const Problem& p, cudaStream_t stream) {
   dim3 grid((p.N + kRows - 1) / kRows, p.BH);
+  cudaError_t e = trace_mark(p, 0, stream);
+  if (e != cudaSuccess) return e;
   fwd_f32_kernel<D><<<grid, kThreads, 0, stream>>>(Q, K, V, O, LSE, p.N, p.scale, p.causal);
-  return cudaGetLastError();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  return trace_mark(p, 1, stream);
 }
 
 }  // namespace

@@ -15,8 +15,9 @@
 //     thread per row, TMEM lane = row), warps 4-7 the softmax of Q1, warp 8 issues TMA
 //     loads, warp 9 issues tcgen05 MMAs from one thread, warps 10-11 only give up their
 //     registers.  The launch grants 168 registers a thread (384 x 168 = 64512); the
-//     control warpgroup drops to 56 and the two softmax warpgroups rise to 224, which
-//     uses exactly that pool (2 x 128 x 224 + 128 x 56 = 64512) and lets a softmax
+//     control warpgroup drops to 88 (enough for fully unrolled MMA issue) and the two
+//     softmax warpgroups rise to 208, which uses exactly that pool
+//     (2 x 128 x 208 + 128 x 88 = 64512) and lets a softmax
 //     thread hold its whole 128-entry score row in registers.
 //   * TMEM (512 columns): S0 | S1 | O0 | O1.  The score tile S_t = Q_t K_j^T lands in
 //     TMEM as fp32; the softmax threads read their row, write the probabilities as bf16
@@ -48,8 +49,8 @@ constexpr int kBM = 128;  // query rows per tile
 constexpr int kBN = 128;  // key rows per tile
 constexpr int kThreads = 384;
 constexpr int kRegsLaunch = 168;   // 65536 / 384, rounded down to a multiple of 8
-constexpr int kRegsControl = 56;
-constexpr int kRegsSoftmax = 224;
+constexpr int kRegsControl = 88;
+constexpr int kRegsSoftmax = 208;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kThreads * kRegsLaunch,
               "register split exceeds the launch pool");
 constexpr int kWarpTMA = 8;
@@ -148,9 +149,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar(L::kBarSFull + t), 1);
-      mbar_init(bar(L::kBarPReady + t), kBM);
+      mbar_init(bar(L::kBarPReady + t), kBM / 32);  // one arrival per softmax warp
       mbar_init(bar(L::kBarODone + t), 1);
-      mbar_init(bar(L::kBarOFree + t), kBM);
+      mbar_init(bar(L::kBarOFree + t), kBM / 32);
     }
     mbar_init(bar(L::kBarDrain), 1);
     fence_mbar_init();
@@ -239,7 +240,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         return r;
       };
       // Descriptors differ only in their start-address field (low 14 bits, address >> 4),
-      // so each K step adds its byte offset >> 4 to a base descriptor.
+      // so each K step adds its byte offset >> 4 to a base descriptor.  The K-step loops
+      // are fully unrolled: one thread issues every MMA, and with loop overhead between
+      // the instructions it cannot keep the tensor pipe fed (a 128 x 128 x 16 MMA takes
+      // only 64 cycles).
       const uint64_t dQ0 = desc_kmajor(base + L::kQ0);
       const uint64_t dQ1 = desc_kmajor(base + L::kQ1);
       const uint64_t dRingK = desc_kmajor(base + L::kRing);
@@ -247,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_s = [&](int t, int kslot) {
         const uint64_t da = t == 0 ? dQ0 : dQ1;
         const uint64_t db = dRingK + static_cast<uint64_t>((kslot * L::kTileBytes) >> 4);
-#pragma unroll 1
+#pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = ((kk / 4) * L::kBoxBytes + (kk % 4) * 32) >> 4;
           mma_ss(tS[t], da + off, db + off, idS, kk > 0 ? 1u : 0u);
@@ -256,7 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       auto issue_pv = [&](int t, int vslot, bool accumulate) {
         const uint64_t db = dRingV + static_cast<uint64_t>((vslot * L::kTileBytes) >> 4);
-#pragma unroll 1
+#pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
           mma_ts(tO[t], tS[t] + kk * 8, db + static_cast<uint64_t>((kk * 2048) >> 4), idPV,
                  (accumulate || kk > 0) ? 1u : 0u);
@@ -284,7 +288,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; ok && j < n; ++j) {
           int vslot, knext = -1;
           ok = next_slot(vslot);
-          if (ok && j + 1 < n) ok = next_slot(knext);
           if (!ok) break;
           for (int t = 0; t < 2 && ok; ++t) {
             if (j >= nt[t]) continue;
@@ -296,6 +299,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             issue_pv(t, vslot, j > 0);
             if (j + 1 < nt[t]) {
+              // the next key tile is needed only now, not before the P V product above
+              if (knext < 0) ok = next_slot(knext);
+              if (!ok) break;
+              tc_fence_after();
               issue_s(t, knext);
               if (j + 2 == nt[t]) mma_commit(bar(L::kBarQEmpty + t));
             }
@@ -349,9 +356,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < kBN; ++c)
             if (kv0 + c >= lim) s[c] = -INFINITY;
         }
-        float mx = s[0];
+        // row max as 8 independent chains folded at the end (a single chain of 128
+        // dependent max operations would sit on the critical path of every tile)
+        float mx8[8];
 #pragma unroll
-        for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, s[c]);
+        for (int k = 0; k < 8; ++k) mx8[k] = s[k];
+#pragma unroll
+        for (int c = 8; c < kBN; ++c) mx8[c % 8] = fmaxf(mx8[c % 8], s[c]);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) mx8[k] = fmaxf(mx8[k], mx8[k + 4]);
+        const float mx = fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3]));
         const float m_tile = mx * args.scale_log2;
         float alpha = 1.f;
         bool rescale = false;
@@ -381,21 +395,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         l *= alpha;
         const float mref = (m == -INFINITY) ? 0.f : m;
         uint32_t pk[kBN / 2];
-        float ls0 = 0.f, ls1 = 0.f;
+        float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c = 0; c < kBN / 2; ++c) {
           const float p0 = ex2_approx(fmaf(s[2 * c], args.scale_log2, -mref));
           const float p1 = ex2_approx(fmaf(s[2 * c + 1], args.scale_log2, -mref));
-          ls0 += p0;
-          ls1 += p1;
+          ls[(2 * c) % 8] += p0;
+          ls[(2 * c + 1) % 8] += p1;
           pk[c] = pack_bf16x2(p0, p1);
         }
-        l += ls0 + ls1;
+        l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
         tmem_st32(tSrow, &pk[0]);
         tmem_st32(tSrow + 32, &pk[32]);
         tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar(L::kBarPReady + t));
+        warp_arrive(bar(L::kBarPReady + t));
       }
       if (!ok) break;
       // epilogue: O = acc / l, LSE = (m + log2 l) * ln 2
@@ -424,8 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
         }
       }
-      tc_fence_before();
-      mbar_arrive(bar(L::kBarOFree + t));
+      warp_arrive(bar(L::kBarOFree + t));
       if (args.LSE != nullptr && q_row < args.N)
         args.LSE[static_cast<size_t>(bh) * args.N + q_row] =
             (m + __log2f(l)) * 0.69314718055994531f;
@@ -465,8 +477,10 @@ cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUten
                            L::kAlloc);
   if (e != cudaSuccess) return e;
   const int grid = a.total_units < num_sms ? a.total_units : num_sms;
+  if ((e = trace_mark(p, 0, stream)) != cudaSuccess) return e;
   fwd_sm100_kernel<D><<<grid, kThreads, L::kAlloc, stream>>>(tmQ, tmK, tmV, a);
-  return cudaGetLastError();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  return trace_mark(p, 1, stream);
 }
 
 }  // namespace

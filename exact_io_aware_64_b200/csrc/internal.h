@@ -16,7 +16,17 @@ struct Problem {
   float scale;
   int causal;
   unsigned int* err;  // device address of the library's error word
+  // optional kernel-boundary events (fa_trace_events): trace[0] before the first kernel,
+  // trace[k] after the k-th; n_trace entries
+  cudaEvent_t* trace;
+  int n_trace;
 };
+
+// Record trace event k of `p` on `stream` if the caller asked for it.
+inline cudaError_t trace_mark(const Problem& p, int k, cudaStream_t stream) {
+  if (p.trace == nullptr || k >= p.n_trace) return cudaSuccess;
+  return cudaEventRecord(p.trace[k], stream);
+}
 
 // Forward, bf16, tcgen05.  Tensor maps describe Q, K, V as 3-D [BH][N][d] bf16 with
 // 64 x 128 x 1 boxes and the 128-byte swizzle.

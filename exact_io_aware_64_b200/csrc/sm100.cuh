@@ -23,12 +23,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ uint64_t globaltimer_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
@@ -65,11 +59,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Upper bound on any single pipeline wait.  Every wait in these kernels is on work
-// that the same CTA has already issued or will issue within microseconds; a wait
-// this long means the pipeline is broken, so the kernel records an error and winds
-// down instead of spinning forever.
-constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s
+// Upper bound on any single pipeline wait, in SM clock cycles (4 s at 2 GHz, longer at
+// lower clocks).  Every wait in these kernels is on work that the same CTA has already
+// issued or will issue within microseconds; a wait this long means the pipeline is
+// broken, so the kernel records an error and winds down instead of spinning forever.
+constexpr long long kWaitLimitCycles = 8000000000ll;
+// The spin loop looks at the clock and the abort flag only every kSpinCheck tries, so
+// that a completed phase is noticed one try_wait after it completes.
+constexpr uint32_t kSpinCheck = 256;
 
 // Bit set in the library's device error word when a wait runs out of time.
 constexpr unsigned int kErrWaitTimeout = 1u;
@@ -80,28 +77,31 @@ constexpr unsigned int kErrWaitTimeout = 1u;
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           volatile int* abort, unsigned int* err) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      atomicOr(err, kErrWaitTimeout);
-      *abort = 1;
-      return false;
+  const long long t0 = clock64();
+  uint32_t spins = 0;
+  while (!mbar_try_wait(bar, parity)) {
+    if (++spins % kSpinCheck == 0) {
+      if (*abort) return false;
+      if (clock64() - t0 > kWaitLimitCycles) {
+        atomicOr(err, kErrWaitTimeout);
+        *abort = 1;
+        return false;
+      }
     }
   }
+  return true;
 }
 
 // Wait used while winding down after an abort: ignores the abort flag (the point is to
 // let asynchronous work the CTA already issued finish before it exits) but still gives
-// up after kDrainLimitNs.
-constexpr uint64_t kDrainLimitNs = 1000000000ull;  // 1 s
+// up after kDrainLimitCycles.
+constexpr long long kDrainLimitCycles = 2000000000ll;
 
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity,
                                                 unsigned int* err) {
-  const uint64_t t0 = globaltimer_ns();
+  const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > kDrainLimitNs) {
+    if (clock64() - t0 > kDrainLimitCycles) {
       atomicOr(err, kErrWaitTimeout);
       return false;
     }
@@ -149,6 +149,17 @@ __device__ __forceinline__ void tc_fence_before() {
 
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// One arrival per warp instead of one per thread: 128 or 256 threads arriving on the
+// same mbarrier serialise on one shared-memory word.  The calling warp must be
+// converged.  Tensor-memory accesses completed before the call (tcgen05.wait::ld/st)
+// are ordered before the arrival: fence, warp-wide sync, then lane 0 arrives with
+// release semantics.  The barrier's expected count is the number of arriving warps.
+__device__ __forceinline__ void warp_arrive(uint32_t bar) {
+  tc_fence_before();
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
 // D[tmem] (+)= A[smem] * B[smem]

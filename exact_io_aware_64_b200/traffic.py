@@ -55,3 +55,10 @@ def bwd_compulsory_bytes(B: int, H: int, N: int, d: int, elem_bytes: int = 2) ->
     """Bytes the backward must move at least once: read Q, K, V, O, dO, LSE; write dQ, dK,
     dV; write and read D once (fp32)."""
     return 8 * B * H * N * d * elem_bytes + 4 * B * H * N * 3
+
+
+def bwd_prep_bytes(B: int, H: int, N: int, d: int, elem_bytes: int = 2) -> int:
+    """Bytes of the backward's preparation pass: read O and dO and the LSE rows, write D
+    and LSE*log2(e) for every row padded to whole 128-row tiles."""
+    npad = (N + 127) // 128 * 128
+    return 2 * B * H * N * d * elem_bytes + 4 * B * H * N + 8 * B * H * npad

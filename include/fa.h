@@ -143,6 +143,17 @@ FA_API fa_status fa_bwd_noalloc(const void* Q, const void* K, const void* V, con
 /* Size of the fixed scratch array behind fa_bwd_noalloc, in bytes. */
 FA_API size_t fa_bwd_noalloc_max_scratch_bytes(void);
 
+/*
+ * Kernel-boundary timing, for profilers.  While a list of events is set on the calling
+ * thread, every fa_fwd, fa_fwd_f32 and fa_bwd call records events[0] on its stream just
+ * before its first kernel and events[k] just after its k-th kernel; fa_fwd and
+ * fa_fwd_f32 launch one kernel, fa_bwd three (D/LSE preparation, dK/dV, dQ).  Boundaries
+ * beyond n - 1 are not recorded.  The events are caller-created cudaEvent_t (timing
+ * enabled) and stay caller-owned.  fa_trace_events(NULL, 0) stops recording.
+ * Returns FA_ERR_INVALID_ARG if n < 0, n > 8, or events is NULL with n > 0.
+ */
+FA_API fa_status fa_trace_events(cudaEvent_t* events, int n);
+
 /* Static text for a status code ("FA_OK", ...). */
 FA_API const char* fa_status_string(fa_status status);
 

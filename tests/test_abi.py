@@ -124,6 +124,14 @@ def test_bwd_validation(lib):
     assert lib.fa_bwd(*small) != binding.FA_ERR_INVALID_ARG
 
 
+def test_trace_events_validation(lib):
+    assert lib.fa_trace_events(None, 0) == binding.FA_OK
+    assert lib.fa_trace_events(None, 2) == binding.FA_ERR_INVALID_ARG
+    assert lib.fa_trace_events(None, -1) == binding.FA_ERR_INVALID_ARG
+    arr = (ctypes.c_void_p * 9)()
+    assert lib.fa_trace_events(arr, 9) == binding.FA_ERR_INVALID_ARG
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(binding, "_lib", None)
     monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "missing.so"))

@@ -149,3 +149,23 @@ def test_empty_and_lse_optional():
     O1, LSE1 = binding.fwd(q, k, v, causal=True)
     O2, LSE2 = binding.fwd(q, k, v, causal=True, want_lse=False)
     assert LSE2 is None and torch.equal(O1, O2)
+
+
+def test_trace_events_bracket_each_kernel():
+    """fa_trace_events: one boundary before and after the forward kernel, four around the
+    backward's three kernels, all in stream order."""
+    ins = inputs.make_inputs(1, 4, 2048, 128, seed=21, with_dO=True)
+    q, k, v, do = (ins[n].cuda() for n in ("Q", "K", "V", "dO"))
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    with binding.trace_kernels(ev[0:2]):
+        O, LSE = binding.fwd(q, k, v, causal=True)
+    with binding.trace_kernels(ev[2:6]):
+        binding.bwd(q, k, v, O, do, LSE, causal=True)
+    torch.cuda.synchronize()
+    spans = [ev[0].elapsed_time(ev[1])] + [ev[i].elapsed_time(ev[i + 1]) for i in range(2, 5)]
+    assert all(t > 0 for t in spans), spans
+    # outside the context nothing is recorded any more
+    before = ev[1].elapsed_time(ev[2])
+    binding.fwd(q, k, v, causal=True)
+    torch.cuda.synchronize()
+    assert ev[1].elapsed_time(ev[2]) == before
