@@ -189,6 +189,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto wait = [&](uint32_t b, uint32_t parity) -> bool {
     return mbar_wait(b, parity, abort_flag, args.err);
   };
+  // the same for a whole converged warp: every lane gets the same answer
+  auto wait_warp = [&](uint32_t b, uint32_t parity) -> bool {
+    return __all_sync(0xffffffffu, mbar_wait(b, parity, abort_flag, args.err));
+  };
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -231,35 +235,37 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp >= kWarpTMA) regs_dec<kRegsControl>();
   if (warp == kWarpTMA) {
-    if (lane == 0) {
+    // the whole warp runs the loop; one elected lane issues each copy
+    {
       int stage = 0, units = 0, kv_loads = 0;
       uint32_t phase = 0;
       int issued[L::kStages] = {};
       uint32_t issued_phase[L::kStages] = {};
       bool ok = true;
-      for (int w = blockIdx.x; ok && w < args.total_units; w += gridDim.x, ++units) {
+      for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
+         w = snake_unit(++r), ++units) {
         int bh, j, i0;
         unit(w, bh, j, i0);
-        if (units > 0) ok = wait(bar(L::kBarKVEmpty), (units - 1) & 1);
+        if (units > 0) ok = wait_warp(bar(L::kBarKVEmpty), (units - 1) & 1);
         if (!ok) break;
-        mbar_arrive_expect_tx(bar(L::kBarKVFull), 2 * L::kTileBytes);
+        mbar_arrive_expect_tx_elect(bar(L::kBarKVFull), 2 * L::kTileBytes);
         for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(base + L::kK + c * L::kBoxBytes, &tmK, bar(L::kBarKVFull), c * 64, j * kTile, bh);
-          tma_load_3d(base + L::kV + c * L::kBoxBytes, &tmV, bar(L::kBarKVFull), c * 64, j * kTile, bh);
+          tma_load_3d_elect(base + L::kK + c * L::kBoxBytes, &tmK, bar(L::kBarKVFull), c * 64, j * kTile, bh);
+          tma_load_3d_elect(base + L::kV + c * L::kBoxBytes, &tmV, bar(L::kBarKVFull), c * 64, j * kTile, bh);
         }
         ++kv_loads;
         for (int i = i0; ok && i < args.n_tiles; ++i) {
-          ok = wait(bar(L::kBarQEmpty + stage), phase ^ 1);
+          ok = wait_warp(bar(L::kBarQEmpty + stage), phase ^ 1);
           if (!ok) break;
           const uint32_t fb = bar(L::kBarQFull + stage);
           const uint32_t sb = base + L::kStage0 + stage * L::kStageBytes;
-          mbar_arrive_expect_tx(fb, 2 * L::kTileBytes + 1024);
+          mbar_arrive_expect_tx_elect(fb, 2 * L::kTileBytes + 1024);
           for (int c = 0; c < D / 64; ++c) {
-            tma_load_3d(sb + L::kStageQ + c * L::kBoxBytes, &tmQ, fb, c * 64, i * kTile, bh);
-            tma_load_3d(sb + L::kStageDO + c * L::kBoxBytes, &tmdO, fb, c * 64, i * kTile, bh);
+            tma_load_3d_elect(sb + L::kStageQ + c * L::kBoxBytes, &tmQ, fb, c * 64, i * kTile, bh);
+            tma_load_3d_elect(sb + L::kStageDO + c * L::kBoxBytes, &tmdO, fb, c * 64, i * kTile, bh);
           }
-          tma_load_3d(sb + L::kStageL, &tmL2, fb, i * kTile, bh, 0);
-          tma_load_3d(sb + L::kStageD, &tmD, fb, i * kTile, bh, 0);
+          tma_load_3d_elect(sb + L::kStageL, &tmL2, fb, i * kTile, bh, 0);
+          tma_load_3d_elect(sb + L::kStageD, &tmD, fb, i * kTile, bh, 0);
           issued[stage] = 1;
           issued_phase[stage] = phase;
           if (++stage == L::kStages) stage = 0, phase ^= 1;
@@ -273,7 +279,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == kWarpMMA) {
-    if (lane == 0) {
+    // the whole warp runs the loop so descriptors stay warp-uniform; one elected lane
+    // issues each tcgen05 instruction
+    {
       constexpr uint32_t idSS = idesc_bf16_f32(kTile, false);
       constexpr uint32_t idTS = idesc_bf16_f32(D, true);
       const uint64_t dK0 = desc_kmajor(base + L::kK);
@@ -290,24 +298,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = ((kk / 4) * L::kBoxBytes + (kk % 4) * 32) >> 4;
-          mma_ss(dtm, da + off, db + off, idSS, kk > 0 ? 1u : 0u);
+          mma_ss_elect(dtm, da + off, db + off, idSS, kk > 0 ? 1u : 0u);
         }
-        mma_commit(done_bar);
+        mma_commit_elect(done_bar);
       };
       // acc += A(TMEM, 128 x 128 bf16) * B(smem tile, 128 rows x D, MN-major)
       auto issue_ts = [&](uint32_t acc, uint32_t a_tmem, uint32_t b_saddr, bool accumulate) {
         const uint64_t db = desc_mnmajor(b_saddr, L::kBoxBytes);
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ts(acc, split_operand_col(a_tmem, kk), db + static_cast<uint64_t>((kk * 2048) >> 4),
+          mma_ts_elect(acc, split_operand_col(a_tmem, kk), db + static_cast<uint64_t>((kk * 2048) >> 4),
                  idTS, (accumulate || kk > 0) ? 1u : 0u);
       };
-      for (int w = blockIdx.x; ok && w < args.total_units; w += gridDim.x, ++units) {
+      for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
+         w = snake_unit(++r), ++units) {
         int bh, j, i0;
         unit(w, bh, j, i0);
         const int m = args.n_tiles - i0;
-        ok = wait(bar(L::kBarKVFull), units & 1);
-        if (ok) ok = wait(bar(L::kBarQFull + stage), phase);
+        ok = wait_warp(bar(L::kBarKVFull), units & 1);
+        if (ok) ok = wait_warp(bar(L::kBarQFull + stage), phase);
         if (!ok) break;
         tc_fence_after();
         int cur = stage;
@@ -315,37 +324,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_ss(tS, dK0, stage_base(cur) + L::kStageQ, bar(L::kBarSFull));
         issue_ss(tdP, dV0, stage_base(cur) + L::kStageDO, bar(L::kBarDPFull));
         for (int t = 0; t < m; ++t) {
-          ok = wait(bar(L::kBarPReady), p_cnt & 1);
-          if (ok && t == 0 && units > 0) ok = wait(bar(L::kBarAccFree), (units - 1) & 1);
+          ok = wait_warp(bar(L::kBarPReady), p_cnt & 1);
+          if (ok && t == 0 && units > 0) ok = wait_warp(bar(L::kBarAccFree), (units - 1) & 1);
           if (!ok) break;
           ++p_cnt;
           tc_fence_after();
           issue_ts(tdV, tS, stage_base(cur) + L::kStageDO, t > 0);  // dV += P^T dO
           int nxt = -1;
           if (t + 1 < m) {
-            ok = wait(bar(L::kBarQFull + stage), phase);
+            ok = wait_warp(bar(L::kBarQFull + stage), phase);
             if (!ok) break;
             nxt = stage;
             if (++stage == L::kStages) stage = 0, phase ^= 1;
             tc_fence_after();
             issue_ss(tS, dK0, stage_base(nxt) + L::kStageQ, bar(L::kBarSFull));
           }
-          ok = wait(bar(L::kBarDSReady), ds_cnt & 1);
+          ok = wait_warp(bar(L::kBarDSReady), ds_cnt & 1);
           if (!ok) break;
           ++ds_cnt;
           tc_fence_after();
           issue_ts(tdK, tdP, stage_base(cur) + L::kStageQ, t > 0);  // dK += dS^T Q
-          mma_commit(bar(L::kBarQEmpty + cur));
+          mma_commit_elect(bar(L::kBarQEmpty + cur));
           if (nxt >= 0) {
             issue_ss(tdP, dV0, stage_base(nxt) + L::kStageDO, bar(L::kBarDPFull));
             cur = nxt;
           }
         }
         if (!ok) break;
-        mma_commit(bar(L::kBarKVEmpty));
-        mma_commit(bar(L::kBarAccFull));
+        mma_commit_elect(bar(L::kBarKVEmpty));
+        mma_commit_elect(bar(L::kBarAccFull));
       }
-      mma_commit(bar(L::kBarDrain));
+      mma_commit_elect(bar(L::kBarDrain));
       mbar_wait_drain(bar(L::kBarDrain), 0, args.err);
     }
   } else if (warp < kWarpTMA) {
@@ -357,15 +366,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     int stage = 0, units = 0, s_cnt = 0, dp_cnt = 0;
     uint32_t phase = 0;
     bool ok = true;
-    for (int w = blockIdx.x; ok && w < args.total_units; w += gridDim.x, ++units) {
+    for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
+         w = snake_unit(++r), ++units) {
       int bh, j, i0;
       unit(w, bh, j, i0);
       for (int i = i0; i < args.n_tiles; ++i) {
         const uint8_t* sb = smem + L::kStage0 + stage * L::kStageBytes;
         const float* sL = reinterpret_cast<const float*>(sb + L::kStageL) + col0;
         const float* sD = reinterpret_cast<const float*>(sb + L::kStageD) + col0;
-        ok = wait(bar(L::kBarQFull + stage), phase);
-        if (ok) ok = wait(bar(L::kBarSFull), s_cnt & 1);
+        ok = wait_warp(bar(L::kBarQFull + stage), phase);
+        if (ok) ok = wait_warp(bar(L::kBarSFull), s_cnt & 1);
         if (!ok) break;
         ++s_cnt;
         tc_fence_after();
@@ -392,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_wait_st();
         warp_arrive(bar(L::kBarPReady));
-        ok = wait(bar(L::kBarDPFull), dp_cnt & 1);
+        ok = wait_warp(bar(L::kBarDPFull), dp_cnt & 1);
         if (!ok) break;
         ++dp_cnt;
         tc_fence_after();
@@ -419,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       // epilogue: dV and scale * dK for this key row; group g writes columns of its half
-      ok = wait(bar(L::kBarAccFull), units & 1);
+      ok = wait_warp(bar(L::kBarAccFull), units & 1);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
@@ -494,6 +504,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto wait = [&](uint32_t b, uint32_t parity) -> bool {
     return mbar_wait(b, parity, abort_flag, args.err);
   };
+  // the same for a whole converged warp: every lane gets the same answer
+  auto wait_warp = [&](uint32_t b, uint32_t parity) -> bool {
+    return __all_sync(0xffffffffu, mbar_wait(b, parity, abort_flag, args.err));
+  };
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -536,32 +550,34 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp >= kWarpTMA) regs_dec<kRegsControl>();
   if (warp == kWarpTMA) {
-    if (lane == 0) {
+    // the whole warp runs the loop; one elected lane issues each copy
+    {
       int stage = 0, units = 0, q_loads = 0;
       uint32_t phase = 0;
       int issued[L::kStages] = {};
       uint32_t issued_phase[L::kStages] = {};
       bool ok = true;
-      for (int w = blockIdx.x; ok && w < args.total_units; w += gridDim.x, ++units) {
+      for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
+         w = snake_unit(++r), ++units) {
         int bh, i, m;
         unit(w, bh, i, m);
-        if (units > 0) ok = wait(bar(L::kBarQEmpty), (units - 1) & 1);
+        if (units > 0) ok = wait_warp(bar(L::kBarQEmpty), (units - 1) & 1);
         if (!ok) break;
-        mbar_arrive_expect_tx(bar(L::kBarQFull), 2 * L::kTileBytes);
+        mbar_arrive_expect_tx_elect(bar(L::kBarQFull), 2 * L::kTileBytes);
         for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(base + L::kQ + c * L::kBoxBytes, &tmQ, bar(L::kBarQFull), c * 64, i * kTile, bh);
-          tma_load_3d(base + L::kDO + c * L::kBoxBytes, &tmdO, bar(L::kBarQFull), c * 64, i * kTile, bh);
+          tma_load_3d_elect(base + L::kQ + c * L::kBoxBytes, &tmQ, bar(L::kBarQFull), c * 64, i * kTile, bh);
+          tma_load_3d_elect(base + L::kDO + c * L::kBoxBytes, &tmdO, bar(L::kBarQFull), c * 64, i * kTile, bh);
         }
         ++q_loads;
         for (int j = 0; ok && j < m; ++j) {
-          ok = wait(bar(L::kBarKVEmpty + stage), phase ^ 1);
+          ok = wait_warp(bar(L::kBarKVEmpty + stage), phase ^ 1);
           if (!ok) break;
           const uint32_t fb = bar(L::kBarKVFull + stage);
           const uint32_t sb = base + L::kStage0 + stage * L::kStageBytes;
-          mbar_arrive_expect_tx(fb, 2 * L::kTileBytes);
+          mbar_arrive_expect_tx_elect(fb, 2 * L::kTileBytes);
           for (int c = 0; c < D / 64; ++c) {
-            tma_load_3d(sb + L::kStageK + c * L::kBoxBytes, &tmK, fb, c * 64, j * kTile, bh);
-            tma_load_3d(sb + L::kStageV + c * L::kBoxBytes, &tmV, fb, c * 64, j * kTile, bh);
+            tma_load_3d_elect(sb + L::kStageK + c * L::kBoxBytes, &tmK, fb, c * 64, j * kTile, bh);
+            tma_load_3d_elect(sb + L::kStageV + c * L::kBoxBytes, &tmV, fb, c * 64, j * kTile, bh);
           }
           issued[stage] = 1;
           issued_phase[stage] = phase;
@@ -575,7 +591,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == kWarpMMA) {
-    if (lane == 0) {
+    // the whole warp runs the loop so descriptors stay warp-uniform; one elected lane
+    // issues each tcgen05 instruction
+    {
       constexpr uint32_t idSS = idesc_bf16_f32(kTile, false);
       constexpr uint32_t idTS = idesc_bf16_f32(D, true);
       const uint64_t dQd = desc_kmajor(base + L::kQ);
@@ -589,15 +607,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = ((kk / 4) * L::kBoxBytes + (kk % 4) * 32) >> 4;
-          mma_ss(dtm, da + off, db + off, idSS, kk > 0 ? 1u : 0u);
+          mma_ss_elect(dtm, da + off, db + off, idSS, kk > 0 ? 1u : 0u);
         }
-        mma_commit(done_bar);
+        mma_commit_elect(done_bar);
       };
-      for (int w = blockIdx.x; ok && w < args.total_units; w += gridDim.x, ++units) {
+      for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
+         w = snake_unit(++r), ++units) {
         int bh, i, m;
         unit(w, bh, i, m);
-        ok = wait(bar(L::kBarQFull), units & 1);
-        if (ok) ok = wait(bar(L::kBarKVFull + stage), phase);
+        ok = wait_warp(bar(L::kBarQFull), units & 1);
+        if (ok) ok = wait_warp(bar(L::kBarKVFull + stage), phase);
         if (!ok) break;
         tc_fence_after();
         int cur = stage;
@@ -607,8 +626,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < m; ++t) {
           int nxt = -1;
           if (t + 1 < m) {
-            ok = wait(bar(L::kBarKVFull + stage), phase);
-            if (ok) ok = wait(bar(L::kBarSFree), sfree_cnt & 1);
+            ok = wait_warp(bar(L::kBarKVFull + stage), phase);
+            if (ok) ok = wait_warp(bar(L::kBarSFree), sfree_cnt & 1);
             if (!ok) break;
             ++sfree_cnt;
             nxt = stage;
@@ -616,8 +635,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             issue_ss(tS, dQd, stage_base(nxt) + L::kStageK, bar(L::kBarSFull));
           }
-          ok = wait(bar(L::kBarDSReady), ds_cnt & 1);
-          if (ok && t == 0 && units > 0) ok = wait(bar(L::kBarAccFree), (units - 1) & 1);
+          ok = wait_warp(bar(L::kBarDSReady), ds_cnt & 1);
+          if (ok && t == 0 && units > 0) ok = wait_warp(bar(L::kBarAccFree), (units - 1) & 1);
           if (!ok) break;
           ++ds_cnt;
           tc_fence_after();
@@ -625,9 +644,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t db = desc_mnmajor(stage_base(cur) + L::kStageK, L::kBoxBytes);
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
-            mma_ts(tdQ, split_operand_col(tdP, kk), db + static_cast<uint64_t>((kk * 2048) >> 4),
+            mma_ts_elect(tdQ, split_operand_col(tdP, kk), db + static_cast<uint64_t>((kk * 2048) >> 4),
                    idTS, (t > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(bar(L::kBarKVEmpty + cur));
+          mma_commit_elect(bar(L::kBarKVEmpty + cur));
           if (nxt >= 0) {
             issue_ss(tdP, ddO, stage_base(nxt) + L::kStageV, bar(L::kBarDPFull));
             cur = nxt;
@@ -635,13 +654,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
         // the last unit's S tile was read by the element-wise warps: consume that signal
-        ok = wait(bar(L::kBarSFree), sfree_cnt & 1);
+        ok = wait_warp(bar(L::kBarSFree), sfree_cnt & 1);
         if (!ok) break;
         ++sfree_cnt;
-        mma_commit(bar(L::kBarQEmpty));
-        mma_commit(bar(L::kBarAccFull));
+        mma_commit_elect(bar(L::kBarQEmpty));
+        mma_commit_elect(bar(L::kBarAccFull));
       }
-      mma_commit(bar(L::kBarDrain));
+      mma_commit_elect(bar(L::kBarDrain));
       mbar_wait_drain(bar(L::kBarDrain), 0, args.err);
     }
   } else if (warp < kWarpTMA) {
@@ -652,7 +671,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>((warp % 4) * 32) << 16;
     int units = 0, s_cnt = 0, dp_cnt = 0;
     bool ok = true;
-    for (int w = blockIdx.x; ok && w < args.total_units; w += gridDim.x, ++units) {
+    for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
+         w = snake_unit(++r), ++units) {
       int bh, i, m;
       unit(w, bh, i, m);
       const int q_row = i * kTile + row;
@@ -660,7 +680,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float l2 = args.L2pad[prow];
       const float drow = args.Dpad[prow];
       for (int j = 0; j < m; ++j) {
-        ok = wait(bar(L::kBarSFull), s_cnt & 1);
+        ok = wait_warp(bar(L::kBarSFull), s_cnt & 1);
         if (!ok) break;
         ++s_cnt;
         tc_fence_after();
@@ -682,7 +702,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             p[c] = e;
           }
         }
-        ok = wait(bar(L::kBarDPFull), dp_cnt & 1);
+        ok = wait_warp(bar(L::kBarDPFull), dp_cnt & 1);
         if (!ok) break;
         ++dp_cnt;
         tc_fence_after();
@@ -704,7 +724,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         warp_arrive(bar(L::kBarDSReady));
       }
       if (!ok) break;
-      ok = wait(bar(L::kBarAccFull), units & 1);
+      ok = wait_warp(bar(L::kBarAccFull), units & 1);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();

@@ -136,6 +136,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto wait = [&](uint32_t b, uint32_t parity) -> bool {
     return mbar_wait(b, parity, abort_flag, args.err);
   };
+  // the same for a whole converged warp: every lane gets the same answer
+  auto wait_warp = [&](uint32_t b, uint32_t parity) -> bool {
+    return __all_sync(0xffffffffu, mbar_wait(b, parity, abort_flag, args.err));
+  };
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -175,7 +179,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp >= 8) regs_dec<kRegsControl>();
   if (warp == kWarpTMA) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    // (the whole warp runs the loop; one elected lane issues each copy)
+    {
       int stage = 0;
       uint32_t phase = 0;
       int q_uses[2] = {0, 0};
@@ -183,31 +188,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       int issued[L::kStages];
       uint32_t issued_phase[L::kStages];
       for (int s = 0; s < L::kStages; ++s) issued[s] = 0, issued_phase[s] = 0;
-      for (int w = blockIdx.x; ok && w < args.total_units; w += gridDim.x) {
+      for (int r = 0, w = snake_unit(0); ok && w < args.total_units; w = snake_unit(++r)) {
         const UnitInfo ui = unit_info(w, args);
         for (int t = 0; t < 2 && ok; ++t) {
           if (t == 1 && ui.n1 == 0) break;
           if (q_uses[t] > 0)
-            ok = wait(bar(L::kBarQEmpty + t), (q_uses[t] - 1) & 1);
+            ok = wait_warp(bar(L::kBarQEmpty + t), (q_uses[t] - 1) & 1);
           if (!ok) break;
           const uint32_t qb = bar(L::kBarQFull + t);
-          mbar_arrive_expect_tx(qb, L::kTileBytes);
+          mbar_arrive_expect_tx_elect(qb, L::kTileBytes);
           const uint32_t dst = base + (t == 0 ? L::kQ0 : L::kQ1);
           for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(dst + c * L::kBoxBytes, &tmQ, qb, c * 64, (2 * ui.u + t) * kBM, ui.bh);
+            tma_load_3d_elect(dst + c * L::kBoxBytes, &tmQ, qb, c * 64, (2 * ui.u + t) * kBM, ui.bh);
           ++q_uses[t];
         }
         const int n = max(ui.n0, ui.n1);
         for (int j = 0; ok && j < n; ++j) {
           for (int kv = 0; kv < 2; ++kv) {  // K_j then V_j
-            ok = wait(bar(L::kBarKVEmpty + stage), phase ^ 1);
+            ok = wait_warp(bar(L::kBarKVEmpty + stage), phase ^ 1);
             if (!ok) break;
             const uint32_t fb = bar(L::kBarKVFull + stage);
-            mbar_arrive_expect_tx(fb, L::kTileBytes);
+            mbar_arrive_expect_tx_elect(fb, L::kTileBytes);
             const uint32_t dst = base + L::kRing + stage * L::kTileBytes;
             const CUtensorMap* tm = kv == 0 ? &tmK : &tmV;
             for (int c = 0; c < D / 64; ++c)
-              tma_load_3d(dst + c * L::kBoxBytes, tm, fb, c * 64, j * kBN, ui.bh);
+              tma_load_3d_elect(dst + c * L::kBoxBytes, tm, fb, c * 64, j * kBN, ui.bh);
             issued[stage] = 1;
             issued_phase[stage] = phase;
             if (++stage == L::kStages) stage = 0, phase ^= 1;
@@ -225,7 +230,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kWarpMMA) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // (the whole warp runs the loop so descriptors stay warp-uniform; one elected lane
+    // issues each tcgen05 instruction)
+    {
       constexpr uint32_t idS = idesc_bf16_f32(kBN, false);
       constexpr uint32_t idPV = idesc_bf16_f32(D, true);
       int stage = 0;
@@ -235,7 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       auto next_slot = [&](int& slot) -> bool {
         slot = stage;
-        const bool r = wait(bar(L::kBarKVFull + stage), phase);
+        const bool r = wait_warp(bar(L::kBarKVFull + stage), phase);
         if (++stage == L::kStages) stage = 0, phase ^= 1;
         return r;
       };
@@ -254,25 +261,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = ((kk / 4) * L::kBoxBytes + (kk % 4) * 32) >> 4;
-          mma_ss(tS[t], da + off, db + off, idS, kk > 0 ? 1u : 0u);
+          mma_ss_elect(tS[t], da + off, db + off, idS, kk > 0 ? 1u : 0u);
         }
-        mma_commit(bar(L::kBarSFull + t));
+        mma_commit_elect(bar(L::kBarSFull + t));
       };
       auto issue_pv = [&](int t, int vslot, bool accumulate) {
         const uint64_t db = dRingV + static_cast<uint64_t>((vslot * L::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
-          mma_ts(tO[t], tS[t] + kk * 8, db + static_cast<uint64_t>((kk * 2048) >> 4), idPV,
+          mma_ts_elect(tO[t], tS[t] + kk * 8, db + static_cast<uint64_t>((kk * 2048) >> 4), idPV,
                  (accumulate || kk > 0) ? 1u : 0u);
         }
-        mma_commit(bar(L::kBarODone + t));
+        mma_commit_elect(bar(L::kBarODone + t));
       };
-      for (int w = blockIdx.x; ok && w < args.total_units; w += gridDim.x) {
+      for (int r = 0, w = snake_unit(0); ok && w < args.total_units; w = snake_unit(++r)) {
         const UnitInfo ui = unit_info(w, args);
         const int nt[2] = {ui.n0, ui.n1};
         const int n = max(ui.n0, ui.n1);
         for (int t = 0; t < 2 && ok; ++t)
-          if (nt[t] > 0) ok = wait(bar(L::kBarQFull + t), uses[t] & 1);
+          if (nt[t] > 0) ok = wait_warp(bar(L::kBarQFull + t), uses[t] & 1);
         if (!ok) break;
         int kslot;
         ok = next_slot(kslot);
@@ -281,10 +288,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < 2; ++t) {
           if (nt[t] > 0) {
             issue_s(t, kslot);
-            if (nt[t] == 1) mma_commit(bar(L::kBarQEmpty + t));
+            if (nt[t] == 1) mma_commit_elect(bar(L::kBarQEmpty + t));
           }
         }
-        mma_commit(bar(L::kBarKVEmpty + kslot));
+        mma_commit_elect(bar(L::kBarKVEmpty + kslot));
         for (int j = 0; ok && j < n; ++j) {
           int vslot, knext = -1;
           ok = next_slot(vslot);
@@ -292,8 +299,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int t = 0; t < 2 && ok; ++t) {
             if (j >= nt[t]) continue;
             if (j == 0 && uses[t] > 0)
-              ok = wait(bar(L::kBarOFree + t), (uses[t] - 1) & 1);
-            if (ok) ok = wait(bar(L::kBarPReady + t), p_count[t] & 1);
+              ok = wait_warp(bar(L::kBarOFree + t), (uses[t] - 1) & 1);
+            if (ok) ok = wait_warp(bar(L::kBarPReady + t), p_count[t] & 1);
             if (!ok) break;
             ++p_count[t];
             tc_fence_after();
@@ -304,18 +311,18 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (!ok) break;
               tc_fence_after();
               issue_s(t, knext);
-              if (j + 2 == nt[t]) mma_commit(bar(L::kBarQEmpty + t));
+              if (j + 2 == nt[t]) mma_commit_elect(bar(L::kBarQEmpty + t));
             }
           }
           if (!ok) break;
-          mma_commit(bar(L::kBarKVEmpty + vslot));
-          if (knext >= 0) mma_commit(bar(L::kBarKVEmpty + knext));
+          mma_commit_elect(bar(L::kBarKVEmpty + vslot));
+          if (knext >= 0) mma_commit_elect(bar(L::kBarKVEmpty + knext));
         }
         for (int t = 0; t < 2; ++t)
           if (nt[t] > 0) ++uses[t];
       }
       // drain: every MMA issued has completed before TMEM is released
-      mma_commit(bar(L::kBarDrain));
+      mma_commit_elect(bar(L::kBarDrain));
       mbar_wait_drain(bar(L::kBarDrain), 0, args.err);
     }
   } else if (warp < 8) {
@@ -328,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tOrow = tO[t] + lane_off;
     int s_count = 0, o_count = 0;
     bool ok = true;
-    for (int w = blockIdx.x; ok && w < args.total_units; w += gridDim.x) {
+    for (int r = 0, w = snake_unit(0); ok && w < args.total_units; w = snake_unit(++r)) {
       const UnitInfo ui = unit_info(w, args);
       const int n_t = t == 0 ? ui.n0 : ui.n1;
       if (n_t == 0) continue;
@@ -337,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float m = -INFINITY;  // running max, log2 units (scaled logits * log2 e)
       float l = 0.f;
       for (int j = 0; j < n_t; ++j) {
-        ok = wait(bar(L::kBarSFull + t), s_count & 1);
+        ok = wait_warp(bar(L::kBarSFull + t), s_count & 1);
         if (!ok) break;
         ++s_count;
         tc_fence_after();
@@ -377,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (__any_sync(0xffffffffu, rescale && j > 0)) {
           // O_t holds the sum through key tile j-1: wait for that product, then scale
-          ok = wait(bar(L::kBarODone + t), (o_count + j - 1) & 1);
+          ok = wait_warp(bar(L::kBarODone + t), (o_count + j - 1) & 1);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           tc_fence_after();
@@ -412,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       // epilogue: O = acc / l, LSE = (m + log2 l) * ln 2
-      ok = wait(bar(L::kBarODone + t), (o_count + n_t - 1) & 1);
+      ok = wait_warp(bar(L::kBarODone + t), (o_count + n_t - 1) & 1);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       o_count += n_t;
@@ -420,24 +427,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv_l = 1.f / l;
       const int bh = ui.bh;
       __nv_bfloat16* orow = args.O + (static_cast<size_t>(bh) * args.N + q_row) * D;
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tOrow + c * 32, v);
-        tmem_wait_ld();
-        if (q_row < args.N) {
+      // take the whole O row into registers first, so the MMA warp may start the next
+      // unit's first P V product while this row is being converted and stored
+      uint32_t ov[D];
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) tmem_ld32(tOrow + c * 32, &ov[c * 32]);
+      tmem_wait_ld();
+      warp_arrive(bar(L::kBarOFree + t));
+      if (q_row < args.N) {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int k = 0; k < 16; ++k)
-            pk[k] = pack_bf16x2(__uint_as_float(v[2 * k]) * inv_l,
-                                __uint_as_float(v[2 * k + 1]) * inv_l);
+            pk[k] = pack_bf16x2(__uint_as_float(ov[c * 32 + 2 * k]) * inv_l,
+                                __uint_as_float(ov[c * 32 + 2 * k + 1]) * inv_l);
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
         }
       }
-      warp_arrive(bar(L::kBarOFree + t));
       if (args.LSE != nullptr && q_row < args.N)
         args.LSE[static_cast<size_t>(bh) * args.N + q_row] =
             (m + __log2f(l)) * 0.69314718055994531f;

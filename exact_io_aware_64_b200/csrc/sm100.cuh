@@ -109,6 +109,21 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity,
   return true;
 }
 
+// ---------------------------------------------------------------- elected issue
+// The TMA and MMA roles run as whole, converged warps so that the values they compute
+// (addresses, descriptors) stay warp-uniform and live in uniform registers; the
+// instructions that must come from one thread are issued by the lane that elect.sync
+// picks, inside the same asm statement, so no divergent branch breaks that uniformity.
+
+__device__ __forceinline__ void mbar_arrive_expect_tx_elect(uint32_t bar, uint32_t bytes) {
+  asm volatile(
+      "{\n\t.reg .pred P1;\n\t.reg .b64 st;\n\t"
+      "elect.sync _|P1, 0xffffffff;\n\t"
+      "@P1 mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(bar),
+      "r"(bytes)
+      : "memory");
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
@@ -121,6 +136,18 @@ __device__ __forceinline__ void tma_load_3d(uint32_t smem_dst, const void* tmap,
   asm volatile(
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_dst),
+      "l"(tmap), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+// tma_load_3d issued by one elected lane of a converged warp.
+__device__ __forceinline__ void tma_load_3d_elect(uint32_t smem_dst, const void* tmap,
+                                                  uint32_t bar, int c0, int c1, int c2) {
+  asm volatile(
+      "{\n\t.reg .pred P1;\n\t"
+      "elect.sync _|P1, 0xffffffff;\n\t"
+      "@P1 cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];\n\t}" ::"r"(smem_dst),
       "l"(tmap), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
@@ -181,6 +208,38 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Elected-lane forms of the MMA and commit, for a converged warp.
+__device__ __forceinline__ void mma_ss_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, P1;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|P1, 0xffffffff;\n\t"
+      "@P1 tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, P1;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|P1, 0xffffffff;\n\t"
+      "@P1 tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit_elect(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred P1;\n\t"
+      "elect.sync _|P1, 0xffffffff;\n\t"
+      "@P1 tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+          bar)
       : "memory");
 }
 
@@ -290,6 +349,17 @@ __device__ __forceinline__ void regs_dec() {
 template <int N>
 __device__ __forceinline__ void regs_inc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// ---------------------------------------------------------------- persistent schedule
+// Index of this CTA's r-th work unit when the units are listed heaviest first and dealt
+// to the CTAs in boustrophedon order (round 0 left to right, round 1 right to left, ...),
+// which evens out the per-CTA sums far better than plain round robin when unit costs
+// fall steadily (causal masking).  The sequence increases with r; the first index at or
+// past the unit count ends the CTA's work.
+__device__ __forceinline__ int snake_unit(int r) {
+  const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+  return r * G + ((r & 1) ? G - 1 - c : c);
 }
 
 // ---------------------------------------------------------------- math
