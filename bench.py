@@ -34,6 +34,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from exact_io_aware_64_b200 import dist as fa_dist  # noqa: E402
 from exact_io_aware_64_b200 import inputs as fa_inputs  # noqa: E402
 from exact_io_aware_64_b200 import traffic  # noqa: E402
 
@@ -134,36 +135,6 @@ class ClockSampler:
                 "power_w_max": max(power) if power else None}
 
 
-def dist_setup(n_gpus: int):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(0)
-    return rank, world, local
-
-
-def barrier(world):
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-
-
-def max_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch.distributed as dist
-    t = torch.tensor([x], device="cuda", dtype=torch.float64)
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
-
-
 def step_flops(w) -> float:
     return traffic.fwd_flops(w.B, w.H, w.N, w.d, w.causal) + \
         traffic.bwd_flops(w.B, w.H, w.N, w.d, w.causal)
@@ -232,11 +203,14 @@ def run_reference(args, w):
 # ------------------------------------------------------------------ GPU arm
 def run_gpu(args, w):
     from exact_io_aware_64_b200 import binding
-    rank, world, local = dist_setup(args.gpus)
+    info = fa_dist.rank_info()
+    fa_dist.init(info, "nccl")
+    rank, world, local = info.rank, info.world, info.local_rank
+    torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     B, H, N, d = w.B, w.H, w.N, w.d
     with_bwd = not args.fwd_only
-    ins = fa_inputs.make_inputs(B, H, N, d, w.seed + 101 * rank, sigma_qk=w.sigma_qk,
+    ins = fa_inputs.make_inputs(B, H, N, d, fa_dist.replica_seed(w.seed, info), sigma_qk=w.sigma_qk,
                                 sigma_v=w.sigma_v, with_dO=True, device=str(dev))
     q, k, v, do = ins["Q"], ins["K"], ins["V"], ins["dO"]
     O = torch.empty_like(q)
@@ -268,7 +242,7 @@ def run_gpu(args, w):
         step()
     binding.check_device_error()
     marks = [[ev() for _ in range(6)] for _ in range(args.steps)]
-    barrier(world)
+    fa_dist.barrier(info)
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
         start, end = ev(), ev()
@@ -277,10 +251,10 @@ def run_gpu(args, w):
             step(marks[i])
         end.record(stream)
         torch.cuda.synchronize()
-    barrier(world)
+    fa_dist.barrier(info)
     binding.check_device_error()
     ms_local = start.elapsed_time(end) / args.steps
-    ms = max_over_ranks(ms_local, world)
+    ms = fa_dist.max_over_ranks(ms_local, info, device=str(dev))
     def span(a, b):
         return statistics.mean(m[a].elapsed_time(m[b]) for m in marks)
 
@@ -302,7 +276,7 @@ def run_gpu(args, w):
             kinfo["tflops"] = kinfo["flops"] / (kinfo["ms"] * 1e-3) / 1e12
         else:
             kinfo["gbs"] = kinfo["bytes"] / (kinfo["ms"] * 1e-3) / 1e9
-    value = world * (f_fwd + f_bwd) / (ms * 1e-3) / 1e12
+    value = fa_dist.aggregate_throughput(f_fwd + f_bwd, ms * 1e-3, info) / 1e12
 
     # ---- end to end through the public API with host buffers
     pin = lambda t: t.detach().to("cpu").pin_memory()  # noqa: E731
@@ -326,7 +300,7 @@ def run_gpu(args, w):
     for _ in range(2):
         e2e_step()
     torch.cuda.synchronize()
-    barrier(world)
+    fa_dist.barrier(info)
     e0, e1 = ev(), ev()
     e0.record(stream)
     e2e_steps = max(2, min(args.steps, 10))
@@ -334,13 +308,11 @@ def run_gpu(args, w):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
-    e2e_value = world * (f_fwd + f_bwd) / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = fa_dist.max_over_ranks(e0.elapsed_time(e1) / e2e_steps, info, device=str(dev))
+    e2e_value = fa_dist.aggregate_throughput(f_fwd + f_bwd, e2e_ms * 1e-3, info) / 1e12
 
     if rank != 0:
-        if world > 1:
-            import torch.distributed as dist
-            dist.destroy_process_group()
+        fa_dist.shutdown(info)
         return 0
 
     peaks, peak_src = load_peaks()
@@ -377,9 +349,7 @@ def run_gpu(args, w):
         line["cpu_baseline"] = {"value": v_cpu, "unit": "TFLOP/s", "cores": threads,
                                 "kind": "oracle", "sample": sample}
     print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    fa_dist.shutdown(info)
     return 0
 
 
