@@ -34,11 +34,12 @@ FLAGS = [
 
 
 def _digest(paths) -> str:
+    """Hash of the sources and flags, independent of where the tree is checked out."""
     h = hashlib.sha256()
     for p in paths:
         with open(p, "rb") as f:
-            h.update(p.encode() + b"\0" + f.read())
-    h.update(" ".join(FLAGS).encode())
+            h.update(os.path.relpath(p, ROOT).encode() + b"\0" + f.read())
+    h.update(" ".join(FLAGS).replace(ROOT, "<root>").encode())
     return h.hexdigest()
 
 

@@ -19,8 +19,10 @@
 //          dS^T = P^T * (dP^T - D_i)
 //          dV_j += P^T dO_i,  dK_j += dS^T Q_i             (TS MMAs, P^T/dS^T from TMEM)
 //      TMEM: dV | dK | S^T (P^T over its first 64 columns) | dP^T (dS^T likewise).
-//   3. bwd_dq: one work unit per (batch*head, 128-row query tile i); key/value tiles
-//      stream past:  S = Q_i K_j^T, dP = dO_i V_j^T, P, dS as above, dQ_i += dS K_j.
+//   3. bwd_dq: one work unit per (batch*head, 128-row query tile i); key and value tiles
+//      stream past through separate rings (3 slots for K, which the last product of a
+//      tile still reads, 2 for V):  S = Q_i K_j^T, dP = dO_i V_j^T, P, dS as above,
+//      dQ_i += dS K_j.
 //      TMEM: dQ | S | dP (dS over its first 64 columns).
 //
 // Both tensor-core kernels are persistent (one CTA per SM) with 384 threads: warps 0-7
@@ -461,29 +463,34 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ------------------------------------------------------------------ 3. dQ
 template <int D>
 struct DqLayout {
+  // Q_i and dO_i stay for the whole unit; K_j and V_j stream through separate rings.
+  // K_j is read until the dQ product of its tile, V_j only by the dP product, so K gets
+  // one more slot: both are then loaded a tile and a half before they are needed.
   static constexpr int kTileBytes = kTile * D * 2;
   static constexpr int kBoxBytes = 128 * 128;
-  static constexpr int kStages = 2;
+  static constexpr int kKStages = 3;
+  static constexpr int kVStages = 2;
   static constexpr int kQ = 0;
   static constexpr int kDO = kTileBytes;
-  static constexpr int kStage0 = 2 * kTileBytes;
-  static constexpr int kStageK = 0;
-  static constexpr int kStageV = kTileBytes;
-  static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kBar = kStage0 + kStages * kStageBytes;
+  static constexpr int kK0 = 2 * kTileBytes;
+  static constexpr int kV0 = kK0 + kKStages * kTileBytes;
+  static constexpr int kBar = kV0 + kVStages * kTileBytes;
   static constexpr int kBarQFull = 0, kBarQEmpty = 1;
-  static constexpr int kBarKVFull = 2;              // [kStages]
-  static constexpr int kBarKVEmpty = 2 + kStages;   // [kStages]
-  static constexpr int kBarSFull = 2 + 2 * kStages;
-  static constexpr int kBarSFree = 3 + 2 * kStages;
-  static constexpr int kBarDPFull = 4 + 2 * kStages;
-  static constexpr int kBarDSReady = 5 + 2 * kStages;
-  static constexpr int kBarAccFull = 6 + 2 * kStages;
-  static constexpr int kBarAccFree = 7 + 2 * kStages;
-  static constexpr int kBarDrain = 8 + 2 * kStages;
-  static constexpr int kNumBars = 9 + 2 * kStages;
+  static constexpr int kBarKFull = 2;                          // [kKStages]
+  static constexpr int kBarKEmpty = kBarKFull + kKStages;      // [kKStages]
+  static constexpr int kBarVFull = kBarKEmpty + kKStages;      // [kVStages]
+  static constexpr int kBarVEmpty = kBarVFull + kVStages;      // [kVStages]
+  static constexpr int kBarSFull = kBarVEmpty + kVStages;
+  static constexpr int kBarSFree = kBarSFull + 1;
+  static constexpr int kBarDPFull = kBarSFull + 2;
+  static constexpr int kBarDSReady = kBarSFull + 3;
+  static constexpr int kBarAccFull = kBarSFull + 4;
+  static constexpr int kBarAccFree = kBarSFull + 5;
+  static constexpr int kBarDrain = kBarSFull + 6;
+  static constexpr int kNumBars = kBarDrain + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kAlloc = kMisc + 16 + 1024;
+  static_assert(kAlloc <= 232448, "shared memory over the 227 KB per-block limit");
 };
 
 template <int D>
@@ -513,9 +520,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     mbar_init(bar(L::kBarQFull), 1);
     mbar_init(bar(L::kBarQEmpty), 1);
-    for (int s = 0; s < L::kStages; ++s) {
-      mbar_init(bar(L::kBarKVFull + s), 1);
-      mbar_init(bar(L::kBarKVEmpty + s), 1);
+    for (int s = 0; s < L::kKStages; ++s) {
+      mbar_init(bar(L::kBarKFull + s), 1);
+      mbar_init(bar(L::kBarKEmpty + s), 1);
+    }
+    for (int s = 0; s < L::kVStages; ++s) {
+      mbar_init(bar(L::kBarVFull + s), 1);
+      mbar_init(bar(L::kBarVEmpty + s), 1);
     }
     mbar_init(bar(L::kBarSFull), 1);
     mbar_init(bar(L::kBarSFree), kEw / 32);
@@ -552,10 +563,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kWarpTMA) {
     // the whole warp runs the loop; one elected lane issues each copy
     {
-      int stage = 0, units = 0, q_loads = 0;
-      uint32_t phase = 0;
-      int issued[L::kStages] = {};
-      uint32_t issued_phase[L::kStages] = {};
+      int ks = 0, vs = 0, units = 0, q_loads = 0;
+      uint32_t kph = 0, vph = 0;
+      int k_issued[L::kKStages] = {}, v_issued[L::kVStages] = {};
+      uint32_t k_phase[L::kKStages] = {}, v_phase[L::kVStages] = {};
       bool ok = true;
       for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
          w = snake_unit(++r), ++units) {
@@ -570,23 +581,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ++q_loads;
         for (int j = 0; ok && j < m; ++j) {
-          ok = wait_warp(bar(L::kBarKVEmpty + stage), phase ^ 1);
+          ok = wait_warp(bar(L::kBarKEmpty + ks), kph ^ 1);
           if (!ok) break;
-          const uint32_t fb = bar(L::kBarKVFull + stage);
-          const uint32_t sb = base + L::kStage0 + stage * L::kStageBytes;
-          mbar_arrive_expect_tx_elect(fb, 2 * L::kTileBytes);
-          for (int c = 0; c < D / 64; ++c) {
-            tma_load_3d_elect(sb + L::kStageK + c * L::kBoxBytes, &tmK, fb, c * 64, j * kTile, bh);
-            tma_load_3d_elect(sb + L::kStageV + c * L::kBoxBytes, &tmV, fb, c * 64, j * kTile, bh);
-          }
-          issued[stage] = 1;
-          issued_phase[stage] = phase;
-          if (++stage == L::kStages) stage = 0, phase ^= 1;
+          mbar_arrive_expect_tx_elect(bar(L::kBarKFull + ks), L::kTileBytes);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d_elect(base + L::kK0 + ks * L::kTileBytes + c * L::kBoxBytes, &tmK,
+                              bar(L::kBarKFull + ks), c * 64, j * kTile, bh);
+          k_issued[ks] = 1;
+          k_phase[ks] = kph;
+          if (++ks == L::kKStages) ks = 0, kph ^= 1;
+          ok = wait_warp(bar(L::kBarVEmpty + vs), vph ^ 1);
+          if (!ok) break;
+          mbar_arrive_expect_tx_elect(bar(L::kBarVFull + vs), L::kTileBytes);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d_elect(base + L::kV0 + vs * L::kTileBytes + c * L::kBoxBytes, &tmV,
+                              bar(L::kBarVFull + vs), c * 64, j * kTile, bh);
+          v_issued[vs] = 1;
+          v_phase[vs] = vph;
+          if (++vs == L::kVStages) vs = 0, vph ^= 1;
         }
       }
       if (!ok) {
-        for (int s = 0; s < L::kStages; ++s)
-          if (issued[s]) mbar_wait_drain(bar(L::kBarKVFull + s), issued_phase[s], args.err);
+        // let the loads already issued land before the CTA exits
+        for (int s = 0; s < L::kKStages; ++s)
+          if (k_issued[s]) mbar_wait_drain(bar(L::kBarKFull + s), k_phase[s], args.err);
+        for (int s = 0; s < L::kVStages; ++s)
+          if (v_issued[s]) mbar_wait_drain(bar(L::kBarVFull + s), v_phase[s], args.err);
         if (q_loads > 0) mbar_wait_drain(bar(L::kBarQFull), (q_loads - 1) & 1, args.err);
       }
     }
@@ -598,10 +618,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idTS = idesc_bf16_f32(D, true);
       const uint64_t dQd = desc_kmajor(base + L::kQ);
       const uint64_t ddO = desc_kmajor(base + L::kDO);
-      int stage = 0, units = 0, sfree_cnt = 0, ds_cnt = 0;
-      uint32_t phase = 0;
+      int kc = 0, vc = 0, units = 0, sfree_cnt = 0, ds_cnt = 0;
+      uint32_t kcph = 0, vcph = 0;
       bool ok = true;
-      auto stage_base = [&](int s) { return base + L::kStage0 + s * L::kStageBytes; };
+      auto kslot = [&](int s) { return base + L::kK0 + s * L::kTileBytes; };
+      auto vslot = [&](int s) { return base + L::kV0 + s * L::kTileBytes; };
+      // S = Q K^T or dP = dO V^T: both operands K-major, K extent = D
       auto issue_ss = [&](uint32_t dtm, uint64_t da, uint32_t b_saddr, uint32_t done_bar) {
         const uint64_t db = desc_kmajor(b_saddr);
 #pragma unroll
@@ -611,29 +633,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit_elect(done_bar);
       };
+      // dP = dO V^T into TMEM, then release V's slot once that product completes
+      auto issue_dp = [&]() -> bool {
+        if (!wait_warp(bar(L::kBarVFull + vc), vcph)) return false;
+        tc_fence_after();
+        issue_ss(tdP, ddO, vslot(vc), bar(L::kBarDPFull));
+        mma_commit_elect(bar(L::kBarVEmpty + vc));
+        if (++vc == L::kVStages) vc = 0, vcph ^= 1;
+        return true;
+      };
       for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
          w = snake_unit(++r), ++units) {
         int bh, i, m;
         unit(w, bh, i, m);
         ok = wait_warp(bar(L::kBarQFull), units & 1);
-        if (ok) ok = wait_warp(bar(L::kBarKVFull + stage), phase);
+        if (ok) ok = wait_warp(bar(L::kBarKFull + kc), kcph);
         if (!ok) break;
         tc_fence_after();
-        int cur = stage;
-        if (++stage == L::kStages) stage = 0, phase ^= 1;
-        issue_ss(tS, dQd, stage_base(cur) + L::kStageK, bar(L::kBarSFull));
-        issue_ss(tdP, ddO, stage_base(cur) + L::kStageV, bar(L::kBarDPFull));
+        int cur = kc;
+        if (++kc == L::kKStages) kc = 0, kcph ^= 1;
+        issue_ss(tS, dQd, kslot(cur), bar(L::kBarSFull));
+        ok = issue_dp();
+        if (!ok) break;
         for (int t = 0; t < m; ++t) {
           int nxt = -1;
           if (t + 1 < m) {
-            ok = wait_warp(bar(L::kBarKVFull + stage), phase);
+            ok = wait_warp(bar(L::kBarKFull + kc), kcph);
             if (ok) ok = wait_warp(bar(L::kBarSFree), sfree_cnt & 1);
             if (!ok) break;
             ++sfree_cnt;
-            nxt = stage;
-            if (++stage == L::kStages) stage = 0, phase ^= 1;
+            nxt = kc;
+            if (++kc == L::kKStages) kc = 0, kcph ^= 1;
             tc_fence_after();
-            issue_ss(tS, dQd, stage_base(nxt) + L::kStageK, bar(L::kBarSFull));
+            issue_ss(tS, dQd, kslot(nxt), bar(L::kBarSFull));
           }
           ok = wait_warp(bar(L::kBarDSReady), ds_cnt & 1);
           if (ok && t == 0 && units > 0) ok = wait_warp(bar(L::kBarAccFree), (units - 1) & 1);
@@ -641,14 +673,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++ds_cnt;
           tc_fence_after();
           // dQ += dS K_j: A = dS (TMEM), B = K_j (128 key rows x D, MN-major)
-          const uint64_t db = desc_mnmajor(stage_base(cur) + L::kStageK, L::kBoxBytes);
+          const uint64_t db = desc_mnmajor(kslot(cur), L::kBoxBytes);
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
             mma_ts_elect(tdQ, split_operand_col(tdP, kk), db + static_cast<uint64_t>((kk * 2048) >> 4),
-                   idTS, (t > 0 || kk > 0) ? 1u : 0u);
-          mma_commit_elect(bar(L::kBarKVEmpty + cur));
+                         idTS, (t > 0 || kk > 0) ? 1u : 0u);
+          mma_commit_elect(bar(L::kBarKEmpty + cur));
           if (nxt >= 0) {
-            issue_ss(tdP, ddO, stage_base(nxt) + L::kStageV, bar(L::kBarDPFull));
+            ok = issue_dp();
+            if (!ok) break;
             cur = nxt;
           }
         }
