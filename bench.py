@@ -353,6 +353,62 @@ def run_gpu(args, w):
     return 0
 
 
+# ------------------------------------------------------------------ N sweep
+SWEEP_N = (256, 512, 1024, 2048, 4096, 8192, 16384, 32768)
+
+
+def run_sweep(args):
+    """TFLOP/s of fa_fwd and fa_bwd against N (the metric's "vs N"): B*N = 16384 tokens
+    (B = max(1, 16384 / N)), H = 2048 / d, d in {64, 128}, causal in {0, 1}, bf16.
+    Each call is timed alone with CUDA events; for N <= 1024 a 256 MB buffer is
+    rewritten between calls so every call starts with a cold L2.  One JSON line per
+    point."""
+    from exact_io_aware_64_b200 import binding
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    peaks, peak_src = load_peaks()
+    peak = peaks["bf16_tflops"]
+    for d in (64, 128):
+        for causal in (False, True):
+            for N in SWEEP_N:
+                B, H = max(1, 16384 // N), 2048 // d
+                ins = fa_inputs.make_inputs(B, H, N, d, seed=N + d, with_dO=True, device="cuda")
+                q, k, v, do = ins["Q"], ins["K"], ins["V"], ins["dO"]
+                O = torch.empty_like(q)
+                LSE = torch.empty((B, H, N), device=dev, dtype=torch.float32)
+                dQ, dK, dV = (torch.empty_like(q) for _ in range(3))
+                ws = torch.empty(max(binding.workspace_bytes(B, H, N, d), 1), device=dev,
+                                 dtype=torch.uint8)
+                fwd = lambda: binding.fwd(q, k, v, causal=causal, O=O, LSE=LSE)  # noqa: E731
+                bwd = lambda: binding.bwd(q, k, v, O, do, LSE, causal=causal, dQ=dQ,  # noqa: E731
+                                          dK=dK, dV=dV, workspace=ws)
+                res = {}
+                for name, fn, flops in (("fwd", fwd, traffic.fwd_flops(B, H, N, d, causal)),
+                                        ("bwd", bwd, traffic.bwd_flops(B, H, N, d, causal))):
+                    for _ in range(args.warmup):
+                        fn()
+                    times = []
+                    for _ in range(args.steps):
+                        if N <= 1024:
+                            flush.fill_(1)
+                        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                        e0.record()
+                        fn()
+                        e1.record()
+                        torch.cuda.synchronize()
+                        times.append(e0.elapsed_time(e1))
+                    ms = statistics.median(times)
+                    res[name] = {"ms": ms, "tflops": flops / (ms * 1e-3) / 1e12,
+                                 "frac": flops / (ms * 1e-3) / 1e12 / peak}
+                binding.check_device_error()
+                print(json.dumps({"sweep": "attention TFLOP/s vs N", "N": N, "B": B, "H": H, "d": d,
+                                  "causal": causal, "dtype": "bf16", "peak": peak,
+                                  "peak_source": f"{peak_src} burst bf16", **res}), flush=True)
+                del ins, q, k, v, do, O, LSE, dQ, dK, dV, ws
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -364,6 +420,8 @@ def main():
     ap.add_argument("--sustained-peak", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=20.0)
+    ap.add_argument("--sweep", action="store_true",
+                    help="print TFLOP/s of fa_fwd and fa_bwd against N instead of the step")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -372,6 +430,8 @@ def main():
         ap.error("the benchmark runs the bf16 path")
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.sweep:
+        return run_sweep(args)
     return run_gpu(args, w)
 
 

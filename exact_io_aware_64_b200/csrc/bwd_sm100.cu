@@ -23,7 +23,8 @@
 //      stream past through separate rings (3 slots for K, which the last product of a
 //      tile still reads, 2 for V):  S = Q_i K_j^T, dP = dO_i V_j^T, P, dS as above,
 //      dQ_i += dS K_j.
-//      TMEM: dQ | S | dP (dS over its first 64 columns).
+//      TMEM: dQ | S | dP | dS.  dS has its own region, so S(j+1) and dP(j+1) are issued
+//      as soon as the element-wise warps have read S(j) and dP(j), ahead of dQ(j).
 //
 // Both tensor-core kernels are persistent (one CTA per SM) with 384 threads: warps 0-7
 // are two element-wise warpgroups that split every 128 x 128 tile by columns (group g
@@ -33,7 +34,7 @@
 // each other's TMEM, and the MMA reads the bf16 operand as two 32-column pieces.  The MMA order is chosen so the
 // tensor core works on one product while the element-wise warps build the next operand
 // (dK/dV: S^T(i) dP^T(i) | dV(i) S^T(i+1) | dK(i) dP^T(i+1) | ...;
-//  dQ: S(j) dP(j) | S(j+1) | dQ(j) dP(j+1) | S(j+2) | ...).
+//  dQ: S(j) dP(j) | S(j+1) dP(j+1) | dQ(j) | S(j+2) dP(j+2) | dQ(j+1) ...).
 // Causal work units are ordered heaviest first.
 #include <cstdint>
 
@@ -68,48 +69,67 @@ __device__ __forceinline__ uint32_t split_operand_col(uint32_t base, int kk) {
 }
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
+// Every kPolyEvery-th exponential of a row may be computed on the FMA pipe (exp2_poly)
+// instead of the MUFU unit; masked entries are zeroed after the exponential either way.
+// Measured on B200 at 1-in-2 and 1-in-4 it made the backward slower, so 0: off.
+constexpr int kPolyEvery = 0;
+constexpr int kPolyStride = kPolyEvery > 0 ? kPolyEvery : 1;
 
 __host__ __device__ constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
 // ------------------------------------------------------------------ 1. preparation
 // D[bh][r] = sum_k dO[bh][r][k] * O[bh][r][k];  L2[bh][r] = LSE[bh][r] * log2(e).
-// Padded rows r in [N, Npad): D = 0, L2 = +inf.  One warp per row, 16-byte loads.
+// Padded rows r in [N, Npad): D = 0, L2 = +inf.  Bandwidth bound: each thread reads 16
+// bytes of O and of dO for kRowsPerThread rows (independent loads in flight), the
+// D / 8 threads of a row combine their partial sums with shuffles.
+constexpr int kPrepThreads = 256;
+constexpr int kPrepRowsPerThread = 4;
+
 template <int D>
-__global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __restrict__ O,
-                                                       const __nv_bfloat16* __restrict__ dO,
-                                                       const float* __restrict__ LSE,
-                                                       float* __restrict__ Dout,
-                                                       float* __restrict__ L2out, int BH,
-                                                       int N, int Npad) {
-  const long long row = static_cast<long long>(blockIdx.x) * 8 + threadIdx.x / 32;
-  const int lane = threadIdx.x % 32;
-  if (row >= static_cast<long long>(BH) * Npad) return;
-  const int bh = static_cast<int>(row / Npad);
-  const int r = static_cast<int>(row % Npad);
-  float acc = 0.f;
-  if (r < N) {
-    const size_t base = (static_cast<size_t>(bh) * N + r) * D;
-    constexpr int kVec = 8;  // bf16 per 16-byte load
-    for (int c = lane * kVec; c < D; c += 32 * kVec) {
-      const uint4 a = *reinterpret_cast<const uint4*>(O + base + c);
-      const uint4 b = *reinterpret_cast<const uint4*>(dO + base + c);
+__global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(
+    const __nv_bfloat16* __restrict__ O, const __nv_bfloat16* __restrict__ dO,
+    const float* __restrict__ LSE, float* __restrict__ Dout, float* __restrict__ L2out, int BH,
+    int N, int Npad) {
+  constexpr int kPer = D / 8;                         // threads per row (8 bf16 each)
+  constexpr int kRowsPerPass = kPrepThreads / kPer;   // rows covered by one pass
+  const int part = threadIdx.x % kPer;
+  const long long total = static_cast<long long>(BH) * Npad;
+  const long long row0 = (static_cast<long long>(blockIdx.x) * kPrepRowsPerThread) * kRowsPerPass +
+                         threadIdx.x / kPer;
+  float acc[kPrepRowsPerThread];
+#pragma unroll
+  for (int k = 0; k < kPrepRowsPerThread; ++k) {
+    acc[k] = 0.f;
+    const long long row = row0 + static_cast<long long>(k) * kRowsPerPass;
+    if (row >= total) continue;
+    const int bh = static_cast<int>(row / Npad);
+    const int r = static_cast<int>(row % Npad);
+    if (r < N) {
+      const size_t off = (static_cast<size_t>(bh) * N + r) * D + part * 8;
+      const uint4 a = *reinterpret_cast<const uint4*>(O + off);
+      const uint4 b = *reinterpret_cast<const uint4*>(dO + off);
       const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
       const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float2 fa = __bfloat1622float2(pa[k]);
-        const float2 fb = __bfloat1622float2(pb[k]);
-        acc = fmaf(fa.x, fb.x, acc);
-        acc = fmaf(fa.y, fb.y, acc);
+      for (int e = 0; e < 4; ++e) {
+        const float2 fa = __bfloat1622float2(pa[e]);
+        const float2 fb = __bfloat1622float2(pb[e]);
+        acc[k] = fmaf(fa.x, fb.x, acc[k]);
+        acc[k] = fmaf(fa.y, fb.y, acc[k]);
       }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
   }
-  if (lane == 0) {
-    const size_t out = static_cast<size_t>(bh) * Npad + r;
-    Dout[out] = acc;
-    L2out[out] = r < N ? LSE[static_cast<size_t>(bh) * N + r] * kLog2e : INFINITY;
+#pragma unroll
+  for (int k = 0; k < kPrepRowsPerThread; ++k) {
+#pragma unroll
+    for (int o = kPer / 2; o > 0; o >>= 1) acc[k] += __shfl_xor_sync(0xffffffffu, acc[k], o);
+    const long long row = row0 + static_cast<long long>(k) * kRowsPerPass;
+    if (part == 0 && row < total) {
+      const int bh = static_cast<int>(row / Npad);
+      const int r = static_cast<int>(row % Npad);
+      Dout[row] = acc[k];
+      L2out[row] = r < N ? LSE[static_cast<size_t>(bh) * N + r] * kLog2e : INFINITY;
+    }
   }
 }
 
@@ -144,32 +164,42 @@ __device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t* 
 // ------------------------------------------------------------------ 2. dK, dV
 template <int D>
 struct DkdvLayout {
+  // K_j and V_j stay for the whole unit.  Query tiles stream through two rings: Q_i
+  // (3 slots; its last reader is the dK product) and dO_i together with the tile's
+  // LSE*log2(e) and D rows (2 slots; read by dP^T, dV and the element-wise warps).
+  // With 3 Q slots the next query tile is loaded a full tile ahead of the S^T product
+  // that needs it.  The layout uses 231.6 KB of the 227 KB (232448 B) a CTA may have,
+  // so it leaves no slack for aligning the base: the kernel checks that the dynamic
+  // shared memory starts on a 1024-byte boundary (the 128-byte swizzle atoms need it)
+  // and reports kErrSmemAlign instead of running if it does not.
   static constexpr int kTileBytes = kTile * D * 2;
   static constexpr int kBoxBytes = 128 * 128;
-  static constexpr int kStages = 2;
+  static constexpr int kQStages = 3;
+  static constexpr int kDOStages = 2;
   static constexpr int kK = 0;
   static constexpr int kV = kTileBytes;
-  static constexpr int kStage0 = 2 * kTileBytes;
-  // per stage: Q tile, dO tile, L2 row (512 B), D row (512 B)
-  static constexpr int kStageQ = 0;
-  static constexpr int kStageDO = kTileBytes;
-  static constexpr int kStageL = 2 * kTileBytes;
-  static constexpr int kStageD = 2 * kTileBytes + 512;
-  static constexpr int kStageBytes = 2 * kTileBytes + 1024;
-  static constexpr int kBar = kStage0 + kStages * kStageBytes;
+  static constexpr int kQ0 = 2 * kTileBytes;
+  static constexpr int kDO0 = kQ0 + kQStages * kTileBytes;
+  static constexpr int kDOSlotBytes = kTileBytes + 1024;  // dO tile, L2 row, D row
+  static constexpr int kSlotL = kTileBytes;
+  static constexpr int kSlotD = kTileBytes + 512;
+  static constexpr int kBar = kDO0 + kDOStages * kDOSlotBytes;
   static constexpr int kBarKVFull = 0, kBarKVEmpty = 1;
-  static constexpr int kBarQFull = 2;                 // [kStages]
-  static constexpr int kBarQEmpty = 2 + kStages;      // [kStages]
-  static constexpr int kBarSFull = 2 + 2 * kStages;
-  static constexpr int kBarDPFull = 3 + 2 * kStages;
-  static constexpr int kBarPReady = 4 + 2 * kStages;
-  static constexpr int kBarDSReady = 5 + 2 * kStages;
-  static constexpr int kBarAccFull = 6 + 2 * kStages;
-  static constexpr int kBarAccFree = 7 + 2 * kStages;
-  static constexpr int kBarDrain = 8 + 2 * kStages;
-  static constexpr int kNumBars = 9 + 2 * kStages;
+  static constexpr int kBarQFull = 2;                            // [kQStages]
+  static constexpr int kBarQEmpty = kBarQFull + kQStages;        // [kQStages]
+  static constexpr int kBarDOFull = kBarQEmpty + kQStages;       // [kDOStages]
+  static constexpr int kBarDOEmpty = kBarDOFull + kDOStages;     // [kDOStages]
+  static constexpr int kBarSFull = kBarDOEmpty + kDOStages;
+  static constexpr int kBarDPFull = kBarSFull + 1;
+  static constexpr int kBarPReady = kBarSFull + 2;
+  static constexpr int kBarDSReady = kBarSFull + 3;
+  static constexpr int kBarAccFull = kBarSFull + 4;
+  static constexpr int kBarAccFree = kBarSFull + 5;
+  static constexpr int kBarDrain = kBarSFull + 6;
+  static constexpr int kNumBars = kBarDrain + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;
-  static constexpr int kAlloc = kMisc + 16 + 1024;
+  static constexpr int kAlloc = kMisc + 16;
+  static_assert(kAlloc <= 232448, "shared memory over the 227 KB per-block limit");
 };
 
 template <int D>
@@ -179,19 +209,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tmL2, const __grid_constant__ CUtensorMap tmD,
                     const BwdArgs args) {
   using L = DkdvLayout<D>;
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw_addr = smem_u32(smem_raw);
-  const uint32_t base = (raw_addr + 1023u) & ~1023u;
-  uint8_t* smem = smem_raw + (base - raw_addr);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t base = smem_u32(smem_raw);
+  if (base & 1023u) {  // see DkdvLayout: the layout has no room to realign
+    if (threadIdx.x == 0) atomicOr(args.err, kErrSmemAlign);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   auto bar = [&](int i) -> uint32_t { return base + L::kBar + 8 * i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
-  auto wait = [&](uint32_t b, uint32_t parity) -> bool {
-    return mbar_wait(b, parity, abort_flag, args.err);
-  };
-  // the same for a whole converged warp: every lane gets the same answer
+  // a wait for a whole converged warp: every lane gets the same answer
   auto wait_warp = [&](uint32_t b, uint32_t parity) -> bool {
     return __all_sync(0xffffffffu, mbar_wait(b, parity, abort_flag, args.err));
   };
@@ -200,9 +230,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     mbar_init(bar(L::kBarKVFull), 1);
     mbar_init(bar(L::kBarKVEmpty), 1);
-    for (int s = 0; s < L::kStages; ++s) {
+    for (int s = 0; s < L::kQStages; ++s) {
       mbar_init(bar(L::kBarQFull + s), 1);
-      mbar_init(bar(L::kBarQEmpty + s), 1 + kEw / 32);  // MMA commit + element-wise warps
+      mbar_init(bar(L::kBarQEmpty + s), 1);
+    }
+    for (int s = 0; s < L::kDOStages; ++s) {
+      mbar_init(bar(L::kBarDOFull + s), 1);
+      mbar_init(bar(L::kBarDOEmpty + s), 1 + kEw / 32);  // MMA commit + element-wise warps
     }
     mbar_init(bar(L::kBarSFull), 1);
     mbar_init(bar(L::kBarDPFull), 1);
@@ -234,131 +268,150 @@ __global__ void __launch_bounds__(kThreads, 1)
       i0 = 0;
     }
   };
+  auto qslot = [&](int s) -> uint32_t { return base + L::kQ0 + s * L::kTileBytes; };
+  auto doslot = [&](int s) -> uint32_t { return base + L::kDO0 + s * L::kDOSlotBytes; };
 
   if (warp >= kWarpTMA) regs_dec<kRegsControl>();
   if (warp == kWarpTMA) {
     // the whole warp runs the loop; one elected lane issues each copy
-    {
-      int stage = 0, units = 0, kv_loads = 0;
-      uint32_t phase = 0;
-      int issued[L::kStages] = {};
-      uint32_t issued_phase[L::kStages] = {};
-      bool ok = true;
-      for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
+    int qs = 0, ds = 0, units = 0, kv_loads = 0;
+    uint32_t qph = 0, dph = 0;
+    int q_issued[L::kQStages] = {}, d_issued[L::kDOStages] = {};
+    uint32_t q_phase[L::kQStages] = {}, d_phase[L::kDOStages] = {};
+    bool ok = true;
+    for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
          w = snake_unit(++r), ++units) {
-        int bh, j, i0;
-        unit(w, bh, j, i0);
-        if (units > 0) ok = wait_warp(bar(L::kBarKVEmpty), (units - 1) & 1);
+      int bh, j, i0;
+      unit(w, bh, j, i0);
+      if (units > 0) ok = wait_warp(bar(L::kBarKVEmpty), (units - 1) & 1);
+      if (!ok) break;
+      mbar_arrive_expect_tx_elect(bar(L::kBarKVFull), 2 * L::kTileBytes);
+      for (int c = 0; c < D / 64; ++c) {
+        tma_load_3d_elect(base + L::kK + c * L::kBoxBytes, &tmK, bar(L::kBarKVFull), c * 64, j * kTile, bh);
+        tma_load_3d_elect(base + L::kV + c * L::kBoxBytes, &tmV, bar(L::kBarKVFull), c * 64, j * kTile, bh);
+      }
+      ++kv_loads;
+      for (int i = i0; ok && i < args.n_tiles; ++i) {
+        ok = wait_warp(bar(L::kBarQEmpty + qs), qph ^ 1);
         if (!ok) break;
-        mbar_arrive_expect_tx_elect(bar(L::kBarKVFull), 2 * L::kTileBytes);
-        for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d_elect(base + L::kK + c * L::kBoxBytes, &tmK, bar(L::kBarKVFull), c * 64, j * kTile, bh);
-          tma_load_3d_elect(base + L::kV + c * L::kBoxBytes, &tmV, bar(L::kBarKVFull), c * 64, j * kTile, bh);
-        }
-        ++kv_loads;
-        for (int i = i0; ok && i < args.n_tiles; ++i) {
-          ok = wait_warp(bar(L::kBarQEmpty + stage), phase ^ 1);
-          if (!ok) break;
-          const uint32_t fb = bar(L::kBarQFull + stage);
-          const uint32_t sb = base + L::kStage0 + stage * L::kStageBytes;
-          mbar_arrive_expect_tx_elect(fb, 2 * L::kTileBytes + 1024);
-          for (int c = 0; c < D / 64; ++c) {
-            tma_load_3d_elect(sb + L::kStageQ + c * L::kBoxBytes, &tmQ, fb, c * 64, i * kTile, bh);
-            tma_load_3d_elect(sb + L::kStageDO + c * L::kBoxBytes, &tmdO, fb, c * 64, i * kTile, bh);
-          }
-          tma_load_3d_elect(sb + L::kStageL, &tmL2, fb, i * kTile, bh, 0);
-          tma_load_3d_elect(sb + L::kStageD, &tmD, fb, i * kTile, bh, 0);
-          issued[stage] = 1;
-          issued_phase[stage] = phase;
-          if (++stage == L::kStages) stage = 0, phase ^= 1;
-        }
+        mbar_arrive_expect_tx_elect(bar(L::kBarQFull + qs), L::kTileBytes);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d_elect(qslot(qs) + c * L::kBoxBytes, &tmQ, bar(L::kBarQFull + qs), c * 64,
+                            i * kTile, bh);
+        q_issued[qs] = 1;
+        q_phase[qs] = qph;
+        if (++qs == L::kQStages) qs = 0, qph ^= 1;
+        ok = wait_warp(bar(L::kBarDOEmpty + ds), dph ^ 1);
+        if (!ok) break;
+        const uint32_t fb = bar(L::kBarDOFull + ds);
+        mbar_arrive_expect_tx_elect(fb, L::kTileBytes + 1024);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d_elect(doslot(ds) + c * L::kBoxBytes, &tmdO, fb, c * 64, i * kTile, bh);
+        tma_load_3d_elect(doslot(ds) + L::kSlotL, &tmL2, fb, i * kTile, bh, 0);
+        tma_load_3d_elect(doslot(ds) + L::kSlotD, &tmD, fb, i * kTile, bh, 0);
+        d_issued[ds] = 1;
+        d_phase[ds] = dph;
+        if (++ds == L::kDOStages) ds = 0, dph ^= 1;
       }
-      if (!ok) {
-        // let the loads already issued land before the CTA exits
-        for (int s = 0; s < L::kStages; ++s)
-          if (issued[s]) mbar_wait_drain(bar(L::kBarQFull + s), issued_phase[s], args.err);
-        if (kv_loads > 0) mbar_wait_drain(bar(L::kBarKVFull), (kv_loads - 1) & 1, args.err);
-      }
+    }
+    if (!ok) {
+      // let the loads already issued land before the CTA exits
+      for (int s = 0; s < L::kQStages; ++s)
+        if (q_issued[s]) mbar_wait_drain(bar(L::kBarQFull + s), q_phase[s], args.err);
+      for (int s = 0; s < L::kDOStages; ++s)
+        if (d_issued[s]) mbar_wait_drain(bar(L::kBarDOFull + s), d_phase[s], args.err);
+      if (kv_loads > 0) mbar_wait_drain(bar(L::kBarKVFull), (kv_loads - 1) & 1, args.err);
     }
   } else if (warp == kWarpMMA) {
     // the whole warp runs the loop so descriptors stay warp-uniform; one elected lane
     // issues each tcgen05 instruction
-    {
-      constexpr uint32_t idSS = idesc_bf16_f32(kTile, false);
-      constexpr uint32_t idTS = idesc_bf16_f32(D, true);
-      const uint64_t dK0 = desc_kmajor(base + L::kK);
-      const uint64_t dV0 = desc_kmajor(base + L::kV);
-      int stage = 0, units = 0, p_cnt = 0, ds_cnt = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      auto stage_base = [&](int s) { return base + L::kStage0 + s * L::kStageBytes; };
-      // S^T = K Q^T or dP^T = V dO^T: both operands K-major, K extent = D.  The K-step
-      // loops are fully unrolled so that the single issuing thread keeps up with the
-      // tensor pipe (64 cycles per 128 x 128 x 16 MMA).
-      auto issue_ss = [&](uint32_t dtm, uint64_t da, uint32_t b_saddr, uint32_t done_bar) {
-        const uint64_t db = desc_kmajor(b_saddr);
+    constexpr uint32_t idSS = idesc_bf16_f32(kTile, false);
+    constexpr uint32_t idTS = idesc_bf16_f32(D, true);
+    const uint64_t dK0 = desc_kmajor(base + L::kK);
+    const uint64_t dV0 = desc_kmajor(base + L::kV);
+    int qc = 0, dc = 0, units = 0, p_cnt = 0, ds_cnt = 0;
+    uint32_t qcph = 0, dcph = 0;
+    bool ok = true;
+    // S^T = K Q^T or dP^T = V dO^T: both operands K-major, K extent = D.  The K-step
+    // loops are fully unrolled so that the single issuing thread keeps up with the
+    // tensor pipe (64 cycles per 128 x 128 x 16 MMA).
+    auto issue_ss = [&](uint32_t dtm, uint64_t da, uint32_t b_saddr, uint32_t done_bar) {
+      const uint64_t db = desc_kmajor(b_saddr);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = ((kk / 4) * L::kBoxBytes + (kk % 4) * 32) >> 4;
-          mma_ss_elect(dtm, da + off, db + off, idSS, kk > 0 ? 1u : 0u);
-        }
-        mma_commit_elect(done_bar);
-      };
-      // acc += A(TMEM, 128 x 128 bf16) * B(smem tile, 128 rows x D, MN-major)
-      auto issue_ts = [&](uint32_t acc, uint32_t a_tmem, uint32_t b_saddr, bool accumulate) {
-        const uint64_t db = desc_mnmajor(b_saddr, L::kBoxBytes);
-#pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ts_elect(acc, split_operand_col(a_tmem, kk), db + static_cast<uint64_t>((kk * 2048) >> 4),
-                 idTS, (accumulate || kk > 0) ? 1u : 0u);
-      };
-      for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
-         w = snake_unit(++r), ++units) {
-        int bh, j, i0;
-        unit(w, bh, j, i0);
-        const int m = args.n_tiles - i0;
-        ok = wait_warp(bar(L::kBarKVFull), units & 1);
-        if (ok) ok = wait_warp(bar(L::kBarQFull + stage), phase);
-        if (!ok) break;
-        tc_fence_after();
-        int cur = stage;
-        if (++stage == L::kStages) stage = 0, phase ^= 1;
-        issue_ss(tS, dK0, stage_base(cur) + L::kStageQ, bar(L::kBarSFull));
-        issue_ss(tdP, dV0, stage_base(cur) + L::kStageDO, bar(L::kBarDPFull));
-        for (int t = 0; t < m; ++t) {
-          ok = wait_warp(bar(L::kBarPReady), p_cnt & 1);
-          if (ok && t == 0 && units > 0) ok = wait_warp(bar(L::kBarAccFree), (units - 1) & 1);
-          if (!ok) break;
-          ++p_cnt;
-          tc_fence_after();
-          issue_ts(tdV, tS, stage_base(cur) + L::kStageDO, t > 0);  // dV += P^T dO
-          int nxt = -1;
-          if (t + 1 < m) {
-            ok = wait_warp(bar(L::kBarQFull + stage), phase);
-            if (!ok) break;
-            nxt = stage;
-            if (++stage == L::kStages) stage = 0, phase ^= 1;
-            tc_fence_after();
-            issue_ss(tS, dK0, stage_base(nxt) + L::kStageQ, bar(L::kBarSFull));
-          }
-          ok = wait_warp(bar(L::kBarDSReady), ds_cnt & 1);
-          if (!ok) break;
-          ++ds_cnt;
-          tc_fence_after();
-          issue_ts(tdK, tdP, stage_base(cur) + L::kStageQ, t > 0);  // dK += dS^T Q
-          mma_commit_elect(bar(L::kBarQEmpty + cur));
-          if (nxt >= 0) {
-            issue_ss(tdP, dV0, stage_base(nxt) + L::kStageDO, bar(L::kBarDPFull));
-            cur = nxt;
-          }
-        }
-        if (!ok) break;
-        mma_commit_elect(bar(L::kBarKVEmpty));
-        mma_commit_elect(bar(L::kBarAccFull));
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = ((kk / 4) * L::kBoxBytes + (kk % 4) * 32) >> 4;
+        mma_ss_elect(dtm, da + off, db + off, idSS, kk > 0 ? 1u : 0u);
       }
-      mma_commit_elect(bar(L::kBarDrain));
-      mbar_wait_drain(bar(L::kBarDrain), 0, args.err);
+      mma_commit_elect(done_bar);
+    };
+    // acc += A(TMEM, 128 x 128 bf16) * B(smem tile, 128 rows x D, MN-major)
+    auto issue_ts = [&](uint32_t acc, uint32_t a_tmem, uint32_t b_saddr, bool accumulate) {
+      const uint64_t db = desc_mnmajor(b_saddr, L::kBoxBytes);
+#pragma unroll
+      for (int kk = 0; kk < kTile / 16; ++kk)
+        mma_ts_elect(acc, split_operand_col(a_tmem, kk), db + static_cast<uint64_t>((kk * 2048) >> 4),
+                     idTS, (accumulate || kk > 0) ? 1u : 0u);
+    };
+    // S^T(next query tile) from the next Q slot
+    auto next_s = [&](int& slot) -> bool {
+      if (!wait_warp(bar(L::kBarQFull + qc), qcph)) return false;
+      slot = qc;
+      if (++qc == L::kQStages) qc = 0, qcph ^= 1;
+      tc_fence_after();
+      issue_ss(tS, dK0, qslot(slot), bar(L::kBarSFull));
+      return true;
+    };
+    // dP^T(next query tile) from the next dO slot
+    auto next_dp = [&](int& slot) -> bool {
+      if (!wait_warp(bar(L::kBarDOFull + dc), dcph)) return false;
+      slot = dc;
+      if (++dc == L::kDOStages) dc = 0, dcph ^= 1;
+      tc_fence_after();
+      issue_ss(tdP, dV0, doslot(slot), bar(L::kBarDPFull));
+      return true;
+    };
+    for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
+         w = snake_unit(++r), ++units) {
+      int bh, j, i0;
+      unit(w, bh, j, i0);
+      const int m = args.n_tiles - i0;
+      ok = wait_warp(bar(L::kBarKVFull), units & 1);
+      int curq = 0, curd = 0;
+      if (ok) ok = next_s(curq);
+      if (ok) ok = next_dp(curd);
+      if (!ok) break;
+      for (int t = 0; t < m; ++t) {
+        ok = wait_warp(bar(L::kBarPReady), p_cnt & 1);
+        if (ok && t == 0 && units > 0) ok = wait_warp(bar(L::kBarAccFree), (units - 1) & 1);
+        if (!ok) break;
+        ++p_cnt;
+        tc_fence_after();
+        issue_ts(tdV, tS, doslot(curd), t > 0);  // dV += P^T dO
+        mma_commit_elect(bar(L::kBarDOEmpty + curd));
+        int nq = -1, nd = -1;
+        if (t + 1 < m) {
+          ok = next_s(nq);
+          if (!ok) break;
+        }
+        ok = wait_warp(bar(L::kBarDSReady), ds_cnt & 1);
+        if (!ok) break;
+        ++ds_cnt;
+        tc_fence_after();
+        issue_ts(tdK, tdP, qslot(curq), t > 0);  // dK += dS^T Q
+        mma_commit_elect(bar(L::kBarQEmpty + curq));
+        if (t + 1 < m) {
+          ok = next_dp(nd);
+          if (!ok) break;
+          curq = nq;
+          curd = nd;
+        }
+      }
+      if (!ok) break;
+      mma_commit_elect(bar(L::kBarKVEmpty));
+      mma_commit_elect(bar(L::kBarAccFull));
     }
+    mma_commit_elect(bar(L::kBarDrain));
+    mbar_wait_drain(bar(L::kBarDrain), 0, args.err);
   } else if (warp < kWarpTMA) {
     regs_inc<kRegsEw>();
     const int g = warp / 4;            // column group
@@ -373,10 +426,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       int bh, j, i0;
       unit(w, bh, j, i0);
       for (int i = i0; i < args.n_tiles; ++i) {
-        const uint8_t* sb = smem + L::kStage0 + stage * L::kStageBytes;
-        const float* sL = reinterpret_cast<const float*>(sb + L::kStageL) + col0;
-        const float* sD = reinterpret_cast<const float*>(sb + L::kStageD) + col0;
-        ok = wait_warp(bar(L::kBarQFull + stage), phase);
+        // this tile's L2 and D rows sit in its dO slot
+        const uint8_t* sb = smem + L::kDO0 + stage * L::kDOSlotBytes;
+        const float* sL = reinterpret_cast<const float*>(sb + L::kSlotL) + col0;
+        const float* sD = reinterpret_cast<const float*>(sb + L::kSlotD) + col0;
+        ok = wait_warp(bar(L::kBarDOFull + stage), phase);
         if (ok) ok = wait_warp(bar(L::kBarSFull), s_cnt & 1);
         if (!ok) break;
         ++s_cnt;
@@ -391,7 +445,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool diag = args.causal && i == j;
 #pragma unroll
           for (int c = 0; c < kCols; ++c) {
-            float e = ex2_approx(fmaf(__uint_as_float(r[c]), args.scale_log2, -sL[c]));
+            const float x = fmaf(__uint_as_float(r[c]), args.scale_log2, -sL[c]);
+            float e = (kPolyEvery > 0 && c % kPolyStride == kPolyStride - 1) ? exp2_poly(x)
+                                                                            : ex2_approx(x);
             if (diag && col0 + c < row) e = 0.f;  // query i*128+col0+c before key j*128+row
             p[c] = e;
           }
@@ -426,8 +482,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_wait_st();
         warp_arrive(bar(L::kBarDSReady));
-        if (lane == 0) mbar_arrive(bar(L::kBarQEmpty + stage));  // done with its L2, D rows
-        if (++stage == L::kStages) stage = 0, phase ^= 1;
+        if (lane == 0) mbar_arrive(bar(L::kBarDOEmpty + stage));  // done with its L2, D rows
+        if (++stage == L::kDOStages) stage = 0, phase ^= 1;
       }
       if (!ok) break;
       // epilogue: dV and scale * dK for this key row; group g writes columns of its half
@@ -487,7 +543,9 @@ struct DqLayout {
   static constexpr int kBarAccFull = kBarSFull + 4;
   static constexpr int kBarAccFree = kBarSFull + 5;
   static constexpr int kBarDrain = kBarSFull + 6;
-  static constexpr int kNumBars = kBarDrain + 1;
+  static constexpr int kBarDPFree = kBarSFull + 7;   // element-wise warps have read dP
+  static constexpr int kBarDQDone = kBarSFull + 8;   // the dQ product has read dS
+  static constexpr int kNumBars = kBarDQDone + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kAlloc = kMisc + 16 + 1024;
   static_assert(kAlloc <= 232448, "shared memory over the 227 KB per-block limit");
@@ -535,6 +593,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(L::kBarAccFull), 1);
     mbar_init(bar(L::kBarAccFree), kEw / 32);
     mbar_init(bar(L::kBarDrain), 1);
+    mbar_init(bar(L::kBarDPFree), kEw / 32);
+    mbar_init(bar(L::kBarDQDone), 1);
     fence_mbar_init();
   }
   if (warp == kWarpMMA) {
@@ -545,7 +605,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tdQ = tmem, tS = tmem + 128, tdP = tmem + 256;
+  // dS has a region of its own (rather than overwriting dP), so the next tile's S and
+  // dP products can start as soon as the element-wise warps have read this tile's.
+  const uint32_t tdQ = tmem, tS = tmem + 128, tdP = tmem + 256, tdS = tmem + 384;
 
   auto unit = [&](int w, int& bh, int& i, int& m) {
     if (args.causal) {
@@ -642,6 +704,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (++vc == L::kVStages) vc = 0, vcph ^= 1;
         return true;
       };
+      int dpfree_cnt = 0;
       for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
          w = snake_unit(++r), ++units) {
         int bh, i, m;
@@ -658,6 +721,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < m; ++t) {
           int nxt = -1;
           if (t + 1 < m) {
+            // S(t+1) once the element-wise warps hold S(t) in registers
             ok = wait_warp(bar(L::kBarKFull + kc), kcph);
             if (ok) ok = wait_warp(bar(L::kBarSFree), sfree_cnt & 1);
             if (!ok) break;
@@ -666,6 +730,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (++kc == L::kKStages) kc = 0, kcph ^= 1;
             tc_fence_after();
             issue_ss(tS, dQd, kslot(nxt), bar(L::kBarSFull));
+            // dP(t+1) once they hold dP(t)
+            ok = wait_warp(bar(L::kBarDPFree), dpfree_cnt & 1);
+            if (!ok) break;
+            ++dpfree_cnt;
+            tc_fence_after();
+            ok = issue_dp();
+            if (!ok) break;
           }
           ok = wait_warp(bar(L::kBarDSReady), ds_cnt & 1);
           if (ok && t == 0 && units > 0) ok = wait_warp(bar(L::kBarAccFree), (units - 1) & 1);
@@ -676,20 +747,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t db = desc_mnmajor(kslot(cur), L::kBoxBytes);
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
-            mma_ts_elect(tdQ, split_operand_col(tdP, kk), db + static_cast<uint64_t>((kk * 2048) >> 4),
+            mma_ts_elect(tdQ, split_operand_col(tdS, kk), db + static_cast<uint64_t>((kk * 2048) >> 4),
                          idTS, (t > 0 || kk > 0) ? 1u : 0u);
           mma_commit_elect(bar(L::kBarKEmpty + cur));
-          if (nxt >= 0) {
-            ok = issue_dp();
-            if (!ok) break;
-            cur = nxt;
-          }
+          mma_commit_elect(bar(L::kBarDQDone));
+          if (nxt >= 0) cur = nxt;
         }
         if (!ok) break;
-        // the last unit's S tile was read by the element-wise warps: consume that signal
+        // the unit's last S and dP tiles were read by the element-wise warps: consume
+        // those signals before the next unit overwrites the regions
         ok = wait_warp(bar(L::kBarSFree), sfree_cnt & 1);
+        if (ok) ok = wait_warp(bar(L::kBarDPFree), dpfree_cnt & 1);
         if (!ok) break;
         ++sfree_cnt;
+        ++dpfree_cnt;
         mma_commit_elect(bar(L::kBarQEmpty));
         mma_commit_elect(bar(L::kBarAccFull));
       }
@@ -702,7 +773,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int col0 = g * kCols;        // first tile column (key) of this group
     const int row = (warp % 4) * 32 + lane;  // query row within the tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp % 4) * 32) << 16;
-    int units = 0, s_cnt = 0, dp_cnt = 0;
+    int units = 0, s_cnt = 0, dp_cnt = 0, dq_cnt = 0;
     bool ok = true;
     for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
          w = snake_unit(++r), ++units) {
@@ -730,7 +801,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int lim = args.causal ? min(args.N, q_row + 1) : args.N;
 #pragma unroll
           for (int c = 0; c < kCols; ++c) {
-            float e = ex2_approx(fmaf(__uint_as_float(r[c]), args.scale_log2, -l2));
+            const float x = fmaf(__uint_as_float(r[c]), args.scale_log2, -l2);
+            float e = (kPolyEvery > 0 && c % kPolyStride == kPolyStride - 1) ? exp2_poly(x)
+                                                                            : ex2_approx(x);
             if (need_mask && kv0 + c >= lim) e = 0.f;
             p[c] = e;
           }
@@ -739,20 +812,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         ++dp_cnt;
         tc_fence_after();
+        uint32_t dpv[kCols];
 #pragma unroll
-        for (int c = 0; c < kCols / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tdP + lane_off + col0 + c * 32, r);
-          tmem_wait_ld();
-          uint32_t pk[16];
+        for (int c = 0; c < kCols / 32; ++c) tmem_ld32(tdP + lane_off + col0 + c * 32, &dpv[c * 32]);
+        tmem_wait_ld();
+        warp_arrive(bar(L::kBarDPFree));  // dP(t+1) may now be written over it
+        uint32_t pk[kCols / 2];
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const int c0 = c * 32 + 2 * k;
-            pk[k] = pack_bf16x2(p[c0] * (__uint_as_float(r[2 * k]) - drow),
-                                p[c0 + 1] * (__uint_as_float(r[2 * k + 1]) - drow));
-          }
-          tmem_st16(tdP + lane_off + col0 + c * 16, pk);
+        for (int k = 0; k < kCols / 2; ++k)
+          pk[k] = pack_bf16x2(p[2 * k] * (__uint_as_float(dpv[2 * k]) - drow),
+                              p[2 * k + 1] * (__uint_as_float(dpv[2 * k + 1]) - drow));
+        // the previous tile's dQ product must have read the dS region before it is reused
+        if (dq_cnt > 0) {
+          ok = wait_warp(bar(L::kBarDQDone), (dq_cnt - 1) & 1);
+          if (!ok) break;
         }
+        ++dq_cnt;
+        tc_fence_after();
+        tmem_st32(tdS + lane_off + col0, pk);  // this group's 32-column piece of dS
         tmem_wait_st();
         warp_arrive(bar(L::kBarDSReady));
       }
@@ -807,9 +884,11 @@ cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUten
   a.L2pad = L2pad;
 
   const long long rows = static_cast<long long>(p.BH) * a.Npad;
+  const long long rows_per_block = static_cast<long long>(kPrepThreads / (D / 8)) * kPrepRowsPerThread;
   cudaError_t e = trace_mark(p, 0, stream);
   if (e != cudaSuccess) return e;
-  bwd_prep_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
+  bwd_prep_kernel<D><<<static_cast<unsigned>((rows + rows_per_block - 1) / rows_per_block),
+                       kPrepThreads, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO), LSE, Dpad,
       L2pad, p.BH, p.N, a.Npad);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;

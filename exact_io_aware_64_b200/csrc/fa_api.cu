@@ -329,6 +329,10 @@ fa_status fa_check_device_error(cudaStream_t stream) {
     const unsigned int zero = 0;
     e = cudaMemcpy(dev.err, &zero, sizeof(zero), cudaMemcpyHostToDevice);
     if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+    if (word & 2u)
+      return fail(FA_ERR_CUDA,
+                  "a kernel found its dynamic shared memory misaligned and did no work "
+                  "(error word 0x%x)", word);
     return fail(FA_ERR_TIMEOUT, "a kernel pipeline wait timed out (error word 0x%x)", word);
   }
   return FA_OK;

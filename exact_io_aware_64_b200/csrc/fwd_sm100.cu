@@ -56,6 +56,11 @@ static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kThreads * kRegsLau
 constexpr int kWarpTMA = 8;
 constexpr int kWarpMMA = 9;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Every kPolyEvery-th pair of exponentials (unmasked tiles only) may be computed on the
+// FMA pipe with exp2_poly instead of MUFU.  Measured on B200 at 1-in-4 and 1-in-8 it did
+// not speed the forward up (the softmax here is not limited by MUFU alone), so 0: off.
+constexpr int kPolyEvery = 0;
+constexpr int kPolyStride = kPolyEvery > 0 ? kPolyEvery : 1;
 constexpr uint32_t kTmemCols = 512;
 
 template <int D>
@@ -403,13 +408,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float mref = (m == -INFINITY) ? 0.f : m;
         uint32_t pk[kBN / 2];
         float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (need_mask) {
+          // masked tiles: every exponential on MUFU, so masked entries are exactly 0
 #pragma unroll
-        for (int c = 0; c < kBN / 2; ++c) {
-          const float p0 = ex2_approx(fmaf(s[2 * c], args.scale_log2, -mref));
-          const float p1 = ex2_approx(fmaf(s[2 * c + 1], args.scale_log2, -mref));
-          ls[(2 * c) % 8] += p0;
-          ls[(2 * c + 1) % 8] += p1;
-          pk[c] = pack_bf16x2(p0, p1);
+          for (int c = 0; c < kBN / 2; ++c) {
+            const float p0 = ex2_approx(fmaf(s[2 * c], args.scale_log2, -mref));
+            const float p1 = ex2_approx(fmaf(s[2 * c + 1], args.scale_log2, -mref));
+            ls[(2 * c) % 8] += p0;
+            ls[(2 * c + 1) % 8] += p1;
+            pk[c] = pack_bf16x2(p0, p1);
+          }
+        } else {
+          // the MUFU unit (16 exp2 per clock per SM) costs as much per score tile as
+          // the two MMAs; every kPolyEvery-th pair goes to the FMA pipe instead
+#pragma unroll
+          for (int c = 0; c < kBN / 2; ++c) {
+            const float x0 = fmaf(s[2 * c], args.scale_log2, -mref);
+            const float x1 = fmaf(s[2 * c + 1], args.scale_log2, -mref);
+            const bool poly = kPolyEvery > 0 && c % kPolyStride == kPolyStride - 1;
+            const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
+            const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);
+            ls[(2 * c) % 8] += p0;
+            ls[(2 * c + 1) % 8] += p1;
+            pk[c] = pack_bf16x2(p0, p1);
+          }
         }
         l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
         tmem_st32(tSrow, &pk[0]);

@@ -68,8 +68,10 @@ constexpr long long kWaitLimitCycles = 8000000000ll;
 // that a completed phase is noticed one try_wait after it completes.
 constexpr uint32_t kSpinCheck = 256;
 
-// Bit set in the library's device error word when a wait runs out of time.
+// Bits of the library's device error word: a wait ran out of time; a kernel found its
+// dynamic shared memory not aligned as its layout requires (it then does no work).
 constexpr unsigned int kErrWaitTimeout = 1u;
+constexpr unsigned int kErrSmemAlign = 2u;
 
 // Wait until the phase with the given parity has completed.  Returns false if the time
 // limit runs out (then it also sets kErrWaitTimeout in *err and raises *abort so the
@@ -367,6 +369,22 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA and integer pipes instead of the MUFU unit, for x >= -126 (smaller x
+// is clamped; the result is then below 2^-126).  Cody-Waite style range reduction
+// x = n + f with n = round(x) taken by adding 1.5 * 2^23 (its low mantissa bits then hold
+// n), f in [-1/2, 1/2]; 2^f by a cubic fitted with the Remez exchange algorithm on the
+// relative error (gen_exp2_poly.py: max relative error 7.5e-5, well below bf16
+// rounding); 2^n applied by adding n to the exponent field.
+__device__ __forceinline__ float exp2_poly(float x) {
+  constexpr float kC0 = 0.99992806f, kC1 = 0.69326097f, kC2 = 0.24261113f, kC3 = 0.05517167f;
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  x = fmaxf(x, -126.0f);
+  const float t = x + kRound;
+  const float f = x - (t - kRound);
+  const float p = fmaf(fmaf(fmaf(kC3, f, kC2), f, kC1), f, kC0);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -162,7 +162,8 @@ FA_API const char* fa_last_error_message(void);
 
 /*
  * Synchronises `stream`, then reports and clears the device-side error word that the
- * kernels set when a pipeline wait exceeds its time limit (FA_ERR_TIMEOUT), or
+ * kernels set when a pipeline wait exceeds its time limit (FA_ERR_TIMEOUT) or when a
+ * kernel finds its shared memory misaligned and skips its work (FA_ERR_CUDA), or
  * FA_ERR_CUDA if the stream itself reports an error.
  */
 FA_API fa_status fa_check_device_error(cudaStream_t stream);
