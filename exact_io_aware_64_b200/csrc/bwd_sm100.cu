@@ -8,9 +8,10 @@
 //     dQ = scale dS K,  dK = scale dS^T Q.
 //
 // Three kernels, no atomics (bitwise reproducible):
-//   1. bwd_prep: D = rowsum(dO * O) and L2 = L * log2(e), both stored padded to whole
-//      128-row tiles in the caller's workspace (rows past N: D = 0, L2 = +inf, so their
-//      probabilities are exactly 0) so that TMA can stream them.
+//   1. bwd_prep: -D = -rowsum(dO * O) and -L2 = -L * log2(e), both stored padded to
+//      whole 128-row tiles in the caller's workspace (rows past N: 0 and -inf, so their
+//      probabilities are exactly 0) so that TMA can stream them.  They are stored
+//      negated because the element-wise steps add them (packed fused multiply-adds).
 //   2. bwd_dkdv: one work unit per (batch*head, 128-row key tile j).  K_j and V_j stay in
 //      shared memory while the query tiles i stream past; the tile products are taken
 //      transposed so that the key row is the TMEM lane:
@@ -69,17 +70,20 @@ __device__ __forceinline__ uint32_t split_operand_col(uint32_t base, int kk) {
 }
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
-// Every kPolyEvery-th exponential of a row may be computed on the FMA pipe (exp2_poly)
-// instead of the MUFU unit; masked entries are zeroed after the exponential either way.
-// Measured on B200 at 1-in-2 and 1-in-4 it made the backward slower, so 0: off.
-constexpr int kPolyEvery = 0;
-constexpr int kPolyStride = kPolyEvery > 0 ? kPolyEvery : 1;
+// Every PolyEvery<D>-th exponential of a row may be computed on the FMA pipe
+// (exp2_poly) instead of the MUFU unit; masked entries are zeroed after the exponential
+// either way; 0 keeps all of them on MUFU.
+template <int D>
+struct PolyEvery {
+  static constexpr int value = 0;
+};
 
 __host__ __device__ constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
 // ------------------------------------------------------------------ 1. preparation
-// D[bh][r] = sum_k dO[bh][r][k] * O[bh][r][k];  L2[bh][r] = LSE[bh][r] * log2(e).
-// Padded rows r in [N, Npad): D = 0, L2 = +inf.  Bandwidth bound: each thread reads 16
+// Stores the negated row statistics the element-wise steps add:
+//   ND[bh][r] = -sum_k dO[bh][r][k] * O[bh][r][k],   NL2[bh][r] = -LSE[bh][r] * log2(e).
+// Padded rows r in [N, Npad): ND = 0, NL2 = -inf (their probabilities are exactly 0).  Bandwidth bound: each thread reads 16
 // bytes of O and of dO for kRowsPerThread rows (independent loads in flight), the
 // D / 8 threads of a row combine their partial sums with shuffles.
 constexpr int kPrepThreads = 256;
@@ -127,8 +131,8 @@ __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(
     if (part == 0 && row < total) {
       const int bh = static_cast<int>(row / Npad);
       const int r = static_cast<int>(row % Npad);
-      Dout[row] = acc[k];
-      L2out[row] = r < N ? LSE[static_cast<size_t>(bh) * N + r] * kLog2e : INFINITY;
+      Dout[row] = -acc[k];
+      L2out[row] = r < N ? -LSE[static_cast<size_t>(bh) * N + r] * kLog2e : -INFINITY;
     }
   }
 }
@@ -138,8 +142,8 @@ struct BwdArgs {
   __nv_bfloat16* dQ;
   __nv_bfloat16* dK;
   __nv_bfloat16* dV;
-  const float* Dpad;   // [BH][Npad]
-  const float* L2pad;  // [BH][Npad]
+  const float* Dpad;   // [BH][Npad]: -D
+  const float* L2pad;  // [BH][Npad]: -LSE * log2(e)
   int BH;
   int N;
   int Npad;
@@ -435,6 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         ++s_cnt;
         tc_fence_after();
+        constexpr int kStride = PolyEvery<D>::value > 0 ? PolyEvery<D>::value : 1;
         float p[kCols];
         {
           uint32_t r[kCols];
@@ -443,13 +448,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld32(tS + lane_off + col0 + c * 32, &r[c * 32]);
           tmem_wait_ld();
           const bool diag = args.causal && i == j;
+          const uint64_t scale2 = f32x2(args.scale_log2, args.scale_log2);
 #pragma unroll
-          for (int c = 0; c < kCols; ++c) {
-            const float x = fmaf(__uint_as_float(r[c]), args.scale_log2, -sL[c]);
-            float e = (kPolyEvery > 0 && c % kPolyStride == kPolyStride - 1) ? exp2_poly(x)
-                                                                            : ex2_approx(x);
-            if (diag && col0 + c < row) e = 0.f;  // query i*128+col0+c before key j*128+row
-            p[c] = e;
+          for (int c = 0; c < kCols; c += 2) {
+            // x = S^T * scale * log2e - L2 for two query columns in one packed FMA
+            const uint64_t nl = *reinterpret_cast<const uint64_t*>(sL + c);
+            float x0, x1;
+            f32x2_split(fma_x2(f32x2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), scale2, nl),
+                        x0, x1);
+            const bool poly = PolyEvery<D>::value > 0 && c % kStride == kStride - 1;
+            float e0 = poly ? exp2_poly(x0) : ex2_approx(x0);
+            float e1 = poly ? exp2_poly(x1) : ex2_approx(x1);
+            if (diag && col0 + c < row) e0 = 0.f;  // query i*128+col0+c before key j*128+row
+            if (diag && col0 + c + 1 < row) e1 = 0.f;
+            p[c] = e0;
+            p[c + 1] = e1;
           }
         }
         {
@@ -472,9 +485,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
+            // dS = P (dP - D) for two query columns: one packed add, one packed multiply
             const int c0 = c * 32 + 2 * k;
-            const float ds0 = p[c0] * (__uint_as_float(r[2 * k]) - sD[c0]);
-            const float ds1 = p[c0 + 1] * (__uint_as_float(r[2 * k + 1]) - sD[c0 + 1]);
+            const uint64_t nd = *reinterpret_cast<const uint64_t*>(sD + c0);
+            float ds0, ds1;
+            f32x2_split(mul_x2(f32x2(p[c0], p[c0 + 1]),
+                               add_x2(f32x2(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1])), nd)),
+                        ds0, ds1);
             pk[k] = pack_bf16x2(ds0, ds1);
           }
           // dS for columns c*32.. lands on columns this group has already read
@@ -781,13 +798,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       unit(w, bh, i, m);
       const int q_row = i * kTile + row;
       const size_t prow = static_cast<size_t>(bh) * args.Npad + q_row;  // q_row < Npad
-      const float l2 = args.L2pad[prow];
-      const float drow = args.Dpad[prow];
+      const float nl2row = args.L2pad[prow];   // -LSE * log2(e) of this query row
+      const float ndrow = args.Dpad[prow];     // -D of this query row
       for (int j = 0; j < m; ++j) {
         ok = wait_warp(bar(L::kBarSFull), s_cnt & 1);
         if (!ok) break;
         ++s_cnt;
         tc_fence_after();
+        constexpr int kStride = PolyEvery<D>::value > 0 ? PolyEvery<D>::value : 1;
         float p[kCols];
         {
           uint32_t r[kCols];
@@ -799,13 +817,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int kv0 = j * kTile + col0;
           const bool need_mask = (kv0 + kCols > args.N) || (args.causal && j == i);
           const int lim = args.causal ? min(args.N, q_row + 1) : args.N;
+          const uint64_t scale2 = f32x2(args.scale_log2, args.scale_log2);
+          const uint64_t nl2 = f32x2(nl2row, nl2row);
 #pragma unroll
-          for (int c = 0; c < kCols; ++c) {
-            const float x = fmaf(__uint_as_float(r[c]), args.scale_log2, -l2);
-            float e = (kPolyEvery > 0 && c % kPolyStride == kPolyStride - 1) ? exp2_poly(x)
-                                                                            : ex2_approx(x);
-            if (need_mask && kv0 + c >= lim) e = 0.f;
-            p[c] = e;
+          for (int c = 0; c < kCols; c += 2) {
+            float x0, x1;
+            f32x2_split(fma_x2(f32x2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), scale2, nl2),
+                        x0, x1);
+            const bool poly = PolyEvery<D>::value > 0 && c % kStride == kStride - 1;
+            float e0 = poly ? exp2_poly(x0) : ex2_approx(x0);
+            float e1 = poly ? exp2_poly(x1) : ex2_approx(x1);
+            if (need_mask && kv0 + c >= lim) e0 = 0.f;
+            if (need_mask && kv0 + c + 1 >= lim) e1 = 0.f;
+            p[c] = e0;
+            p[c + 1] = e1;
           }
         }
         ok = wait_warp(bar(L::kBarDPFull), dp_cnt & 1);
@@ -818,10 +843,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         warp_arrive(bar(L::kBarDPFree));  // dP(t+1) may now be written over it
         uint32_t pk[kCols / 2];
+        const uint64_t nd2 = f32x2(ndrow, ndrow);
 #pragma unroll
-        for (int k = 0; k < kCols / 2; ++k)
-          pk[k] = pack_bf16x2(p[2 * k] * (__uint_as_float(dpv[2 * k]) - drow),
-                              p[2 * k + 1] * (__uint_as_float(dpv[2 * k + 1]) - drow));
+        for (int k = 0; k < kCols / 2; ++k) {
+          // dS = P (dP - D), two key columns per packed add and multiply
+          float ds0, ds1;
+          f32x2_split(mul_x2(f32x2(p[2 * k], p[2 * k + 1]),
+                             add_x2(f32x2(__uint_as_float(dpv[2 * k]), __uint_as_float(dpv[2 * k + 1])), nd2)),
+                      ds0, ds1);
+          pk[k] = pack_bf16x2(ds0, ds1);
+        }
         // the previous tile's dQ product must have read the dS region before it is reused
         if (dq_cnt > 0) {
           ok = wait_warp(bar(L::kBarDQDone), (dq_cnt - 1) & 1);

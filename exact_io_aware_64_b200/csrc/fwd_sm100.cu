@@ -56,11 +56,12 @@ static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kThreads * kRegsLau
 constexpr int kWarpTMA = 8;
 constexpr int kWarpMMA = 9;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-// Every kPolyEvery-th pair of exponentials (unmasked tiles only) may be computed on the
-// FMA pipe with exp2_poly instead of MUFU.  Measured on B200 at 1-in-4 and 1-in-8 it did
-// not speed the forward up (the softmax here is not limited by MUFU alone), so 0: off.
-constexpr int kPolyEvery = 0;
-constexpr int kPolyStride = kPolyEvery > 0 ? kPolyEvery : 1;
+// Every PolyEvery<D>-th pair of exponentials (unmasked tiles only) may be computed on
+// the FMA pipe with exp2_poly instead of MUFU; 0 keeps all of them on MUFU.
+template <int D>
+struct PolyEvery {
+  static constexpr int value = 0;
+};
 constexpr uint32_t kTmemCols = 512;
 
 template <int D>
@@ -368,16 +369,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < kBN; ++c)
             if (kv0 + c >= lim) s[c] = -INFINITY;
         }
-        // row max as 8 independent chains folded at the end (a single chain of 128
-        // dependent max operations would sit on the critical path of every tile)
+        // row max as 8 independent chains of 3-input max folded at the end (a single
+        // chain of 128 dependent max operations would sit on the critical path)
         float mx8[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) mx8[k] = s[k];
 #pragma unroll
-        for (int c = 8; c < kBN; ++c) mx8[c % 8] = fmaxf(mx8[c % 8], s[c]);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) mx8[k] = fmaxf(mx8[k], mx8[k + 4]);
-        const float mx = fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3]));
+        for (int c = 8; c < kBN; c += 2) mx8[(c / 2) % 8] = max3(mx8[(c / 2) % 8], s[c], s[c + 1]);
+        const float mx = max3(max3(mx8[0], mx8[1], mx8[2]), max3(mx8[3], mx8[4], mx8[5]),
+                              fmaxf(mx8[6], mx8[7]));
         const float m_tile = mx * args.scale_log2;
         float alpha = 1.f;
         bool rescale = false;
@@ -406,33 +406,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         l *= alpha;
         const float mref = (m == -INFINITY) ? 0.f : m;
+        // p = 2^(s * scale * log2e - m): the scale-and-subtract and the row sum run on
+        // packed float pairs (one instruction per two entries), the exponentials on MUFU
         uint32_t pk[kBN / 2];
-        float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        if (need_mask) {
-          // masked tiles: every exponential on MUFU, so masked entries are exactly 0
+        const uint64_t scale2 = f32x2(args.scale_log2, args.scale_log2);
+        const uint64_t negm2 = f32x2(-mref, -mref);
+        uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};
+        constexpr int kEvery = PolyEvery<D>::value;
+        constexpr int kStride = kEvery > 0 ? kEvery : 1;
 #pragma unroll
-          for (int c = 0; c < kBN / 2; ++c) {
-            const float p0 = ex2_approx(fmaf(s[2 * c], args.scale_log2, -mref));
-            const float p1 = ex2_approx(fmaf(s[2 * c + 1], args.scale_log2, -mref));
-            ls[(2 * c) % 8] += p0;
-            ls[(2 * c + 1) % 8] += p1;
-            pk[c] = pack_bf16x2(p0, p1);
-          }
-        } else {
-          // the MUFU unit (16 exp2 per clock per SM) costs as much per score tile as
-          // the two MMAs; every kPolyEvery-th pair goes to the FMA pipe instead
-#pragma unroll
-          for (int c = 0; c < kBN / 2; ++c) {
-            const float x0 = fmaf(s[2 * c], args.scale_log2, -mref);
-            const float x1 = fmaf(s[2 * c + 1], args.scale_log2, -mref);
-            const bool poly = kPolyEvery > 0 && c % kPolyStride == kPolyStride - 1;
-            const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
-            const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);
-            ls[(2 * c) % 8] += p0;
-            ls[(2 * c + 1) % 8] += p1;
-            pk[c] = pack_bf16x2(p0, p1);
-          }
+        for (int c = 0; c < kBN / 2; ++c) {
+          float x0, x1;
+          f32x2_split(fma_x2(f32x2(s[2 * c], s[2 * c + 1]), scale2, negm2), x0, x1);
+          // every kEvery-th pair may go to the FMA pipe (never on masked tiles, so masked
+          // entries stay exactly 0)
+          const bool poly = kEvery > 0 && !need_mask && c % kStride == kStride - 1;
+          const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
+          const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);
+          ls2[c % 4] = add_x2(ls2[c % 4], f32x2(p0, p1));
+          pk[c] = pack_bf16x2(p0, p1);
         }
+        float ls[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) f32x2_split(ls2[k], ls[2 * k], ls[2 * k + 1]);
         l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
         tmem_st32(tSrow, &pk[0]);
         tmem_st32(tSrow + 32, &pk[32]);

@@ -38,9 +38,9 @@ cudaError_t launch_fwd_sm100(const CUtensorMap& tmQ, const CUtensorMap& tmK,
 cudaError_t launch_fwd_f32(const float* Q, const float* K, const float* V, float* O,
                            float* LSE, const Problem& p, cudaStream_t stream);
 
-// Backward, bf16: D = rowsum(dO * O) and L2 = LSE * log2(e) into the workspace, then
-// dK/dV, then dQ.  Workspace layout: D as [BH][Npad] float, then L2 as [BH][Npad] float,
-// Npad = bwd_padded_rows(N).  tmL2 / tmD describe those two arrays as 3-D
+// Backward, bf16: -D = -rowsum(dO * O) and -L2 = -LSE * log2(e) into the workspace,
+// then dK/dV, then dQ.  Workspace layout: -D as [BH][Npad] float, then -L2 as [BH][Npad]
+// float, Npad = bwd_padded_rows(N).  tmL2 / tmD describe those two arrays as 3-D
 // [1][BH][Npad] float tensors with 128 x 1 x 1 boxes.
 int bwd_padded_rows(int N);
 cudaError_t launch_bwd_sm100(const CUtensorMap& tmQ, const CUtensorMap& tmK,
