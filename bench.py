@@ -168,7 +168,8 @@ def time_oracle(w, max_seconds: float = 20.0):
     flops = heads * (traffic.fwd_flops(1, 1, w.N, w.d, w.causal) +
                      traffic.bwd_flops(1, 1, w.N, w.d, w.causal))
     sample = (f"fp64 oracle forward+backward of {heads} whole head(s) of the workload "
-              f"(N={w.N}, d={w.d}, causal={w.causal}); credited FLOPs per second")
+              f"(N={w.N}, d={w.d}, causal={w.causal}); credited FLOPs per second; "
+              f"extrapolated full step ({w.B * w.H} heads) = {el * w.B * w.H / heads:.0f} s")
     return flops / el / 1e12, int(threads), sample, el
 
 
@@ -399,7 +400,9 @@ def run_sweep(args):
                         torch.cuda.synchronize()
                         times.append(e0.elapsed_time(e1))
                     ms = statistics.median(times)
-                    res[name] = {"ms": ms, "tflops": flops / (ms * 1e-3) / 1e12,
+                    pct = statistics.quantiles(times, n=10) if len(times) > 1 else [ms] * 9
+                    res[name] = {"ms": ms, "ms_p10": pct[0], "ms_p90": pct[-1],
+                                 "tflops": flops / (ms * 1e-3) / 1e12,
                                  "frac": flops / (ms * 1e-3) / 1e12 / peak}
                 binding.check_device_error()
                 print(json.dumps({"sweep": "attention TFLOP/s vs N", "N": N, "B": B, "H": H, "d": d,

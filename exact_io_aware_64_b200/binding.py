@@ -37,6 +37,8 @@ SIGNATURES = {
     "fa_bwd_workspace_bytes": ([_i, _i, _i, _i], _sz),
     "fa_bwd": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _sz,
                 _vp], _i),
+    "fa_bwd_f32": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp,
+                    _sz, _vp], _i),
     "fa_bwd_noalloc": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i,
                         _vp], _i),
     "fa_bwd_noalloc_max_scratch_bytes": ([], _sz),
@@ -140,10 +142,16 @@ def bwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, O: torch.Tensor,
         dK: Optional[torch.Tensor] = None, dV: Optional[torch.Tensor] = None,
         workspace: Optional[torch.Tensor] = None,
         stream: Optional[torch.cuda.Stream] = None):
-    """Exact attention backward through ``fa_bwd`` (bf16).  Returns (dQ, dK, dV)."""
+    """Exact attention backward through ``fa_bwd`` (bf16) or ``fa_bwd_f32`` (float32).
+
+    Q, K, V, O, dO: [B, H, N, d] CUDA tensors, contiguous, all bf16 or all float32;
+    LSE: [B, H, N] float32.  Returns (dQ, dK, dV) in the inputs' dtype."""
     B, H, N, d = Q.shape
+    dtype = Q.dtype
+    if dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("Q, K, V, O, dO must be bfloat16 or float32")
     for name, t in (("Q", Q), ("K", K), ("V", V), ("O", O), ("dO", dO)):
-        _check_bhnd(name, t, (B, H, N, d), torch.bfloat16)
+        _check_bhnd(name, t, (B, H, N, d), dtype)
     _check_bhnd("LSE", LSE, (B, H, N), torch.float32)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
@@ -151,16 +159,18 @@ def bwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, O: torch.Tensor,
     dK = torch.empty_like(K) if dK is None else dK
     dV = torch.empty_like(V) if dV is None else dV
     for name, t in (("dQ", dQ), ("dK", dK), ("dV", dV)):
-        _check_bhnd(name, t, (B, H, N, d), torch.bfloat16)
+        _check_bhnd(name, t, (B, H, N, d), dtype)
     need = workspace_bytes(B, H, N, d)
     if workspace is None:
         workspace = torch.empty(max(need, 1), device=Q.device, dtype=torch.uint8)
     ws_bytes = workspace.numel() * workspace.element_size()
+    name = "fa_bwd" if dtype == torch.bfloat16 else "fa_bwd_f32"
     with torch.cuda.device(Q.device):
-        st = lib().fa_bwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _ptr(LSE), _ptr(dQ),
-                          _ptr(dK), _ptr(dV), B, H, N, d, float(scale), int(bool(causal)),
-                          _ptr(workspace), ws_bytes, _stream_handle(stream))
-    _check("fa_bwd", st)
+        st = getattr(lib(), name)(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _ptr(LSE),
+                                  _ptr(dQ), _ptr(dK), _ptr(dV), B, H, N, d, float(scale),
+                                  int(bool(causal)), _ptr(workspace), ws_bytes,
+                                  _stream_handle(stream))
+    _check(name, st)
     return dQ, dK, dV
 
 

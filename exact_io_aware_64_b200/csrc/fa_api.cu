@@ -170,6 +170,44 @@ fa_status check_ptr(const void* p, const char* name) {
     if (_s != FA_OK) return _s;        \
   } while (0)
 
+// Argument checks of fa_bwd and fa_bwd_f32 (elem = bytes per element of the tensors).
+fa_status check_bwd_args(const void* Q, const void* K, const void* V, const void* O,
+                         const void* dO, const float* LSE, const void* dQ, const void* dK,
+                         const void* dV, int B, int H, int N, int d, float scale, int causal,
+                         const void* workspace, size_t workspace_bytes, size_t elem,
+                         bool* noop) {
+  FA_TRY(check_common(B, H, N, d, scale, causal, noop));
+  if (*noop) return FA_OK;
+  FA_TRY(check_ptr(Q, "Q"));
+  FA_TRY(check_ptr(K, "K"));
+  FA_TRY(check_ptr(V, "V"));
+  FA_TRY(check_ptr(O, "O"));
+  FA_TRY(check_ptr(dO, "dO"));
+  FA_TRY(check_ptr(LSE, "LSE"));
+  FA_TRY(check_ptr(dQ, "dQ"));
+  FA_TRY(check_ptr(dK, "dK"));
+  FA_TRY(check_ptr(dV, "dV"));
+  const size_t need = fa_bwd_workspace_bytes(B, H, N, d);
+  if (need > 0) {
+    FA_TRY(check_ptr(workspace, "workspace"));
+    if (workspace_bytes < need)
+      return fail(FA_ERR_INVALID_ARG, "workspace has %zu bytes, %zu needed", workspace_bytes,
+                  need);
+  }
+  const size_t bytes = static_cast<size_t>(B) * H * N * d * elem;
+  const void* ins[5] = {Q, K, V, O, dO};
+  const void* outs[3] = {dQ, dK, dV};
+  for (const void* o : outs) {
+    for (const void* in : ins)
+      if (overlaps(o, in, bytes)) return fail(FA_ERR_INVALID_ARG, "a gradient overlaps an input");
+    if (need > 0 && overlaps(o, bytes, workspace, need))
+      return fail(FA_ERR_INVALID_ARG, "a gradient overlaps the workspace");
+  }
+  if (overlaps(dQ, dK, bytes) || overlaps(dQ, dV, bytes) || overlaps(dK, dV, bytes))
+    return fail(FA_ERR_INVALID_ARG, "gradients overlap each other");
+  return FA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -267,35 +305,9 @@ fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, con
                  cudaStream_t stream) {
   g_last_error[0] = '\0';
   bool noop = false;
-  FA_TRY(check_common(B, H, N, d, scale, causal, &noop));
+  FA_TRY(check_bwd_args(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, scale, causal, workspace,
+                        workspace_bytes, 2, &noop));
   if (noop) return FA_OK;  // empty problem: the pointers are never used (may be NULL)
-  FA_TRY(check_ptr(Q, "Q"));
-  FA_TRY(check_ptr(K, "K"));
-  FA_TRY(check_ptr(V, "V"));
-  FA_TRY(check_ptr(O, "O"));
-  FA_TRY(check_ptr(dO, "dO"));
-  FA_TRY(check_ptr(LSE, "LSE"));
-  FA_TRY(check_ptr(dQ, "dQ"));
-  FA_TRY(check_ptr(dK, "dK"));
-  FA_TRY(check_ptr(dV, "dV"));
-  const size_t need = fa_bwd_workspace_bytes(B, H, N, d);
-  if (need > 0) {
-    FA_TRY(check_ptr(workspace, "workspace"));
-    if (workspace_bytes < need)
-      return fail(FA_ERR_INVALID_ARG, "workspace has %zu bytes, %zu needed", workspace_bytes,
-                  need);
-  }
-  const size_t bytes = static_cast<size_t>(B) * H * N * d * 2;
-  const void* ins[5] = {Q, K, V, O, dO};
-  void* outs[3] = {dQ, dK, dV};
-  for (void* o : outs) {
-    for (const void* in : ins)
-      if (overlaps(o, in, bytes)) return fail(FA_ERR_INVALID_ARG, "a gradient overlaps an input");
-    if (need > 0 && overlaps(o, bytes, workspace, need))
-      return fail(FA_ERR_INVALID_ARG, "a gradient overlaps the workspace");
-  }
-  if (overlaps(dQ, dK, bytes) || overlaps(dQ, dV, bytes) || overlaps(dK, dV, bytes))
-    return fail(FA_ERR_INVALID_ARG, "gradients overlap each other");
   DeviceInfo dev;
   FA_TRY(device_info(&dev));
   FA_TRY(require_sm100(dev));
@@ -313,6 +325,25 @@ fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, con
   cudaError_t e = fa::launch_bwd_sm100(tmQ, tmK, tmV, tmdO, tmL2, tmD, O, dO, LSE, dQ, dK, dV,
                                        ws, p, dev.num_sms, stream);
   if (e != cudaSuccess) return cuda_fail(e, "launching the backward kernels");
+  return FA_OK;
+}
+
+fa_status fa_bwd_f32(const float* Q, const float* K, const float* V, const float* O,
+                     const float* dO, const float* LSE, float* dQ, float* dK, float* dV, int B,
+                     int H, int N, int d, float scale, int causal, void* workspace,
+                     size_t workspace_bytes, cudaStream_t stream) {
+  g_last_error[0] = '\0';
+  bool noop = false;
+  FA_TRY(check_bwd_args(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, scale, causal, workspace,
+                        workspace_bytes, 4, &noop));
+  if (noop) return FA_OK;  // empty problem: the pointers are never used (may be NULL)
+  DeviceInfo dev;
+  FA_TRY(device_info(&dev));
+  fa::Problem p{B * H, N, d, scale, causal, dev.err, g_n_trace ? g_trace : nullptr,
+                g_n_trace};
+  cudaError_t e = fa::launch_bwd_f32(Q, K, V, O, dO, LSE, dQ, dK, dV,
+                                     static_cast<float*>(workspace), p, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "launching the float32 backward kernels");
   return FA_OK;
 }
 

@@ -8,6 +8,8 @@
 // Mapping: a CTA of 128 threads owns 32 query rows of one (batch, head); four threads
 // share a row, each holding every fourth element of q and acc, and combine their partial
 // dot products with two shuffles.  The key and value blocks are staged in shared memory.
+// Blocks are numbered flat over (head, row block), so B*H is not limited by the grid's y
+// extent.
 #include <cmath>
 #include <cstdint>
 
@@ -24,15 +26,16 @@ template <int D>
 __global__ void __launch_bounds__(kThreads)
     fwd_f32_kernel(const float* __restrict__ Q, const float* __restrict__ K,
                    const float* __restrict__ V, float* __restrict__ O,
-                   float* __restrict__ LSE, int N, float scale, int causal) {
+                   float* __restrict__ LSE, int N, int tiles, float scale, int causal) {
   constexpr int E = D / 4;  // elements of q / acc per thread
   __shared__ float Ks[kKeys][D];
   __shared__ float Vs[kKeys][D];
 
-  const int bh = blockIdx.y;
+  const int bh = blockIdx.x / tiles;
+  const int tile = blockIdx.x % tiles;
   const int r = threadIdx.x / 4;  // row within the CTA
   const int part = threadIdx.x % 4;
-  const int row = blockIdx.x * kRows + r;
+  const int row = tile * kRows + r;
   const bool valid = row < N;
   const size_t head = static_cast<size_t>(bh) * N * D;
 
@@ -44,7 +47,7 @@ __global__ void __launch_bounds__(kThreads)
   }
   float m = -INFINITY, l = 0.f;
 
-  const int last_row = min(N - 1, (blockIdx.x + 1) * kRows - 1);
+  const int last_row = min(N - 1, (tile + 1) * kRows - 1);
   const int key_end = causal ? last_row + 1 : N;
   for (int k0 = 0; k0 < key_end; k0 += kKeys) {
     __syncthreads();
@@ -99,10 +102,12 @@ __global__ void __launch_bounds__(kThreads)
 template <int D>
 cudaError_t launch_d(const float* Q, const float* K, const float* V, float* O, float* LSE,
                      const Problem& p, cudaStream_t stream) {
-  dim3 grid((p.N + kRows - 1) / kRows, p.BH);
+  const int tiles = (p.N + kRows - 1) / kRows;
+  const unsigned grid = static_cast<unsigned>(tiles) * static_cast<unsigned>(p.BH);
   cudaError_t e = trace_mark(p, 0, stream);
   if (e != cudaSuccess) return e;
-  fwd_f32_kernel<D><<<grid, kThreads, 0, stream>>>(Q, K, V, O, LSE, p.N, p.scale, p.causal);
+  fwd_f32_kernel<D><<<grid, kThreads, 0, stream>>>(Q, K, V, O, LSE, p.N, tiles, p.scale,
+                                                   p.causal);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   return trace_mark(p, 1, stream);
 }

@@ -50,4 +50,10 @@ cudaError_t launch_bwd_sm100(const CUtensorMap& tmQ, const CUtensorMap& tmK,
                              float* workspace, const Problem& p, int num_sms,
                              cudaStream_t stream);
 
+// Backward, float32 on the CUDA cores: D = rowsum(dO * O) into the workspace as
+// [BH][N] float, then dK/dV, then dQ.
+cudaError_t launch_bwd_f32(const float* Q, const float* K, const float* V, const float* O,
+                           const float* dO, const float* LSE, float* dQ, float* dK, float* dV,
+                           float* workspace, const Problem& p, cudaStream_t stream);
+
 }  // namespace fa

@@ -94,7 +94,7 @@ FA_API fa_status fa_fwd_f32(const float* Q, const float* K, const float* V, floa
                      cudaStream_t stream);
 
 /*
- * Bytes of scratch that fa_bwd needs for given sizes: two float32 per query row
+ * Bytes of scratch that fa_bwd (and fa_bwd_f32) needs for given sizes: two float32 per query row
  * (D_i = sum_k dO_ik O_ik and LSE_i * log2(e)), rows padded to a multiple of 128,
  * rounded up to 256 bytes: 8 * B * H * ceil(N/128) * 128.  Grows as B*H*N, never as N^2.
  */
@@ -116,6 +116,22 @@ FA_API fa_status fa_bwd(const void* Q, const void* K, const void* V, const void*
                  const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
                  int B, int H, int N, int d, float scale, int causal,
                  void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Backward pass, float32: the same computation as fa_bwd with float32 inputs, outputs
+ * and arithmetic (on the CUDA cores; no tensor cores, no bf16 rounding of P or dS).
+ *   Q, K, V, O, dO in : [B,H,N,d] float32
+ *   LSE            in : [B,H,N] float32 from fa_fwd_f32 with the same scale and causal
+ *   dQ, dK, dV     out: [B,H,N,d] float32; must not overlap the inputs or each other
+ *   workspace         : as for fa_bwd (fa_bwd_workspace_bytes(B,H,N,d) bytes, 16-byte
+ *                       aligned); the first 4*B*H*N bytes receive D
+ * Three kernels on `stream` (D; dK and dV per 32 key rows; dQ per 32 query rows), no
+ * atomics.  Errors as for fa_bwd; any sm_100 device.
+ */
+FA_API fa_status fa_bwd_f32(const float* Q, const float* K, const float* V, const float* O,
+                            const float* dO, const float* LSE, float* dQ, float* dK,
+                            float* dV, int B, int H, int N, int d, float scale, int causal,
+                            void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * fa_bwd for callers that cannot allocate device memory (no counterpart on the pages:
@@ -145,9 +161,10 @@ FA_API size_t fa_bwd_noalloc_max_scratch_bytes(void);
 
 /*
  * Kernel-boundary timing, for profilers.  While a list of events is set on the calling
- * thread, every fa_fwd, fa_fwd_f32 and fa_bwd call records events[0] on its stream just
- * before its first kernel and events[k] just after its k-th kernel; fa_fwd and
- * fa_fwd_f32 launch one kernel, fa_bwd three (D/LSE preparation, dK/dV, dQ).  Boundaries
+ * thread, every fa_fwd, fa_fwd_f32, fa_bwd and fa_bwd_f32 call records events[0] on its
+ * stream just before its first kernel and events[k] just after its k-th kernel; fa_fwd
+ * and fa_fwd_f32 launch one kernel, fa_bwd and fa_bwd_f32 three (D preparation, dK/dV,
+ * dQ).  Boundaries
  * beyond n - 1 are not recorded.  The events are caller-created cudaEvent_t (timing
  * enabled) and stay caller-owned.  fa_trace_events(NULL, 0) stops recording.
  * Returns FA_ERR_INVALID_ARG if n < 0, n > 8, or events is NULL with n > 0.

@@ -32,8 +32,8 @@ def lib():
 
 def test_header_declares_the_boundary():
     names = _declared_functions()
-    for required in ("fa_fwd", "fa_bwd", "fa_fwd_f32", "fa_bwd_workspace_bytes",
-                     "fa_status_string", "fa_check_device_error"):
+    for required in ("fa_fwd", "fa_bwd", "fa_fwd_f32", "fa_bwd_f32",
+                     "fa_bwd_workspace_bytes", "fa_status_string", "fa_check_device_error"):
         assert required in names
 
 
@@ -98,9 +98,11 @@ def test_empty_problems_are_noops(lib):
     assert lib.fa_fwd_f32(A, B_, C, D_, E, 1, 3, 0, 128, 0.1, 1, None) == binding.FA_OK
 
 
-def test_bwd_validation(lib):
+@pytest.mark.parametrize("fn,elem", [("fa_bwd", 2), ("fa_bwd_f32", 4)])
+def test_bwd_validation(lib, fn, elem):
     F, G, H_, I, J = 0x600000, 0x700000, 0x800000, 0x900000, 0xA00000
     args = [A, B_, C, D_, E, F, G, H_, I, 1, 2, 64, 128, 0.1, 1, J, 1 << 20, None]
+    call_fn = getattr(lib, fn)
 
     def call(**kw):
         a = list(args)
@@ -108,20 +110,28 @@ def test_bwd_validation(lib):
                  "scale", "causal", "ws", "ws_bytes", "stream"]
         for k, v in kw.items():
             a[names.index(k)] = v
-        return lib.fa_bwd(*a)
+        return call_fn(*a)
 
     assert call(B=0) == binding.FA_OK                      # empty: no-op
+    assert call(N=0, Q=0, dQ=0) == binding.FA_OK           # empty: NULL pointers allowed
     assert lib.fa_fwd(0, 0, 0, 0, 0, 1, 1, 0, 64, 0.1, 0, None) == binding.FA_OK
     assert call(LSE=0) == binding.FA_ERR_INVALID_ARG        # LSE required
+    assert call(dO=0) == binding.FA_ERR_INVALID_ARG
     assert call(ws=0) == binding.FA_ERR_INVALID_ARG
     assert call(ws_bytes=100) == binding.FA_ERR_INVALID_ARG
     assert call(d=80) == binding.FA_ERR_UNSUPPORTED
+    assert call(causal=3) == binding.FA_ERR_INVALID_ARG
+    assert call(scale=-1.0) == binding.FA_ERR_INVALID_ARG
     assert call(dQ=A) == binding.FA_ERR_INVALID_ARG         # gradient overlaps an input
     assert call(dK=G) == binding.FA_ERR_INVALID_ARG         # gradients overlap
     assert call(ws=H_) == binding.FA_ERR_INVALID_ARG        # workspace overlaps dK
-    # a workspace right after a small gradient does not overlap it
-    small = [A, B_, C, D_, E, F, G, H_, I, 1, 1, 1, 64, 0.1, 0, I + 128, 1024, None]
-    assert lib.fa_bwd(*small) != binding.FA_ERR_INVALID_ARG
+    # the overlap checks use the element size: a gradient that ends where the next
+    # buffer starts does not overlap it, one element more does
+    row = 1 * 1 * 1 * 64 * elem
+    small = [A, B_, C, D_, E, F, G, H_, I, 1, 1, 1, 64, 0.1, 0, I + row, 1024, None]
+    assert call_fn(*small) != binding.FA_ERR_INVALID_ARG
+    small[15] = I + row - 16
+    assert call_fn(*small) == binding.FA_ERR_INVALID_ARG
 
 
 def test_trace_events_validation(lib):

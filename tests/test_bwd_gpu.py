@@ -11,7 +11,7 @@ import torch
 
 import oracle
 from exact_io_aware_64_b200 import binding, inputs
-from parity import BF16_MAX_ABS, assert_bf16_close, errors, to64
+from parity import BF16_MAX_ABS, assert_bf16_close, assert_f32_close, errors, to64
 
 pytestmark = pytest.mark.gpu
 
@@ -184,3 +184,79 @@ def test_bwd_large_logits():
                 f"rel_l2={rel_l2:.3e}")
             _, rel_exact = errors(got, exact[k])
             assert rel_exact <= 1e-2, f"sigma 3 {name} h={h} vs exact: rel_l2={rel_exact:.3e}"
+
+
+# ------------------------------------------------------------------ float32 backward
+def _fwd_bwd_f32(ins, scale, causal):
+    q, k, v, do = (ins[n].cuda() for n in ("Q", "K", "V", "dO"))
+    O, LSE = binding.fwd(q, k, v, scale=scale, causal=causal)
+    dQ, dK, dV = binding.bwd(q, k, v, O, do, LSE, scale=scale, causal=causal)
+    binding.check_device_error()
+    assert dQ.dtype == torch.float32
+    return dQ, dK, dV
+
+
+def _check_head_f32(ins, grads, b, h, scale, causal, what=""):
+    """fa_bwd_f32 against the exact fp64 gradient within the float32 tolerance (every
+    step of both the forward that supplies O and LSE and the backward is float32)."""
+    Q, K, V, dO = (to64(ins[n][b, h]) for n in ("Q", "K", "V", "dO"))
+    ref = oracle.attention_bwd_head(Q, K, V, dO, scale, causal)
+    for got, r, name in zip(grads, ref[:3], ("dQ", "dK", "dV")):
+        assert_f32_close(to64(got[b, h]), r, f"{what} {name} b={b} h={h} causal={causal}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_f32_tiny_workload(causal):
+    # B=1 H=1 N=256 d=64 float32: the configuration the float32 path exists for
+    w = inputs.WORKLOADS["tiny_f32"]
+    ins = inputs.make_inputs(w.B, w.H, w.N, w.d, seed=w.seed, dtype=torch.float32,
+                             with_dO=True)
+    grads = _fwd_bwd_f32(ins, w.scale, causal)
+    _check_head_f32(ins, grads, 0, 0, w.scale, causal, w.name)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("N", [1, 31, 32, 33, 100, 300])
+def test_bwd_f32_small(N, d, causal):
+    ins = inputs.make_inputs(1, 2, N, d, seed=3000 + N, dtype=torch.float32, with_dO=True)
+    scale = 1.0 / np.sqrt(d)
+    grads = _fwd_bwd_f32(ins, scale, causal)
+    for h in range(2):
+        _check_head_f32(ins, grads, 0, h, scale, causal, f"f32 N={N} d={d}")
+
+
+def test_bwd_f32_many_heads_and_large_logits():
+    # blocks are numbered flat over (head, row block): 3 * 7 heads of 3 row blocks; logits
+    # of std 9 exercise the exponentials far from the row maximum
+    B, H, N, d = 3, 7, 70, 128
+    ins = inputs.make_inputs(B, H, N, d, seed=77, sigma_qk=3.0, dtype=torch.float32,
+                             with_dO=True)
+    scale = d ** -0.5
+    grads = _fwd_bwd_f32(ins, scale, True)
+    for b, h in ((0, 0), (1, 3), (2, 6)):
+        _check_head_f32(ins, grads, b, h, scale, True, "f32 many heads")
+
+
+def test_bwd_f32_deterministic_and_in_bounds():
+    B, H, N, d = 1, 3, 333, 64
+    ins = inputs.make_inputs(B, H, N, d, seed=9, dtype=torch.float32, with_dO=True)
+    q, k, v, do = (ins[n].cuda() for n in ("Q", "K", "V", "dO"))
+    O, LSE = binding.fwd(q, k, v, causal=False)
+    guard = 1024
+    n = B * H * N * d
+    bufs = [torch.full((2 * guard + n,), 7.0, device="cuda") for _ in range(3)]
+    views = [b[guard:guard + n].view(B, H, N, d) for b in bufs]
+    ws_bytes = binding.workspace_bytes(B, H, N, d)
+    wsbuf = torch.full((ws_bytes + 2 * guard,), 0xCD, device="cuda", dtype=torch.uint8)
+    ws = wsbuf[guard:guard + ws_bytes]
+    outs = []
+    for _ in range(2):
+        binding.bwd(q, k, v, O, do, LSE, dQ=views[0], dK=views[1], dV=views[2], workspace=ws)
+        binding.check_device_error()
+        outs.append([t.clone() for t in views])
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
+    for b in bufs:
+        assert bool((b[:guard] == 7.0).all()) and bool((b[-guard:] == 7.0).all())
+    assert bool((wsbuf[:guard] == 0xCD).all()) and bool((wsbuf[-guard:] == 0xCD).all())
