@@ -70,9 +70,9 @@ __device__ __forceinline__ uint32_t split_operand_col(uint32_t base, int kk) {
 }
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
-// Every PolyEvery<D>-th exponential of a row may be computed on the FMA pipe
-// (exp2_poly) instead of the MUFU unit; masked entries are zeroed after the exponential
-// either way; 0 keeps all of them on MUFU.
+// Every PolyEvery<D>-th pair of exponentials of a row may be computed on the FMA pipe
+// (exp2_poly_x2) instead of the MUFU unit; masked entries are zeroed after the
+// exponential either way; 0 keeps all of them on MUFU.
 template <int D>
 struct PolyEvery {
   static constexpr int value = 0;
@@ -453,12 +453,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < kCols; c += 2) {
             // x = S^T * scale * log2e - L2 for two query columns in one packed FMA
             const uint64_t nl = *reinterpret_cast<const uint64_t*>(sL + c);
-            float x0, x1;
-            f32x2_split(fma_x2(f32x2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), scale2, nl),
-                        x0, x1);
-            const bool poly = PolyEvery<D>::value > 0 && c % kStride == kStride - 1;
-            float e0 = poly ? exp2_poly(x0) : ex2_approx(x0);
-            float e1 = poly ? exp2_poly(x1) : ex2_approx(x1);
+            const uint64_t x2 =
+                fma_x2(f32x2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), scale2, nl);
+            const bool poly = PolyEvery<D>::value > 0 && (c / 2) % kStride == kStride - 1;
+            float e0, e1;
+            exp2_pair(x2, poly, e0, e1);
             if (diag && col0 + c < row) e0 = 0.f;  // query i*128+col0+c before key j*128+row
             if (diag && col0 + c + 1 < row) e1 = 0.f;
             p[c] = e0;
@@ -821,12 +820,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t nl2 = f32x2(nl2row, nl2row);
 #pragma unroll
           for (int c = 0; c < kCols; c += 2) {
-            float x0, x1;
-            f32x2_split(fma_x2(f32x2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), scale2, nl2),
-                        x0, x1);
-            const bool poly = PolyEvery<D>::value > 0 && c % kStride == kStride - 1;
-            float e0 = poly ? exp2_poly(x0) : ex2_approx(x0);
-            float e1 = poly ? exp2_poly(x1) : ex2_approx(x1);
+            const uint64_t x2 =
+                fma_x2(f32x2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), scale2, nl2);
+            const bool poly = PolyEvery<D>::value > 0 && (c / 2) % kStride == kStride - 1;
+            float e0, e1;
+            exp2_pair(x2, poly, e0, e1);
             if (need_mask && kv0 + c >= lim) e0 = 0.f;
             if (need_mask && kv0 + c + 1 >= lim) e1 = 0.f;
             p[c] = e0;

@@ -57,7 +57,7 @@ constexpr int kWarpTMA = 8;
 constexpr int kWarpMMA = 9;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // Every PolyEvery<D>-th pair of exponentials (unmasked tiles only) may be computed on
-// the FMA pipe with exp2_poly instead of MUFU; 0 keeps all of them on MUFU.
+// the FMA pipe with exp2_poly_x2 instead of MUFU; 0 keeps all of them on MUFU.
 template <int D>
 struct PolyEvery {
   static constexpr int value = 0;
@@ -416,13 +416,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr int kStride = kEvery > 0 ? kEvery : 1;
 #pragma unroll
         for (int c = 0; c < kBN / 2; ++c) {
-          float x0, x1;
-          f32x2_split(fma_x2(f32x2(s[2 * c], s[2 * c + 1]), scale2, negm2), x0, x1);
+          const uint64_t x2 = fma_x2(f32x2(s[2 * c], s[2 * c + 1]), scale2, negm2);
           // every kEvery-th pair may go to the FMA pipe (never on masked tiles, so masked
           // entries stay exactly 0)
           const bool poly = kEvery > 0 && !need_mask && c % kStride == kStride - 1;
-          const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
-          const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);
+          float p0, p1;
+          exp2_pair(x2, poly, p0, p1);
           ls2[c % 4] = add_x2(ls2[c % 4], f32x2(p0, p1));
           pk[c] = pack_bf16x2(p0, p1);
         }

@@ -1,5 +1,5 @@
 """Coefficients of the cubic that approximates 2^f on [-1/2, 1/2] (minimax in relative
-error), used by exp2_poly() in sm100.cuh.
+error), used by exp2_poly_x2() in sm100.cuh.
 
 Method: Cody-Waite style range reduction x = n + f with n = round(x), 2^x = 2^n * 2^f;
 2^f by a degree-3 polynomial whose coefficients come from the Remez exchange algorithm

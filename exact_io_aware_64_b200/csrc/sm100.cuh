@@ -408,14 +408,37 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 // n), f in [-1/2, 1/2]; 2^f by a cubic fitted with the Remez exchange algorithm on the
 // relative error (gen_exp2_poly.py: max relative error 7.5e-5, well below bf16
 // rounding); 2^n applied by adding n to the exponent field.
-__device__ __forceinline__ float exp2_poly(float x) {
+// Two values at once: the additions and the polynomial run on packed float pairs;
+// x - round(x) is formed as fma(round(x), -1, x), which is exact.
+__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x2) {
   constexpr float kC0 = 0.99992806f, kC1 = 0.69326097f, kC2 = 0.24261113f, kC3 = 0.05517167f;
   constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  x = fmaxf(x, -126.0f);
-  const float t = x + kRound;
-  const float f = x - (t - kRound);
-  const float p = fmaf(fmaf(fmaf(kC3, f, kC2), f, kC1), f, kC0);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+  float x0, x1;
+  f32x2_split(x2, x0, x1);
+  const uint64_t x = f32x2(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+  const uint64_t t = add_x2(x, f32x2(kRound, kRound));
+  const uint64_t n = add_x2(t, f32x2(-kRound, -kRound));
+  const uint64_t f = fma_x2(n, f32x2(-1.0f, -1.0f), x);
+  uint64_t p = fma_x2(f32x2(kC3, kC3), f, f32x2(kC2, kC2));
+  p = fma_x2(p, f, f32x2(kC1, kC1));
+  p = fma_x2(p, f, f32x2(kC0, kC0));
+  float p0, p1, t0, t1;
+  f32x2_split(p, p0, p1);
+  f32x2_split(t, t0, t1);
+  return f32x2(__int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23)),
+               __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23)));
+}
+
+// 2^x of a packed pair, on MUFU (ex2.approx) or, when `poly`, on the FMA pipe.
+__device__ __forceinline__ void exp2_pair(uint64_t x2, bool poly, float& e0, float& e1) {
+  if (poly) {
+    f32x2_split(exp2_poly_x2(x2), e0, e1);
+  } else {
+    float x0, x1;
+    f32x2_split(x2, x0, x1);
+    e0 = ex2_approx(x0);
+    e1 = ex2_approx(x1);
+  }
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -67,9 +67,10 @@ def _exp2_poly_coefficients():
 
 
 def test_exp2_poly_matches_its_generator_and_error_bound():
-    """The kernel's FMA-pipe exp2 (range reduction + cubic): its coefficients are the
-    Remez fit that csrc/gen_exp2_poly.py produces, and the float32 arithmetic the kernel
-    performs stays within the fit's relative-error bound over the range it is used on."""
+    """The kernels' FMA-pipe exp2 (exp2_poly_x2: range reduction + cubic): its
+    coefficients are the Remez fit that csrc/gen_exp2_poly.py produces, and the float32
+    arithmetic it performs (each step exactly rounded, x - round(x) exact) stays within
+    the fit's relative-error bound over the range it is used on."""
     import importlib.util
     import numpy as np
     c = _exp2_poly_coefficients()
