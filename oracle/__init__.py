@@ -1,5 +1,6 @@
 """fp64 CPU oracle for exact attention.  Test infrastructure only (see attention.py)."""
 from .attention import (  # noqa: F401
+    chunk_positions,
     scores,
     softmax_rows,
     attention_head,

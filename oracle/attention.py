@@ -15,7 +15,11 @@ What it computes, and where the pages fix it
 * The per-row log-sum-exp (LSE) that the forward also returns is the natural-log
   normaliser of the scaled, masked logits: LSE_i = log sum_j exp(S_ij).
 * Causal masking (query i sees keys j <= i, same length for queries and keys) is not on
-  the pages; it is the plain reading used throughout this library.
+  the pages; it is the plain reading used throughout this library.  With fewer queries
+  than keys (Nq < Nk: a chunk of new tokens whose keys follow those of earlier tokens)
+  the queries are the last Nq tokens of the sequence, query i at position i + Nk - Nq
+  (``chunk_positions``), so under causal masking it sees keys j <= i + Nk - Nq
+  (bottom-right alignment); with Nq == Nk this is the rule above.
 * ``attention_head_tiled`` is a second, independent route to the same numbers: the
   online-softmax recurrence of "FlashAttention, simplified", "The trick" (running max m,
   running sum l, accumulator acc, rescale by alpha = exp(m - m_new), one division by l at
@@ -39,6 +43,14 @@ def _f64(x) -> np.ndarray:
 
 def _rows(n_q: int, q_index) -> np.ndarray:
     return np.arange(n_q) if q_index is None else np.asarray(q_index, dtype=np.int64)
+
+
+def chunk_positions(n_q: int, n_k: int) -> np.ndarray:
+    """Positions of n_q queries that are the last n_q tokens of an n_k-token sequence:
+    query i sits at i + n_k - n_q (0..n-1 when n_q == n_k).  Needs n_q <= n_k."""
+    if n_q > n_k:
+        raise ValueError(f"{n_q} queries cannot be the last tokens of {n_k} keys")
+    return np.arange(n_q) + (n_k - n_q)
 
 
 def scores(Q, K, scale: float, causal: bool, q_index=None) -> np.ndarray:
@@ -130,7 +142,7 @@ def attention_head_tiled(Q, K, V, scale: float, causal: bool, block_q: int, bloc
     return O, LSE
 
 
-def attention_bwd_head(Q, K, V, dO, scale: float, causal: bool, O_given=None):
+def attention_bwd_head(Q, K, V, dO, scale: float, causal: bool, O_given=None, q_index=None):
     """Analytic gradients of O = softmax(scale Q K^T [masked]) V for one head.
 
     Returns (dQ, dK, dV, D) where D_i = sum_k dO_ik O_ik.  Masked entries have P = 0 and
@@ -139,13 +151,14 @@ def attention_bwd_head(Q, K, V, dO, scale: float, causal: bool, O_given=None):
     By default D uses the exact O.  A backward pass that is handed the forward's output
     (as the recompute-based backward is) forms D from that stored O instead; pass it as
     ``O_given`` to get exactly that computation.  With O_given equal to the exact O the
-    two agree.
+    two agree.  ``q_index`` gives the query rows' positions as in ``scores`` (default
+    0..n_q-1).
     """
     Q = _f64(Q)
     K = _f64(K)
     V = _f64(V)
     dO = _f64(dO)
-    O, _, P = attention_head(Q, K, V, scale, causal)
+    O, _, P = attention_head(Q, K, V, scale, causal, q_index)
     if O_given is not None:
         O = _f64(O_given)
     dV = P.T @ dO
@@ -176,22 +189,27 @@ def attention_bwd_dq_rows(Q_rows, K, V, dO_rows, scale: float, causal: bool, q_i
 
 
 def attention_fwd(Q, K, V, scale: float, causal: bool):
-    """Forward over [B, H, N, d] arrays: returns (O [B,H,N,d], LSE [B,H,N]), float64."""
+    """Forward over Q [B, H, Nq, d], K and V [B, H, Nk, d] (Nq <= Nk when causal; the
+    queries are the last Nq tokens, see ``chunk_positions``): returns (O [B,H,Nq,d],
+    LSE [B,H,Nq]), float64."""
     Q = _f64(Q)
     B, H, N, _ = Q.shape
+    pos = chunk_positions(N, np.shape(K)[2]) if causal else None
     O = np.empty(Q.shape[:3] + (np.shape(V)[3],))
     LSE = np.empty((B, H, N))
     for b in range(B):
         for h in range(H):
             O[b, h], LSE[b, h], _ = attention_head(Q[b, h], np.asarray(K)[b, h],
-                                                   np.asarray(V)[b, h], scale, causal)
+                                                   np.asarray(V)[b, h], scale, causal, pos)
     return O, LSE
 
 
 def attention_bwd(Q, K, V, dO, scale: float, causal: bool):
-    """Backward over [B, H, N, d] arrays: returns (dQ, dK, dV, D), float64."""
+    """Backward over Q, dO [B, H, Nq, d], K, V [B, H, Nk, d] (as ``attention_fwd``):
+    returns (dQ, dK, dV, D), float64."""
     Q = _f64(Q)
     B, H, N, d = Q.shape
+    pos = chunk_positions(N, np.shape(K)[2]) if causal else None
     dQ = np.empty(Q.shape)
     dK = np.empty(np.shape(K))
     dV = np.empty(np.shape(V))
@@ -200,5 +218,5 @@ def attention_bwd(Q, K, V, dO, scale: float, causal: bool):
         for h in range(H):
             dQ[b, h], dK[b, h], dV[b, h], D[b, h] = attention_bwd_head(
                 Q[b, h], np.asarray(K)[b, h], np.asarray(V)[b, h], np.asarray(dO)[b, h],
-                scale, causal)
+                scale, causal, q_index=pos)
     return dQ, dK, dV, D

@@ -176,15 +176,17 @@ def pin_large_logits(A):
         np.testing.assert_allclose(LSEt, LSE + shift, rtol=0, atol=1e-9)
 
 
-def _brute_force_head(Q, K, V, scale, causal):
-    """Softmax attention with Python scalars and loops, one entry at a time."""
+def _brute_force_head(Q, K, V, scale, causal, first_pos=0):
+    """Softmax attention with Python scalars and loops, one entry at a time.  Query i
+    stands at position first_pos + i of the key sequence (causal: it sees keys up to
+    there)."""
     n, dv = len(Q), len(V[0])
     O = [[0.0] * dv for _ in range(n)]
     LSE = [0.0] * n
     for i in range(n):
         logits = []
         for j in range(len(K)):
-            if causal and j > i:
+            if causal and j > first_pos + i:
                 continue
             logits.append((j, scale * sum(Q[i][t] * K[j][t] for t in range(len(Q[i])))))
         big = max(s for _, s in logits)
@@ -209,6 +211,48 @@ def pin_brute_force_small(A):
                 Ob, LSEb = _brute_force_head(Q.tolist(), K.tolist(), V.tolist(), 0.8, causal)
                 np.testing.assert_allclose(O, Ob, rtol=0, atol=1e-14)
                 np.testing.assert_allclose(LSE, LSEb, rtol=0, atol=1e-14)
+
+
+def pin_chunk_brute_force(A):
+    """Fewer queries than keys: the [B, H, N, d] wrapper treats the queries as the last
+    tokens of the key sequence (bottom-right causal alignment), checked entry by entry
+    against Python loops."""
+    rng = _rng(14)
+    for nq, nk in ((1, 3), (2, 3), (2, 5), (3, 4)):
+        Q = rng.standard_normal((nq, 2))
+        K = rng.standard_normal((nk, 2))
+        V = rng.standard_normal((nk, 3))
+        for causal in (False, True):
+            O, LSE = A.attention_fwd(Q[None, None], K[None, None], V[None, None], 0.9, causal)
+            Ob, LSEb = _brute_force_head(Q.tolist(), K.tolist(), V.tolist(), 0.9, causal,
+                                         first_pos=nk - nq)
+            np.testing.assert_allclose(O[0, 0], Ob, rtol=0, atol=1e-14)
+            np.testing.assert_allclose(LSE[0, 0], LSEb, rtol=0, atol=1e-14)
+
+
+def pin_chunk_is_tail_of_full_sequence(A):
+    """Attention of the last Nq queries against all Nk keys equals the last Nq rows of
+    causal attention over the whole sequence; with the gradient of the earlier rows set
+    to zero, the whole sequence's dK, dV and last dQ rows equal the chunk's."""
+    rng = _rng(15)
+    nk, nq, d, scale = 11, 4, 3, 0.8
+    Qf, K, V = (rng.standard_normal((nk, d)) for _ in range(3))
+    G = np.zeros((nk, d))
+    G[nk - nq:] = rng.standard_normal((nq, d))
+    Of, LSEf, _ = A.attention_head(Qf, K, V, scale, True)
+    O, LSE = A.attention_fwd(Qf[None, None, nk - nq:], K[None, None], V[None, None], scale,
+                             True)
+    np.testing.assert_allclose(O[0, 0], Of[nk - nq:], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(LSE[0, 0], LSEf[nk - nq:], rtol=0, atol=1e-14)
+    dQf, dKf, dVf, _ = A.attention_bwd_head(Qf, K, V, G, scale, True)
+    dQ, dK, dV, _ = A.attention_bwd(Qf[None, None, nk - nq:], K[None, None], V[None, None],
+                                    G[None, None, nk - nq:], scale, True)
+    np.testing.assert_allclose(dQ[0, 0], dQf[nk - nq:], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(dK[0, 0], dKf, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(dV[0, 0], dVf, rtol=0, atol=1e-13)
+    np.testing.assert_array_equal(A.chunk_positions(nq, nk), np.arange(nk - nq, nk))
+    with pytest.raises(ValueError):
+        A.chunk_positions(nk + 1, nk)
 
 
 def pin_tiled_matches_naive(A):
@@ -265,6 +309,27 @@ def pin_finite_differences(A):
                 (dV, _fd_grad(lambda X: loss(Q, K, X), V)),
             ):
                 np.testing.assert_allclose(got, fd, rtol=1e-6, atol=1e-8)
+
+
+def pin_chunk_finite_differences(A):
+    """Central differences confirm the backward for queries placed at later positions
+    (fewer queries than keys, causal)."""
+    rng = _rng(16)
+    nq, nk, d, scale = 3, 6, 2, 0.7
+    pos = A.chunk_positions(nq, nk)
+    Q = rng.standard_normal((nq, d))
+    K = rng.standard_normal((nk, d))
+    V = rng.standard_normal((nk, d))
+    G = rng.standard_normal((nq, d))
+    dQ, dK, dV, _ = A.attention_bwd_head(Q, K, V, G, scale, True, q_index=pos)
+
+    def loss(Qx, Kx, Vx):
+        return float((A.attention_head(Qx, Kx, Vx, scale, True, pos)[0] * G).sum())
+
+    for got, fd in ((dQ, _fd_grad(lambda X: loss(X, K, V), Q)),
+                    (dK, _fd_grad(lambda X: loss(Q, X, V), K)),
+                    (dV, _fd_grad(lambda X: loss(Q, K, X), V))):
+        np.testing.assert_allclose(got, fd, rtol=1e-6, atol=1e-8)
 
 
 def pin_dq_rows_finite_differences(A):
@@ -335,8 +400,11 @@ PINS = [
     pin_shift_invariance,
     pin_large_logits,
     pin_brute_force_small,
+    pin_chunk_brute_force,
+    pin_chunk_is_tail_of_full_sequence,
     pin_tiled_matches_naive,
     pin_finite_differences,
+    pin_chunk_finite_differences,
     pin_dq_rows_finite_differences,
     pin_batched_backward,
     pin_backward_with_given_output,
@@ -382,6 +450,14 @@ MUTANTS = [
      "O[b, h], LSE[b, h], _ = attention_head(Q[b, h], np.asarray(K)[b, 0],"),
     ("attention_bwd", "Q[b, h], np.asarray(K)[b, h], np.asarray(V)[b, h], np.asarray(dO)[b, h],",
      "Q[b, h], np.asarray(K)[b, h], np.asarray(V)[0, h], np.asarray(dO)[b, h],"),
+    ("chunk_positions", "return np.arange(n_q) + (n_k - n_q)", "return np.arange(n_q)"),
+    ("chunk_positions", "return np.arange(n_q) + (n_k - n_q)",
+     "return np.arange(n_q) + (n_q - n_k)"),
+    ("attention_bwd_head", "O, _, P = attention_head(Q, K, V, scale, causal, q_index)",
+     "O, _, P = attention_head(Q, K, V, scale, causal)"),
+    ("attention_bwd", "scale, causal, q_index=pos)", "scale, causal)"),
+    ("attention_fwd", "np.asarray(V)[b, h], scale, causal, pos)",
+     "np.asarray(V)[b, h], scale, causal)"),
 ]
 
 
