@@ -33,10 +33,13 @@ _sz = ctypes.c_size_t
 SIGNATURES = {
     "fa_abi_version": ([], _i),
     "fa_fwd": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp], _i),
+    "fa_fwd_qk": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _vp], _i),
     "fa_fwd_f32": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp], _i),
     "fa_bwd_workspace_bytes": ([_i, _i, _i, _i], _sz),
     "fa_bwd": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _sz,
                 _vp], _i),
+    "fa_bwd_qk": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _vp,
+                   _sz, _vp], _i),
     "fa_bwd_f32": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp,
                     _sz, _vp], _i),
     "fa_bwd_noalloc": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i,
@@ -104,31 +107,47 @@ def fwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, scale: Optional[float
         causal: bool = False, O: Optional[torch.Tensor] = None,
         LSE: Optional[torch.Tensor] = None, want_lse: bool = True,
         stream: Optional[torch.cuda.Stream] = None):
-    """Exact attention forward through ``fa_fwd`` (bf16) or ``fa_fwd_f32`` (float32).
+    """Exact attention forward through ``fa_fwd`` (bf16), ``fa_fwd_qk`` (bf16, fewer
+    queries than keys) or ``fa_fwd_f32`` (float32).
 
-    Q, K, V: [B, H, N, d] CUDA tensors, contiguous, all bf16 or all float32.
+    Q: [B, H, Nq, d]; K, V: [B, H, Nk, d]; CUDA tensors, contiguous, all bf16 or all
+    float32.  With Nq != Nk the queries are the last Nq of the Nk tokens (causal masking
+    aligned at the bottom right); the float32 path takes Nq == Nk only.
     Returns (O, LSE); LSE is None when ``want_lse`` is False and none is passed.
     """
-    B, H, N, d = Q.shape
+    B, H, Nq, d = Q.shape
+    Nk = K.shape[2]
     dtype = Q.dtype
     if dtype not in (torch.bfloat16, torch.float32):
         raise ValueError("Q, K, V must be bfloat16 or float32")
-    for name, t in (("Q", Q), ("K", K), ("V", V)):
-        _check_bhnd(name, t, (B, H, N, d), dtype)
+    _check_bhnd("Q", Q, (B, H, Nq, d), dtype)
+    for name, t in (("K", K), ("V", V)):
+        _check_bhnd(name, t, (B, H, Nk, d), dtype)
+    if dtype == torch.float32 and Nq != Nk:
+        raise ValueError("the float32 path takes as many queries as keys")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if O is None:
         O = torch.empty_like(Q)
-    _check_bhnd("O", O, (B, H, N, d), dtype)
+    _check_bhnd("O", O, (B, H, Nq, d), dtype)
     if LSE is None and want_lse:
-        LSE = torch.empty((B, H, N), device=Q.device, dtype=torch.float32)
+        LSE = torch.empty((B, H, Nq), device=Q.device, dtype=torch.float32)
     if LSE is not None:
-        _check_bhnd("LSE", LSE, (B, H, N), torch.float32)
-    fn = lib().fa_fwd if dtype == torch.bfloat16 else lib().fa_fwd_f32
+        _check_bhnd("LSE", LSE, (B, H, Nq), torch.float32)
     with torch.cuda.device(Q.device):
-        st = fn(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), B, H, N, d, float(scale),
-                int(bool(causal)), _stream_handle(stream))
-    _check("fa_fwd" if dtype == torch.bfloat16 else "fa_fwd_f32", st)
+        if dtype == torch.float32:
+            name = "fa_fwd_f32"
+            st = lib().fa_fwd_f32(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), B, H, Nq, d,
+                                  float(scale), int(bool(causal)), _stream_handle(stream))
+        elif Nq == Nk:
+            name = "fa_fwd"
+            st = lib().fa_fwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), B, H, Nq, d,
+                              float(scale), int(bool(causal)), _stream_handle(stream))
+        else:
+            name = "fa_fwd_qk"
+            st = lib().fa_fwd_qk(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), B, H, Nq, Nk,
+                                 d, float(scale), int(bool(causal)), _stream_handle(stream))
+    _check(name, st)
     return O, LSE
 
 
@@ -142,34 +161,48 @@ def bwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, O: torch.Tensor,
         dK: Optional[torch.Tensor] = None, dV: Optional[torch.Tensor] = None,
         workspace: Optional[torch.Tensor] = None,
         stream: Optional[torch.cuda.Stream] = None):
-    """Exact attention backward through ``fa_bwd`` (bf16) or ``fa_bwd_f32`` (float32).
+    """Exact attention backward through ``fa_bwd`` (bf16), ``fa_bwd_qk`` (bf16, fewer
+    queries than keys) or ``fa_bwd_f32`` (float32).
 
-    Q, K, V, O, dO: [B, H, N, d] CUDA tensors, contiguous, all bf16 or all float32;
-    LSE: [B, H, N] float32.  Returns (dQ, dK, dV) in the inputs' dtype."""
-    B, H, N, d = Q.shape
+    Q, O, dO: [B, H, Nq, d]; K, V: [B, H, Nk, d]; CUDA tensors, contiguous, all bf16 or
+    all float32; LSE: [B, H, Nq] float32.  Returns (dQ, dK, dV) in the inputs' dtype."""
+    B, H, Nq, d = Q.shape
+    Nk = K.shape[2]
     dtype = Q.dtype
     if dtype not in (torch.bfloat16, torch.float32):
         raise ValueError("Q, K, V, O, dO must be bfloat16 or float32")
-    for name, t in (("Q", Q), ("K", K), ("V", V), ("O", O), ("dO", dO)):
-        _check_bhnd(name, t, (B, H, N, d), dtype)
-    _check_bhnd("LSE", LSE, (B, H, N), torch.float32)
+    for name, t in (("Q", Q), ("O", O), ("dO", dO)):
+        _check_bhnd(name, t, (B, H, Nq, d), dtype)
+    for name, t in (("K", K), ("V", V)):
+        _check_bhnd(name, t, (B, H, Nk, d), dtype)
+    _check_bhnd("LSE", LSE, (B, H, Nq), torch.float32)
+    if dtype == torch.float32 and Nq != Nk:
+        raise ValueError("the float32 path takes as many queries as keys")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     dQ = torch.empty_like(Q) if dQ is None else dQ
     dK = torch.empty_like(K) if dK is None else dK
     dV = torch.empty_like(V) if dV is None else dV
-    for name, t in (("dQ", dQ), ("dK", dK), ("dV", dV)):
-        _check_bhnd(name, t, (B, H, N, d), dtype)
-    need = workspace_bytes(B, H, N, d)
+    _check_bhnd("dQ", dQ, (B, H, Nq, d), dtype)
+    for name, t in (("dK", dK), ("dV", dV)):
+        _check_bhnd(name, t, (B, H, Nk, d), dtype)
+    need = workspace_bytes(B, H, Nq, d)
     if workspace is None:
         workspace = torch.empty(max(need, 1), device=Q.device, dtype=torch.uint8)
     ws_bytes = workspace.numel() * workspace.element_size()
-    name = "fa_bwd" if dtype == torch.bfloat16 else "fa_bwd_f32"
+    ptrs = (_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _ptr(LSE), _ptr(dQ), _ptr(dK),
+            _ptr(dV))
+    tail = (float(scale), int(bool(causal)), _ptr(workspace), ws_bytes, _stream_handle(stream))
     with torch.cuda.device(Q.device):
-        st = getattr(lib(), name)(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _ptr(LSE),
-                                  _ptr(dQ), _ptr(dK), _ptr(dV), B, H, N, d, float(scale),
-                                  int(bool(causal)), _ptr(workspace), ws_bytes,
-                                  _stream_handle(stream))
+        if dtype == torch.float32:
+            name = "fa_bwd_f32"
+            st = lib().fa_bwd_f32(*ptrs, B, H, Nq, d, *tail)
+        elif Nq == Nk:
+            name = "fa_bwd"
+            st = lib().fa_bwd(*ptrs, B, H, Nq, d, *tail)
+        else:
+            name = "fa_bwd_qk"
+            st = lib().fa_bwd_qk(*ptrs, B, H, Nq, Nk, d, *tail)
     _check(name, st)
     return dQ, dK, dV
 

@@ -145,10 +145,13 @@ struct BwdArgs {
   const float* Dpad;   // [BH][Npad]: -D
   const float* L2pad;  // [BH][Npad]: -LSE * log2(e)
   int BH;
-  int N;
-  int Npad;
-  int n_tiles;      // ceil(N / 128)
-  int total_units;  // BH * n_tiles
+  int Nq;           // query rows per head (Q, O, dO, dQ, LSE)
+  int Nk;           // key rows per head (K, V, dK, dV)
+  int off;          // causal: Nk - Nq, the position of query row 0 among the keys
+  int Npad;         // Nq rounded up to whole tiles
+  int n_qt;         // ceil(Nq / 128)
+  int n_kt;         // ceil(Nk / 128)
+  int total_units;  // this kernel's units: BH * n_kt (dK/dV) or BH * n_qt (dQ)
   int causal;
   float scale;
   float scale_log2;
@@ -265,10 +268,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (args.causal) {
       j = w / args.BH;  // key tile 0 meets every query tile: heaviest first
       bh = w % args.BH;
-      i0 = j;
+      // first query tile with a row whose position reaches key j*128
+      i0 = j * kTile > args.off ? (j * kTile - args.off) / kTile : 0;
     } else {
-      bh = w / args.n_tiles;
-      j = w % args.n_tiles;
+      bh = w / args.n_kt;
+      j = w % args.n_kt;
       i0 = 0;
     }
   };
@@ -295,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d_elect(base + L::kV + c * L::kBoxBytes, &tmV, bar(L::kBarKVFull), c * 64, j * kTile, bh);
       }
       ++kv_loads;
-      for (int i = i0; ok && i < args.n_tiles; ++i) {
+      for (int i = i0; ok && i < args.n_qt; ++i) {
         ok = wait_warp(bar(L::kBarQEmpty + qs), qph ^ 1);
         if (!ok) break;
         mbar_arrive_expect_tx_elect(bar(L::kBarQFull + qs), L::kTileBytes);
@@ -378,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1)
          w = snake_unit(++r), ++units) {
       int bh, j, i0;
       unit(w, bh, j, i0);
-      const int m = args.n_tiles - i0;
+      const int m = args.n_qt - i0;
       ok = wait_warp(bar(L::kBarKVFull), units & 1);
       int curq = 0, curd = 0;
       if (ok) ok = next_s(curq);
@@ -429,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1)
          w = snake_unit(++r), ++units) {
       int bh, j, i0;
       unit(w, bh, j, i0);
-      for (int i = i0; i < args.n_tiles; ++i) {
+      for (int i = i0; i < args.n_qt; ++i) {
         // this tile's L2 and D rows sit in its dO slot
         const uint8_t* sb = smem + L::kDO0 + stage * L::kDOSlotBytes;
         const float* sL = reinterpret_cast<const float*>(sb + L::kSlotL) + col0;
@@ -447,7 +451,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < kCols / 32; ++c)
             tmem_ld32(tS + lane_off + col0 + c * 32, &r[c * 32]);
           tmem_wait_ld();
-          const bool diag = args.causal && i == j;
+          // causal: key j*128+row is hidden from query i*128+col when col < row + delta
+          const int delta = (j - i) * kTile - args.off;
+          const bool diag = args.causal && delta > -kTile;
           const uint64_t scale2 = f32x2(args.scale_log2, args.scale_log2);
 #pragma unroll
           for (int c = 0; c < kCols; c += 2) {
@@ -458,8 +464,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool poly = PolyEvery<D>::value > 0 && (c / 2) % kStride == kStride - 1;
             float e0, e1;
             exp2_pair(x2, poly, e0, e1);
-            if (diag && col0 + c < row) e0 = 0.f;  // query i*128+col0+c before key j*128+row
-            if (diag && col0 + c + 1 < row) e1 = 0.f;
+            if (diag && col0 + c < row + delta) e0 = 0.f;
+            if (diag && col0 + c + 1 < row + delta) e1 = 0.f;
             p[c] = e0;
             p[c + 1] = e1;
           }
@@ -508,16 +514,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const int kv_row = j * kTile + row;
-      const size_t off = (static_cast<size_t>(bh) * args.N + kv_row) * D;
+      const size_t off = (static_cast<size_t>(bh) * args.Nk + kv_row) * D;
 #pragma unroll 1
       for (int c = g * (D / 64); c < (g + 1) * (D / 64); ++c) {
         uint32_t v[32];
         tmem_ld32(tdV + lane_off + c * 32, v);
         tmem_wait_ld();
-        if (kv_row < args.N) store_row32(args.dV + off + c * 32, v, 1.f);
+        if (kv_row < args.Nk) store_row32(args.dV + off + c * 32, v, 1.f);
         tmem_ld32(tdK + lane_off + c * 32, v);
         tmem_wait_ld();
-        if (kv_row < args.N) store_row32(args.dK + off + c * 32, v, args.scale);
+        if (kv_row < args.Nk) store_row32(args.dK + off + c * 32, v, args.scale);
       }
       warp_arrive(bar(L::kBarAccFree));
     }
@@ -627,13 +633,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   auto unit = [&](int w, int& bh, int& i, int& m) {
     if (args.causal) {
-      i = args.n_tiles - 1 - w / args.BH;  // last query tile meets every key tile
+      i = args.n_qt - 1 - w / args.BH;  // last query tile meets the most key tiles
       bh = w % args.BH;
-      m = i + 1;
+      // key tiles up to the one holding the position of the tile's last row
+      m = min((i * kTile + kTile - 1 + args.off) / kTile + 1, args.n_kt);
     } else {
-      bh = w / args.n_tiles;
-      i = w % args.n_tiles;
-      m = args.n_tiles;
+      bh = w / args.n_qt;
+      i = w % args.n_qt;
+      m = args.n_kt;
     }
   };
 
@@ -814,8 +821,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_ld();
           warp_arrive(bar(L::kBarSFree));
           const int kv0 = j * kTile + col0;
-          const bool need_mask = (kv0 + kCols > args.N) || (args.causal && j == i);
-          const int lim = args.causal ? min(args.N, q_row + 1) : args.N;
+          // a ragged last key tile, or (causal) keys past the position of the tile's
+          // first row
+          const bool need_mask = (kv0 + kCols > args.Nk) ||
+                                 (args.causal && kv0 + kCols - 1 > i * kTile + args.off);
+          const int lim = args.causal ? min(args.Nk, q_row + args.off + 1) : args.Nk;
           const uint64_t scale2 = f32x2(args.scale_log2, args.scale_log2);
           const uint64_t nl2 = f32x2(nl2row, nl2row);
 #pragma unroll
@@ -867,13 +877,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const size_t off = (static_cast<size_t>(bh) * args.N + q_row) * D;
+      const size_t off = (static_cast<size_t>(bh) * args.Nq + q_row) * D;
 #pragma unroll 1
       for (int c = g * (D / 64); c < (g + 1) * (D / 64); ++c) {
         uint32_t v[32];
         tmem_ld32(tdQ + lane_off + c * 32, v);
         tmem_wait_ld();
-        if (q_row < args.N) store_row32(args.dQ + off + c * 32, v, args.scale);
+        if (q_row < args.Nq) store_row32(args.dQ + off + c * 32, v, args.scale);
       }
       warp_arrive(bar(L::kBarAccFree));
     }
@@ -900,10 +910,12 @@ cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUten
   a.dK = static_cast<__nv_bfloat16*>(dK);
   a.dV = static_cast<__nv_bfloat16*>(dV);
   a.BH = p.BH;
-  a.N = p.N;
-  a.n_tiles = (p.N + kTile - 1) / kTile;
-  a.Npad = a.n_tiles * kTile;
-  a.total_units = p.BH * a.n_tiles;
+  a.Nq = p.N;
+  a.Nk = p.Nk;
+  a.off = p.Nk - p.N;
+  a.n_qt = (p.N + kTile - 1) / kTile;
+  a.n_kt = (p.Nk + kTile - 1) / kTile;
+  a.Npad = a.n_qt * kTile;
   a.causal = p.causal;
   a.scale = p.scale;
   a.scale_log2 = p.scale * kLog2e;
@@ -923,7 +935,11 @@ cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUten
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if ((e = trace_mark(p, 1, stream)) != cudaSuccess) return e;
 
-  const int grid = a.total_units < num_sms ? a.total_units : num_sms;
+  BwdArgs a_kv = a, a_q = a;
+  a_kv.total_units = p.BH * a.n_kt;
+  a_q.total_units = p.BH * a.n_qt;
+  const int grid_kv = a_kv.total_units < num_sms ? a_kv.total_units : num_sms;
+  const int grid_q = a_q.total_units < num_sms ? a_q.total_units : num_sms;
   // the in-kernel register split assumes exactly kRegsLaunch registers a thread at launch
   cudaFuncAttributes fattr;
   e = cudaFuncGetAttributes(&fattr, bwd_dkdv_kernel<D>);
@@ -935,14 +951,14 @@ cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUten
   e = cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            DkdvLayout<D>::kAlloc);
   if (e != cudaSuccess) return e;
-  bwd_dkdv_kernel<D><<<grid, kThreads, DkdvLayout<D>::kAlloc, stream>>>(tmQ, tmK, tmV, tmdO,
-                                                                         tmL2, tmD, a);
+  bwd_dkdv_kernel<D><<<grid_kv, kThreads, DkdvLayout<D>::kAlloc, stream>>>(tmQ, tmK, tmV, tmdO,
+                                                                            tmL2, tmD, a_kv);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if ((e = trace_mark(p, 2, stream)) != cudaSuccess) return e;
   e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            DqLayout<D>::kAlloc);
   if (e != cudaSuccess) return e;
-  bwd_dq_kernel<D><<<grid, kThreads, DqLayout<D>::kAlloc, stream>>>(tmQ, tmK, tmV, tmdO, a);
+  bwd_dq_kernel<D><<<grid_q, kThreads, DqLayout<D>::kAlloc, stream>>>(tmQ, tmK, tmV, tmdO, a_q);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   return trace_mark(p, 3, stream);
 }

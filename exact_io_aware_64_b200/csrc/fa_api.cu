@@ -141,10 +141,14 @@ bool overlaps(const void* a, size_t a_bytes, const void* b, size_t b_bytes) {
 
 bool overlaps(const void* a, const void* b, size_t bytes) { return overlaps(a, bytes, b, bytes); }
 
-// Checks shared by every call.  Sets *noop when there is nothing to compute.
-fa_status check_common(int B, int H, int N, int d, float scale, int causal, bool* noop) {
-  if (B < 0 || H < 0 || N < 0)
-    return fail(FA_ERR_INVALID_ARG, "sizes must be non-negative (B=%d H=%d N=%d)", B, H, N);
+// Checks shared by every call: Nq query rows and Nk key rows per head (Nk == Nq for
+// the entry points without the _qk suffix).  Sets *noop when there is nothing to
+// compute.
+fa_status check_common(int B, int H, int Nq, int Nk, int d, float scale, int causal,
+                       bool* noop) {
+  if (B < 0 || H < 0 || Nq < 0 || Nk < 0)
+    return fail(FA_ERR_INVALID_ARG, "sizes must be non-negative (B=%d H=%d Nq=%d Nk=%d)", B,
+                H, Nq, Nk);
   if (d != 64 && d != 128)
     return fail(FA_ERR_UNSUPPORTED, "head dimension d=%d is not supported (64 or 128)", d);
   if (!(std::isfinite(scale) && scale > 0.f))
@@ -152,9 +156,16 @@ fa_status check_common(int B, int H, int N, int d, float scale, int causal, bool
   if (causal != 0 && causal != 1) return fail(FA_ERR_INVALID_ARG, "causal must be 0 or 1");
   const long long bh = static_cast<long long>(B) * H;
   // work units and row indices are 32-bit on the device
-  if (bh > 0 && N > 0 && (bh > (1ll << 31) / ((N + 255) / 256) || bh * N >= (1ll << 31)))
-    return fail(FA_ERR_INVALID_ARG, "B*H*N = %lld rows is too large", bh * N);
-  *noop = (bh == 0 || N == 0);
+  for (const int n : {Nq, Nk})
+    if (bh > 0 && n > 0 && (bh > (1ll << 31) / ((n + 255) / 256) || bh * n >= (1ll << 31)))
+      return fail(FA_ERR_INVALID_ARG, "B*H*N = %lld rows is too large", bh * n);
+  *noop = (bh == 0 || Nq == 0);
+  if (*noop) return FA_OK;
+  if (Nk == 0) return fail(FA_ERR_INVALID_ARG, "queries need at least one key (Nk=0)");
+  if (causal && Nq > Nk)
+    return fail(FA_ERR_INVALID_ARG,
+                "causal attention needs Nq <= Nk: the queries are the last Nq of the Nk "
+                "tokens (Nq=%d Nk=%d)", Nq, Nk);
   return FA_OK;
 }
 
@@ -170,13 +181,33 @@ fa_status check_ptr(const void* p, const char* name) {
     if (_s != FA_OK) return _s;        \
   } while (0)
 
-// Argument checks of fa_bwd and fa_bwd_f32 (elem = bytes per element of the tensors).
+// Argument checks of the forward calls (elem = bytes per element of the tensors).
+fa_status check_fwd_args(const void* Q, const void* K, const void* V, const void* O,
+                         const float* LSE, int B, int H, int Nq, int Nk, int d, float scale,
+                         int causal, size_t elem, bool* noop) {
+  FA_TRY(check_common(B, H, Nq, Nk, d, scale, causal, noop));
+  if (*noop) return FA_OK;
+  FA_TRY(check_ptr(Q, "Q"));
+  FA_TRY(check_ptr(K, "K"));
+  FA_TRY(check_ptr(V, "V"));
+  FA_TRY(check_ptr(O, "O"));
+  if (LSE != nullptr && (reinterpret_cast<uintptr_t>(LSE) & 3u))
+    return fail(FA_ERR_INVALID_ARG, "LSE is not 4-byte aligned");
+  const size_t qb = static_cast<size_t>(B) * H * Nq * d * elem;
+  const size_t kb = static_cast<size_t>(B) * H * Nk * d * elem;
+  if (overlaps(O, qb, Q, qb) || overlaps(O, qb, K, kb) || overlaps(O, qb, V, kb))
+    return fail(FA_ERR_INVALID_ARG, "O overlaps an input");
+  return FA_OK;
+}
+
+// Argument checks of the backward calls (elem = bytes per element of the tensors).
+// Q, O, dO, dQ have Nq rows per head; K, V, dK, dV have Nk.
 fa_status check_bwd_args(const void* Q, const void* K, const void* V, const void* O,
                          const void* dO, const float* LSE, const void* dQ, const void* dK,
-                         const void* dV, int B, int H, int N, int d, float scale, int causal,
-                         const void* workspace, size_t workspace_bytes, size_t elem,
-                         bool* noop) {
-  FA_TRY(check_common(B, H, N, d, scale, causal, noop));
+                         const void* dV, int B, int H, int Nq, int Nk, int d, float scale,
+                         int causal, const void* workspace, size_t workspace_bytes,
+                         size_t elem, bool* noop) {
+  FA_TRY(check_common(B, H, Nq, Nk, d, scale, causal, noop));
   if (*noop) return FA_OK;
   FA_TRY(check_ptr(Q, "Q"));
   FA_TRY(check_ptr(K, "K"));
@@ -187,24 +218,81 @@ fa_status check_bwd_args(const void* Q, const void* K, const void* V, const void
   FA_TRY(check_ptr(dQ, "dQ"));
   FA_TRY(check_ptr(dK, "dK"));
   FA_TRY(check_ptr(dV, "dV"));
-  const size_t need = fa_bwd_workspace_bytes(B, H, N, d);
+  const size_t need = fa_bwd_workspace_bytes(B, H, Nq, d);
   if (need > 0) {
     FA_TRY(check_ptr(workspace, "workspace"));
     if (workspace_bytes < need)
       return fail(FA_ERR_INVALID_ARG, "workspace has %zu bytes, %zu needed", workspace_bytes,
                   need);
   }
-  const size_t bytes = static_cast<size_t>(B) * H * N * d * elem;
-  const void* ins[5] = {Q, K, V, O, dO};
-  const void* outs[3] = {dQ, dK, dV};
-  for (const void* o : outs) {
-    for (const void* in : ins)
-      if (overlaps(o, in, bytes)) return fail(FA_ERR_INVALID_ARG, "a gradient overlaps an input");
-    if (need > 0 && overlaps(o, bytes, workspace, need))
+  const size_t qb = static_cast<size_t>(B) * H * Nq * d * elem;
+  const size_t kb = static_cast<size_t>(B) * H * Nk * d * elem;
+  struct Buf {
+    const void* p;
+    size_t n;
+  };
+  const Buf ins[5] = {{Q, qb}, {K, kb}, {V, kb}, {O, qb}, {dO, qb}};
+  const Buf outs[3] = {{dQ, qb}, {dK, kb}, {dV, kb}};
+  for (const Buf& o : outs) {
+    for (const Buf& in : ins)
+      if (overlaps(o.p, o.n, in.p, in.n))
+        return fail(FA_ERR_INVALID_ARG, "a gradient overlaps an input");
+    if (need > 0 && overlaps(o.p, o.n, workspace, need))
       return fail(FA_ERR_INVALID_ARG, "a gradient overlaps the workspace");
   }
-  if (overlaps(dQ, dK, bytes) || overlaps(dQ, dV, bytes) || overlaps(dK, dV, bytes))
+  if (overlaps(dQ, qb, dK, kb) || overlaps(dQ, qb, dV, kb) || overlaps(dK, kb, dV, kb))
     return fail(FA_ERR_INVALID_ARG, "gradients overlap each other");
+  return FA_OK;
+}
+
+fa_status fwd_impl(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                   int H, int Nq, int Nk, int d, float scale, int causal, cudaStream_t stream) {
+  g_last_error[0] = '\0';
+  bool noop = false;
+  FA_TRY(check_fwd_args(Q, K, V, O, LSE, B, H, Nq, Nk, d, scale, causal, 2, &noop));
+  if (noop) return FA_OK;  // empty problem: the pointers are never used (may be NULL)
+  DeviceInfo dev;
+  FA_TRY(device_info(&dev));
+  FA_TRY(require_sm100(dev));
+  const int BH = B * H;
+  CUtensorMap tmQ, tmK, tmV;
+  FA_TRY(make_tmap(&tmQ, Q, BH, Nq, d));
+  FA_TRY(make_tmap(&tmK, K, BH, Nk, d));
+  FA_TRY(make_tmap(&tmV, V, BH, Nk, d));
+  fa::Problem p{BH, Nq, Nk, d, scale, causal, dev.err, g_n_trace ? g_trace : nullptr,
+                g_n_trace};
+  cudaError_t e = fa::launch_fwd_sm100(tmQ, tmK, tmV, O, LSE, p, dev.num_sms, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "launching the forward kernel");
+  return FA_OK;
+}
+
+fa_status bwd_impl(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                   const float* LSE, void* dQ, void* dK, void* dV, int B, int H, int Nq, int Nk,
+                   int d, float scale, int causal, void* workspace, size_t workspace_bytes,
+                   cudaStream_t stream) {
+  g_last_error[0] = '\0';
+  bool noop = false;
+  FA_TRY(check_bwd_args(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, Nq, Nk, d, scale, causal,
+                        workspace, workspace_bytes, 2, &noop));
+  if (noop) return FA_OK;  // empty problem: the pointers are never used (may be NULL)
+  DeviceInfo dev;
+  FA_TRY(device_info(&dev));
+  FA_TRY(require_sm100(dev));
+  const int BH = B * H;
+  CUtensorMap tmQ, tmK, tmV, tmdO, tmL2, tmD;
+  FA_TRY(make_tmap(&tmQ, Q, BH, Nq, d));
+  FA_TRY(make_tmap(&tmK, K, BH, Nk, d));
+  FA_TRY(make_tmap(&tmV, V, BH, Nk, d));
+  FA_TRY(make_tmap(&tmdO, dO, BH, Nq, d));
+  const int Npad = fa::bwd_padded_rows(Nq);
+  float* ws = static_cast<float*>(workspace);
+  FA_TRY(make_row_tmap(&tmD, ws, BH, Npad));
+  FA_TRY(make_row_tmap(&tmL2, ws + static_cast<size_t>(BH) * Npad, BH, Npad));
+  fa::Problem p{BH, Nq, Nk, d, scale, causal, dev.err, g_n_trace ? g_trace : nullptr,
+                g_n_trace};
+  cudaError_t e = fa::launch_bwd_sm100(tmQ, tmK, tmV, tmdO, tmL2, tmD, O, dO, LSE, dQ, dK, dV,
+                                       ws, p, dev.num_sms, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "launching the backward kernels");
   return FA_OK;
 }
 
@@ -239,31 +327,13 @@ fa_status fa_trace_events(cudaEvent_t* events, int n) {
 
 fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H,
                  int N, int d, float scale, int causal, cudaStream_t stream) {
-  g_last_error[0] = '\0';
-  bool noop = false;
-  FA_TRY(check_common(B, H, N, d, scale, causal, &noop));
-  if (noop) return FA_OK;  // empty problem: the pointers are never used (may be NULL)
-  FA_TRY(check_ptr(Q, "Q"));
-  FA_TRY(check_ptr(K, "K"));
-  FA_TRY(check_ptr(V, "V"));
-  FA_TRY(check_ptr(O, "O"));
-  if (LSE != nullptr && (reinterpret_cast<uintptr_t>(LSE) & 3u))
-    return fail(FA_ERR_INVALID_ARG, "LSE is not 4-byte aligned");
-  const size_t bytes = static_cast<size_t>(B) * H * N * d * 2;
-  if (overlaps(O, Q, bytes) || overlaps(O, K, bytes) || overlaps(O, V, bytes))
-    return fail(FA_ERR_INVALID_ARG, "O overlaps an input");
-  DeviceInfo dev;
-  FA_TRY(device_info(&dev));
-  FA_TRY(require_sm100(dev));
-  const int BH = B * H;
-  CUtensorMap tmQ, tmK, tmV;
-  FA_TRY(make_tmap(&tmQ, Q, BH, N, d));
-  FA_TRY(make_tmap(&tmK, K, BH, N, d));
-  FA_TRY(make_tmap(&tmV, V, BH, N, d));
-  fa::Problem p{BH, N, d, scale, causal, dev.err, g_n_trace ? g_trace : nullptr, g_n_trace};
-  cudaError_t e = fa::launch_fwd_sm100(tmQ, tmK, tmV, O, LSE, p, dev.num_sms, stream);
-  if (e != cudaSuccess) return cuda_fail(e, "launching the forward kernel");
-  return FA_OK;
+  return fwd_impl(Q, K, V, O, LSE, B, H, N, N, d, scale, causal, stream);
+}
+
+fa_status fa_fwd_qk(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                    int H, int Nq, int Nk, int d, float scale, int causal,
+                    cudaStream_t stream) {
+  return fwd_impl(Q, K, V, O, LSE, B, H, Nq, Nk, d, scale, causal, stream);
 }
 
 fa_status fa_fwd_f32(const float* Q, const float* K, const float* V, float* O, float* LSE,
@@ -271,20 +341,11 @@ fa_status fa_fwd_f32(const float* Q, const float* K, const float* V, float* O, f
                      cudaStream_t stream) {
   g_last_error[0] = '\0';
   bool noop = false;
-  FA_TRY(check_common(B, H, N, d, scale, causal, &noop));
+  FA_TRY(check_fwd_args(Q, K, V, O, LSE, B, H, N, N, d, scale, causal, 4, &noop));
   if (noop) return FA_OK;  // empty problem: the pointers are never used (may be NULL)
-  FA_TRY(check_ptr(Q, "Q"));
-  FA_TRY(check_ptr(K, "K"));
-  FA_TRY(check_ptr(V, "V"));
-  FA_TRY(check_ptr(O, "O"));
-  if (LSE != nullptr && (reinterpret_cast<uintptr_t>(LSE) & 3u))
-    return fail(FA_ERR_INVALID_ARG, "LSE is not 4-byte aligned");
-  const size_t bytes = static_cast<size_t>(B) * H * N * d * 4;
-  if (overlaps(O, Q, bytes) || overlaps(O, K, bytes) || overlaps(O, V, bytes))
-    return fail(FA_ERR_INVALID_ARG, "O overlaps an input");
   DeviceInfo dev;
   FA_TRY(device_info(&dev));
-  fa::Problem p{B * H, N, d, scale, causal, dev.err, g_n_trace ? g_trace : nullptr,
+  fa::Problem p{B * H, N, N, d, scale, causal, dev.err, g_n_trace ? g_trace : nullptr,
                 g_n_trace};
   cudaError_t e = fa::launch_fwd_f32(Q, K, V, O, LSE, p, stream);
   if (e != cudaSuccess) return cuda_fail(e, "launching the float32 forward kernel");
@@ -294,7 +355,7 @@ fa_status fa_fwd_f32(const float* Q, const float* K, const float* V, float* O, f
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
   (void)d;
   if (B <= 0 || H <= 0 || N <= 0) return 0;
-  // D and LSE*log2(e), one float each per row, rows padded to whole 128-row tiles
+  // D and LSE*log2(e), one float each per query row, rows padded to whole 128-row tiles
   const size_t raw = 2 * static_cast<size_t>(B) * H * fa::bwd_padded_rows(N) * sizeof(float);
   return (raw + 255) / 256 * 256;
 }
@@ -303,29 +364,16 @@ fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, con
                  const float* LSE, void* dQ, void* dK, void* dV, int B, int H, int N, int d,
                  float scale, int causal, void* workspace, size_t workspace_bytes,
                  cudaStream_t stream) {
-  g_last_error[0] = '\0';
-  bool noop = false;
-  FA_TRY(check_bwd_args(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, scale, causal, workspace,
-                        workspace_bytes, 2, &noop));
-  if (noop) return FA_OK;  // empty problem: the pointers are never used (may be NULL)
-  DeviceInfo dev;
-  FA_TRY(device_info(&dev));
-  FA_TRY(require_sm100(dev));
-  const int BH = B * H;
-  CUtensorMap tmQ, tmK, tmV, tmdO, tmL2, tmD;
-  FA_TRY(make_tmap(&tmQ, Q, BH, N, d));
-  FA_TRY(make_tmap(&tmK, K, BH, N, d));
-  FA_TRY(make_tmap(&tmV, V, BH, N, d));
-  FA_TRY(make_tmap(&tmdO, dO, BH, N, d));
-  const int Npad = fa::bwd_padded_rows(N);
-  float* ws = static_cast<float*>(workspace);
-  FA_TRY(make_row_tmap(&tmD, ws, BH, Npad));
-  FA_TRY(make_row_tmap(&tmL2, ws + static_cast<size_t>(BH) * Npad, BH, Npad));
-  fa::Problem p{BH, N, d, scale, causal, dev.err, g_n_trace ? g_trace : nullptr, g_n_trace};
-  cudaError_t e = fa::launch_bwd_sm100(tmQ, tmK, tmV, tmdO, tmL2, tmD, O, dO, LSE, dQ, dK, dV,
-                                       ws, p, dev.num_sms, stream);
-  if (e != cudaSuccess) return cuda_fail(e, "launching the backward kernels");
-  return FA_OK;
+  return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, N, d, scale, causal, workspace,
+                  workspace_bytes, stream);
+}
+
+fa_status fa_bwd_qk(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                    const float* LSE, void* dQ, void* dK, void* dV, int B, int H, int Nq,
+                    int Nk, int d, float scale, int causal, void* workspace,
+                    size_t workspace_bytes, cudaStream_t stream) {
+  return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, Nq, Nk, d, scale, causal, workspace,
+                  workspace_bytes, stream);
 }
 
 fa_status fa_bwd_f32(const float* Q, const float* K, const float* V, const float* O,
@@ -334,12 +382,12 @@ fa_status fa_bwd_f32(const float* Q, const float* K, const float* V, const float
                      size_t workspace_bytes, cudaStream_t stream) {
   g_last_error[0] = '\0';
   bool noop = false;
-  FA_TRY(check_bwd_args(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, scale, causal, workspace,
-                        workspace_bytes, 4, &noop));
+  FA_TRY(check_bwd_args(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, N, d, scale, causal,
+                        workspace, workspace_bytes, 4, &noop));
   if (noop) return FA_OK;  // empty problem: the pointers are never used (may be NULL)
   DeviceInfo dev;
   FA_TRY(device_info(&dev));
-  fa::Problem p{B * H, N, d, scale, causal, dev.err, g_n_trace ? g_trace : nullptr,
+  fa::Problem p{B * H, N, N, d, scale, causal, dev.err, g_n_trace ? g_trace : nullptr,
                 g_n_trace};
   cudaError_t e = fa::launch_bwd_f32(Q, K, V, O, dO, LSE, dQ, dK, dV,
                                      static_cast<float*>(workspace), p, stream);
@@ -437,7 +485,7 @@ fa_status fa_bwd_noalloc(const void* Q, const void* K, const void* V, const void
   }
   void* scratch = nullptr;
   bool noop = false;
-  fa_status st = check_common(B, H, N, d, scale, causal, &noop);
+  fa_status st = check_common(B, H, N, N, d, scale, causal, &noop);
   if (st != FA_OK || noop) return st;
   st = noalloc_scratch(&scratch);
   if (st != FA_OK) return st;

@@ -31,9 +31,13 @@
 //     the same reference, and keeps every exponential below 2^8.
 //   * K/V tiles stream through a ring of shared-memory slots guarded by mbarriers
 //     (full: TMA transaction bytes; empty: tcgen05.commit from the MMA thread).
-//   * Causal: query tile q needs key tiles 0..q; only the diagonal tile and a ragged
-//     last key tile need element masks.  Rows past N (ragged last query tile) are
-//     computed on zero-filled Q and never stored.
+//   * Queries and keys may differ in number (Nq <= Nk when causal): the queries are then
+//     the last Nq tokens of the sequence, query row r at position r + Nk - Nq, and a
+//     causal row sees keys up to its position (bottom-right alignment; Nq == Nk gives
+//     the usual j <= i).  A query tile needs the key tiles up to the one holding its
+//     last row's position; only tiles that cross a row's limit, and a ragged last key
+//     tile, need element masks.  Rows past Nq (ragged last query tile) are computed on
+//     zero-filled Q and never stored.
 #include <cfloat>
 #include <cstdint>
 
@@ -94,9 +98,11 @@ struct FwdArgs {
   __nv_bfloat16* O;
   float* LSE;
   int BH;
-  int N;
+  int Nq;           // query rows per head
+  int Nk;           // key rows per head
+  int off;          // causal: Nk - Nq, the position of query row 0
   int causal;
-  int n_units;      // units per (batch, head) = ceil(N / 256)
+  int n_units;      // units per (batch, head) = ceil(Nq / 256)
   int total_units;  // BH * n_units
   float scale_log2;  // scale * log2(e)
 };
@@ -115,11 +121,13 @@ __device__ __forceinline__ UnitInfo unit_info(int w, const FwdArgs& a) {
     r.bh = w / a.n_units;
     r.u = w % a.n_units;
   }
-  const int n_kv = (a.N + kBN - 1) / kBN;
+  const int n_kv = (a.Nk + kBN - 1) / kBN;
   const int qt0 = 2 * r.u, qt1 = 2 * r.u + 1;
-  const bool valid1 = qt1 * kBM < a.N;
-  r.n0 = a.causal ? min(qt0 + 1, n_kv) : n_kv;
-  r.n1 = valid1 ? (a.causal ? min(qt1 + 1, n_kv) : n_kv) : 0;
+  const bool valid1 = qt1 * kBM < a.Nq;
+  // causal: key tiles up to the one holding the position of the tile's last row
+  auto n_causal = [&](int qt) { return min((qt * kBM + kBM - 1 + a.off) / kBN + 1, n_kv); };
+  r.n0 = a.causal ? n_causal(qt0) : n_kv;
+  r.n1 = valid1 ? (a.causal ? n_causal(qt1) : n_kv) : 0;
   return r;
 }
 
@@ -362,9 +370,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < kBN; ++c) s[c] = __uint_as_float(sr[c]);
         const int kv0 = j * kBN;
-        const bool need_mask = (kv0 + kBN > args.N) || (args.causal && j == qt);
+        // a ragged last key tile, or (causal) a tile whose last key lies past the
+        // position of the tile's first row
+        const bool need_mask = (kv0 + kBN > args.Nk) ||
+                               (args.causal && kv0 + kBN - 1 > qt * kBM + args.off);
         if (need_mask) {
-          const int lim = args.causal ? min(args.N, q_row + 1) : args.N;
+          const int lim = args.causal ? min(args.Nk, q_row + args.off + 1) : args.Nk;
 #pragma unroll
           for (int c = 0; c < kBN; ++c)
             if (kv0 + c >= lim) s[c] = -INFINITY;
@@ -443,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const float inv_l = 1.f / l;
       const int bh = ui.bh;
-      __nv_bfloat16* orow = args.O + (static_cast<size_t>(bh) * args.N + q_row) * D;
+      __nv_bfloat16* orow = args.O + (static_cast<size_t>(bh) * args.Nq + q_row) * D;
       // take the whole O row into registers first, so the MMA warp may start the next
       // unit's first P V product while this row is being converted and stored
       uint32_t ov[D];
@@ -451,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < D / 32; ++c) tmem_ld32(tOrow + c * 32, &ov[c * 32]);
       tmem_wait_ld();
       warp_arrive(bar(L::kBarOFree + t));
-      if (q_row < args.N) {
+      if (q_row < args.Nq) {
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t pk[16];
@@ -465,8 +476,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
         }
       }
-      if (args.LSE != nullptr && q_row < args.N)
-        args.LSE[static_cast<size_t>(bh) * args.N + q_row] =
+      if (args.LSE != nullptr && q_row < args.Nq)
+        args.LSE[static_cast<size_t>(bh) * args.Nq + q_row] =
             (m + __log2f(l)) * 0.69314718055994531f;
     }
   }
@@ -489,7 +500,9 @@ cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUten
   a.O = static_cast<__nv_bfloat16*>(O);
   a.LSE = LSE;
   a.BH = p.BH;
-  a.N = p.N;
+  a.Nq = p.N;
+  a.Nk = p.Nk;
+  a.off = p.Nk - p.N;
   a.causal = p.causal;
   a.n_units = (p.N + 2 * kBM - 1) / (2 * kBM);
   a.total_units = p.BH * a.n_units;

@@ -8,10 +8,13 @@
 
 namespace fa {
 
-// Problem shared by every kernel: [B*H, N, d] tensors, contiguous.
+// Problem shared by every kernel: [B*H, N, d] query-side tensors (Q, O, dO, dQ, LSE)
+// and [B*H, Nk, d] key-side tensors (K, V, dK, dV), contiguous.  Nk == N except for
+// the Nq != Nk entry points, whose queries are the last N of the Nk tokens.
 struct Problem {
   int BH;
   int N;
+  int Nk;
   int d;
   float scale;
   int causal;

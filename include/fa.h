@@ -86,6 +86,23 @@ FA_API fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, fl
                  int B, int H, int N, int d, float scale, int causal, cudaStream_t stream);
 
 /*
+ * Forward pass with Nq queries and Nk keys per head (no counterpart on the pages, which
+ * treat attention over N tokens; the reading used here: the queries are the last Nq of
+ * the Nk tokens, e.g. a chunk of new tokens whose keys follow earlier ones).
+ *   Q        in : [B,H,Nq,d] bf16
+ *   K, V     in : [B,H,Nk,d] bf16
+ *   O        out: [B,H,Nq,d] bf16; must not overlap Q, K or V
+ *   LSE      out: [B,H,Nq] float32; may be NULL
+ *   causal: query i sees keys j <= i + Nk - Nq (bottom-right alignment) and then needs
+ *   Nq <= Nk (FA_ERR_INVALID_ARG otherwise); non-causal takes any Nq, Nk >= 1.
+ *   fa_fwd(..., N, ...) is fa_fwd_qk(..., N, N, ...).  Same kernel, errors and
+ *   asynchrony as fa_fwd.
+ */
+FA_API fa_status fa_fwd_qk(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                           int B, int H, int Nq, int Nk, int d, float scale, int causal,
+                           cudaStream_t stream);
+
+/*
  * Forward pass with float32 inputs and outputs, computed in float32 on the CUDA cores
  * (same definition and arguments as fa_fwd).
  */
@@ -116,6 +133,19 @@ FA_API fa_status fa_bwd(const void* Q, const void* K, const void* V, const void*
                  const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
                  int B, int H, int N, int d, float scale, int causal,
                  void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Backward pass with Nq queries and Nk keys per head, the gradient of fa_fwd_qk.
+ *   Q, O, dO in : [B,H,Nq,d] bf16;   K, V in : [B,H,Nk,d] bf16
+ *   LSE      in : [B,H,Nq] float32 from fa_fwd_qk with the same scale and causal
+ *   dQ       out: [B,H,Nq,d] bf16;   dK, dV out: [B,H,Nk,d] bf16
+ *   workspace   : fa_bwd_workspace_bytes(B,H,Nq,d) bytes (two floats per query row)
+ * Same kernels, rules and errors as fa_bwd (causal needs Nq <= Nk).
+ */
+FA_API fa_status fa_bwd_qk(const void* Q, const void* K, const void* V, const void* O,
+                           const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                           int B, int H, int Nq, int Nk, int d, float scale, int causal,
+                           void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * Backward pass, float32: the same computation as fa_bwd with float32 inputs, outputs
@@ -161,10 +191,9 @@ FA_API size_t fa_bwd_noalloc_max_scratch_bytes(void);
 
 /*
  * Kernel-boundary timing, for profilers.  While a list of events is set on the calling
- * thread, every fa_fwd, fa_fwd_f32, fa_bwd and fa_bwd_f32 call records events[0] on its
- * stream just before its first kernel and events[k] just after its k-th kernel; fa_fwd
- * and fa_fwd_f32 launch one kernel, fa_bwd and fa_bwd_f32 three (D preparation, dK/dV,
- * dQ).  Boundaries
+ * thread, every forward and backward call records events[0] on its stream just before
+ * its first kernel and events[k] just after its k-th kernel; the forward calls launch
+ * one kernel, the backward calls three (D preparation, dK/dV, dQ).  Boundaries
  * beyond n - 1 are not recorded.  The events are caller-created cudaEvent_t (timing
  * enabled) and stay caller-owned.  fa_trace_events(NULL, 0) stops recording.
  * Returns FA_ERR_INVALID_ARG if n < 0, n > 8, or events is NULL with n > 0.

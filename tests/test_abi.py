@@ -147,3 +147,34 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         binding.lib()
+
+
+def test_qk_validation(lib):
+    """fa_fwd_qk / fa_bwd_qk: Nq queries against Nk keys (queries = the last Nq tokens)."""
+    def fwd(Nq, Nk, causal=1, o=D_, **kw):
+        return lib.fa_fwd_qk(A, B_, C, o, E, 1, 2, Nq, Nk, 64, 0.1, causal, None)
+
+    assert fwd(0, 5) == binding.FA_OK                      # no queries: no-op
+    assert fwd(4, 0) == binding.FA_ERR_INVALID_ARG         # queries without keys
+    assert fwd(8, 4, causal=1) == binding.FA_ERR_INVALID_ARG  # causal needs Nq <= Nk
+    assert "Nq <= Nk" in lib.fa_last_error_message().decode()
+    assert fwd(8, 4, causal=0) != binding.FA_ERR_INVALID_ARG  # non-causal: any lengths
+    assert fwd(-1, 4) == binding.FA_ERR_INVALID_ARG
+    # O is sized by Nq, K and V by Nk: O right after a short K does not overlap it
+    assert fwd(16, 64, o=B_ + 2 * 64 * 64 * 2) != binding.FA_ERR_INVALID_ARG
+    assert fwd(16, 64, o=B_ + 2 * 64 * 64 * 2 - 16) == binding.FA_ERR_INVALID_ARG
+
+    F, G, H_, I, J = 0x600000, 0x700000, 0x800000, 0x900000, 0xA00000
+
+    def bwd(Nq, Nk, causal=1, ws_bytes=1 << 20, dk=H_):
+        return lib.fa_bwd_qk(A, B_, C, D_, E, F, G, dk, I, 1, 2, Nq, Nk, 64, 0.1, causal, J,
+                             ws_bytes, None)
+
+    assert bwd(0, 3) == binding.FA_OK
+    assert bwd(5, 3) == binding.FA_ERR_INVALID_ARG
+    assert bwd(3, 0) == binding.FA_ERR_INVALID_ARG
+    # the workspace is sized by the query rows
+    need = binding.workspace_bytes(1, 2, 100, 64)
+    assert bwd(100, 1000, ws_bytes=need - 4) == binding.FA_ERR_INVALID_ARG
+    assert bwd(100, 1000, ws_bytes=need) != binding.FA_ERR_INVALID_ARG
+    assert bwd(100, 1000, dk=G + 2 * 100 * 64 * 2 - 16) == binding.FA_ERR_INVALID_ARG
