@@ -356,6 +356,7 @@ def run_gpu(args, w):
 
 # ------------------------------------------------------------------ N sweep
 SWEEP_N = (256, 512, 1024, 2048, 4096, 8192, 16384, 32768)
+SWEEP_CHUNK_NQ = (256, 1024, 2048, 4096)
 
 
 def run_sweep(args):
@@ -370,6 +371,7 @@ def run_sweep(args):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     peaks, peak_src = load_peaks()
     peak = peaks["bf16_tflops"]
+    hbm = peaks["hbm_gbs"]
     for d in (64, 128):
         for causal in (False, True):
             for N in SWEEP_N:
@@ -385,8 +387,11 @@ def run_sweep(args):
                 bwd = lambda: binding.bwd(q, k, v, O, do, LSE, causal=causal, dQ=dQ,  # noqa: E731
                                           dK=dK, dV=dV, workspace=ws)
                 res = {}
-                for name, fn, flops in (("fwd", fwd, traffic.fwd_flops(B, H, N, d, causal)),
-                                        ("bwd", bwd, traffic.bwd_flops(B, H, N, d, causal))):
+                for name, fn, flops, nbytes in (
+                        ("fwd", fwd, traffic.fwd_flops(B, H, N, d, causal),
+                         traffic.fwd_compulsory_bytes(B, H, N, d)),
+                        ("bwd", bwd, traffic.bwd_flops(B, H, N, d, causal),
+                         traffic.bwd_compulsory_bytes(B, H, N, d))):
                     for _ in range(args.warmup):
                         fn()
                     times = []
@@ -401,14 +406,58 @@ def run_sweep(args):
                         times.append(e0.elapsed_time(e1))
                     ms = statistics.median(times)
                     pct = statistics.quantiles(times, n=10) if len(times) > 1 else [ms] * 9
+                    # roofline: the slower of the tensor-core time and the time to move
+                    # the compulsory bytes once at the measured HBM bandwidth
+                    t_tensor = flops / (peak * 1e12) * 1e3
+                    t_hbm = nbytes / (hbm * 1e9) * 1e3
                     res[name] = {"ms": ms, "ms_p10": pct[0], "ms_p90": pct[-1],
                                  "tflops": flops / (ms * 1e-3) / 1e12,
-                                 "frac": flops / (ms * 1e-3) / 1e12 / peak}
+                                 "frac": flops / (ms * 1e-3) / 1e12 / peak,
+                                 "gbs": nbytes / (ms * 1e-3) / 1e9,
+                                 "bound": "tensor" if t_tensor >= t_hbm else "hbm",
+                                 "roofline_frac": max(t_tensor, t_hbm) / ms}
                 binding.check_device_error()
                 print(json.dumps({"sweep": "attention TFLOP/s vs N", "N": N, "B": B, "H": H, "d": d,
                                   "causal": causal, "dtype": "bf16", "peak": peak,
-                                  "peak_source": f"{peak_src} burst bf16", **res}), flush=True)
+                                  "hbm_gbs": hbm, "peak_source": f"{peak_src} burst bf16, "
+                                  f"{peak_src} HBM copy", **res}), flush=True)
                 del ins, q, k, v, do, O, LSE, dQ, dK, dV, ws
+    # chunks of queries at the end of a long key sequence (fa_fwd_qk / fa_bwd_qk):
+    # B=1, H=16, Nk=8192, d=128, causal
+    for Nq in SWEEP_CHUNK_NQ:
+        B, H, Nk, d = 1, 16, 8192, 128
+        qi = fa_inputs.make_inputs(B, H, Nq, d, seed=Nq, with_dO=True, device="cuda")
+        ki = fa_inputs.make_inputs(B, H, Nk, d, seed=Nq + 1, device="cuda")
+        q, do, k, v = qi["Q"], qi["dO"], ki["K"], ki["V"]
+        O = torch.empty_like(q)
+        LSE = torch.empty((B, H, Nq), device=dev, dtype=torch.float32)
+        dQ, dK, dV = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(max(binding.workspace_bytes(B, H, Nq, d), 1), device=dev,
+                         dtype=torch.uint8)
+        fwd = lambda: binding.fwd(q, k, v, causal=True, O=O, LSE=LSE)  # noqa: E731
+        bwd = lambda: binding.bwd(q, k, v, O, do, LSE, causal=True, dQ=dQ, dK=dK,  # noqa: E731
+                                  dV=dV, workspace=ws)
+        res = {}
+        for name, fn, flops in (("fwd", fwd, traffic.fwd_flops_qk(B, H, Nq, Nk, d, True)),
+                                ("bwd", bwd, traffic.bwd_flops_qk(B, H, Nq, Nk, d, True))):
+            for _ in range(args.warmup):
+                fn()
+            times = []
+            for _ in range(args.steps):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                fn()
+                e1.record()
+                torch.cuda.synchronize()
+                times.append(e0.elapsed_time(e1))
+            ms = statistics.median(times)
+            res[name] = {"ms": ms, "tflops": flops / (ms * 1e-3) / 1e12,
+                         "frac": flops / (ms * 1e-3) / 1e12 / peak}
+        binding.check_device_error()
+        print(json.dumps({"sweep": "prefill chunk TFLOP/s", "Nq": Nq, "Nk": Nk, "B": B, "H": H,
+                          "d": d, "causal": True, "dtype": "bf16", "peak": peak, **res}),
+              flush=True)
+        del qi, ki, q, do, k, v, O, LSE, dQ, dK, dV, ws
     return 0
 
 

@@ -41,6 +41,23 @@ def bwd_flops(B: int, H: int, N: int, d: int, causal: bool) -> float:
     return f / 2 if causal else f
 
 
+def visible_pairs(Nq: int, Nk: int, causal: bool) -> float:
+    """(query, key) pairs the product covers per head: Nq * Nk, or, causal with the
+    queries as the last Nq of the Nk tokens, Nq * Nk - Nq^2 / 2 (the same halving
+    convention as the square case, where it gives N^2 / 2)."""
+    return Nq * Nk - Nq * Nq / 2.0 if causal else float(Nq) * Nk
+
+
+def fwd_flops_qk(B: int, H: int, Nq: int, Nk: int, d: int, causal: bool) -> float:
+    """Credited forward FLOPs with Nq queries and Nk keys: 4 B H d per visible pair."""
+    return 4.0 * B * H * d * visible_pairs(Nq, Nk, causal)
+
+
+def bwd_flops_qk(B: int, H: int, Nq: int, Nk: int, d: int, causal: bool) -> float:
+    """Credited backward FLOPs with Nq queries and Nk keys: 10 B H d per visible pair."""
+    return 10.0 * B * H * d * visible_pairs(Nq, Nk, causal)
+
+
 def fwd_compulsory_bytes(B: int, H: int, N: int, d: int, elem_bytes: int = 2,
                          lse: bool = True) -> int:
     """Bytes the forward must move at least once: read Q, K, V, write O (and the fp32

@@ -27,6 +27,19 @@ def test_flop_convention():
     assert traffic.bwd_flops(2, 16, 8192, 128, True) == 5 * 2 * 16 * 8192 ** 2 * 128
 
 
+def test_flops_with_fewer_queries_than_keys():
+    # equal lengths reduce to the square convention
+    for causal in (False, True):
+        assert traffic.fwd_flops_qk(2, 3, 256, 256, 64, causal) == \
+            traffic.fwd_flops(2, 3, 256, 64, causal)
+        assert traffic.bwd_flops_qk(2, 3, 256, 256, 64, causal) == \
+            traffic.bwd_flops(2, 3, 256, 64, causal)
+    # a chunk of 1024 queries at the end of 8192 keys: the rectangle before the chunk
+    # plus half the square of the chunk
+    assert traffic.visible_pairs(1024, 8192, True) == 1024 * 7168 + 1024 * 1024 / 2
+    assert traffic.visible_pairs(1024, 8192, False) == 1024 * 8192
+
+
 def test_inputs_are_seeded_and_ordered():
     a = inputs.make_inputs(1, 2, 9, 4, seed=7, with_dO=True)
     b = inputs.make_inputs(1, 2, 9, 4, seed=7, with_dO=True)
