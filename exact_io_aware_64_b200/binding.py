@@ -34,12 +34,16 @@ SIGNATURES = {
     "fa_abi_version": ([], _i),
     "fa_fwd": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp], _i),
     "fa_fwd_qk": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _vp], _i),
+    "fa_fwd_varlen": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _vp],
+                      _i),
     "fa_fwd_f32": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp], _i),
     "fa_bwd_workspace_bytes": ([_i, _i, _i, _i], _sz),
     "fa_bwd": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _sz,
                 _vp], _i),
     "fa_bwd_qk": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _vp,
                    _sz, _vp], _i),
+    "fa_bwd_varlen": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
+                       _i, _f, _i, _vp, _sz, _vp], _i),
     "fa_bwd_f32": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp,
                     _sz, _vp], _i),
     "fa_bwd_noalloc": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i,
@@ -231,6 +235,82 @@ def bwd_noalloc(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, O: torch.Tens
                                   _ptr(dQ), _ptr(dK), _ptr(dV), B, H, N, d, float(scale),
                                   int(bool(causal)), _stream_handle(stream))
     _check("fa_bwd_noalloc", st)
+    return dQ, dK, dV
+
+
+def _check_seqlens(seqlens_q: torch.Tensor, seqlens_k: torch.Tensor, B: int, device) -> None:
+    for name, t in (("seqlens_q", seqlens_q), ("seqlens_k", seqlens_k)):
+        if not t.is_cuda or t.device != device:
+            raise ValueError(f"{name} must be on the inputs' CUDA device")
+        if t.dtype != torch.int32 or tuple(t.shape) != (B,) or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous int32 tensor of shape ({B},)")
+
+
+def fwd_varlen(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, seqlens_q: torch.Tensor,
+               seqlens_k: torch.Tensor, scale: Optional[float] = None, causal: bool = False,
+               O: Optional[torch.Tensor] = None, LSE: Optional[torch.Tensor] = None,
+               stream: Optional[torch.cuda.Stream] = None):
+    """Forward over a padded batch through ``fa_fwd_varlen``: sequence b uses its first
+    seqlens_q[b] query rows of Q [B, H, Nq, d] and seqlens_k[b] key rows of K, V
+    [B, H, Nk, d] (bf16).  Rows of O and LSE past a sequence's length are not written
+    (outputs allocated here start as zeros and -inf).  Returns (O, LSE)."""
+    B, H, Nq, d = Q.shape
+    Nk = K.shape[2]
+    _check_bhnd("Q", Q, (B, H, Nq, d), torch.bfloat16)
+    for name, t in (("K", K), ("V", V)):
+        _check_bhnd(name, t, (B, H, Nk, d), torch.bfloat16)
+    _check_seqlens(seqlens_q, seqlens_k, B, Q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if O is None:
+        O = torch.zeros_like(Q)
+    if LSE is None:
+        LSE = torch.full((B, H, Nq), float("-inf"), device=Q.device, dtype=torch.float32)
+    _check_bhnd("O", O, (B, H, Nq, d), torch.bfloat16)
+    _check_bhnd("LSE", LSE, (B, H, Nq), torch.float32)
+    with torch.cuda.device(Q.device):
+        st = lib().fa_fwd_varlen(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), _ptr(seqlens_q),
+                                 _ptr(seqlens_k), B, H, Nq, Nk, d, float(scale),
+                                 int(bool(causal)), _stream_handle(stream))
+    _check("fa_fwd_varlen", st)
+    return O, LSE
+
+
+def bwd_varlen(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, O: torch.Tensor,
+               dO: torch.Tensor, LSE: torch.Tensor, seqlens_q: torch.Tensor,
+               seqlens_k: torch.Tensor, scale: Optional[float] = None, causal: bool = False,
+               dQ: Optional[torch.Tensor] = None, dK: Optional[torch.Tensor] = None,
+               dV: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+               stream: Optional[torch.cuda.Stream] = None):
+    """Backward over a padded batch through ``fa_bwd_varlen`` (the gradient of
+    ``fwd_varlen`` with the same lengths).  Rows past a sequence's lengths are not
+    written (gradients allocated here start as zeros).  Returns (dQ, dK, dV)."""
+    B, H, Nq, d = Q.shape
+    Nk = K.shape[2]
+    for name, t in (("Q", Q), ("O", O), ("dO", dO)):
+        _check_bhnd(name, t, (B, H, Nq, d), torch.bfloat16)
+    for name, t in (("K", K), ("V", V)):
+        _check_bhnd(name, t, (B, H, Nk, d), torch.bfloat16)
+    _check_bhnd("LSE", LSE, (B, H, Nq), torch.float32)
+    _check_seqlens(seqlens_q, seqlens_k, B, Q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dQ = torch.zeros_like(Q) if dQ is None else dQ
+    dK = torch.zeros_like(K) if dK is None else dK
+    dV = torch.zeros_like(V) if dV is None else dV
+    _check_bhnd("dQ", dQ, (B, H, Nq, d), torch.bfloat16)
+    for name, t in (("dK", dK), ("dV", dV)):
+        _check_bhnd(name, t, (B, H, Nk, d), torch.bfloat16)
+    need = workspace_bytes(B, H, Nq, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), device=Q.device, dtype=torch.uint8)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    with torch.cuda.device(Q.device):
+        st = lib().fa_bwd_varlen(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _ptr(LSE),
+                                 _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(seqlens_q), _ptr(seqlens_k),
+                                 B, H, Nq, Nk, d, float(scale), int(bool(causal)),
+                                 _ptr(workspace), ws_bytes, _stream_handle(stream))
+    _check("fa_bwd_varlen", st)
     return dQ, dK, dV
 
 

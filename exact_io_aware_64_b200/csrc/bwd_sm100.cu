@@ -80,6 +80,51 @@ struct PolyEvery {
 
 __host__ __device__ constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
+struct BwdArgs {
+  unsigned int* err;
+  const int* seqlens_q;  // [B] per-sequence query rows, or null (all Nq)
+  const int* seqlens_k;  // [B] per-sequence key rows, or null (all Nk)
+  int H;
+  __nv_bfloat16* dQ;
+  __nv_bfloat16* dK;
+  __nv_bfloat16* dV;
+  const float* Dpad;   // [BH][Npad]: -D
+  const float* L2pad;  // [BH][Npad]: -LSE * log2(e)
+  int BH;
+  int Nq;           // query rows per head (Q, O, dO, dQ, LSE); padded length with seqlens
+  int Nk;           // key rows per head (K, V, dK, dV); padded length with seqlens
+  int Npad;         // Nq rounded up to whole tiles
+  int n_qt;         // ceil(Nq / 128)
+  int n_kt;         // ceil(Nk / 128)
+  int total_units;  // this kernel's units: BH * n_kt (dK/dV) or BH * n_qt (dQ)
+  int causal;
+  float scale;
+  float scale_log2;
+};
+
+// The lengths of head bh's sequence: (Nq, Nk), or its entries of seqlens_q / seqlens_k.
+// A length out of range sets kErrBadLength and skips the sequence: (0, 0).
+__device__ __forceinline__ void seq_lengths(const BwdArgs& a, int bh, int& lq, int& lk) {
+  lq = a.Nq;
+  lk = a.Nk;
+  if (a.seqlens_q == nullptr) return;
+  const int b = bh / a.H;
+  lq = a.seqlens_q[b];
+  lk = a.seqlens_k[b];
+  if (lq < 0 || lq > a.Nq || lk < 0 || lk > a.Nk || (a.causal && lq > lk)) {
+    atomicOr(a.err, kErrBadLength);
+    lq = 0;
+    lk = 0;
+  }
+}
+
+// Query rows of head bh that hold data (the rest of the padded length is padding).
+__device__ __forceinline__ int row_limit(const BwdArgs& a, int bh) {
+  int lq, lk;
+  seq_lengths(a, bh, lq, lk);
+  return lq;
+}
+
 // ------------------------------------------------------------------ 1. preparation
 // Stores the negated row statistics the element-wise steps add:
 //   ND[bh][r] = -sum_k dO[bh][r][k] * O[bh][r][k],   NL2[bh][r] = -LSE[bh][r] * log2(e).
@@ -92,8 +137,9 @@ constexpr int kPrepRowsPerThread = 4;
 template <int D>
 __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(
     const __nv_bfloat16* __restrict__ O, const __nv_bfloat16* __restrict__ dO,
-    const float* __restrict__ LSE, float* __restrict__ Dout, float* __restrict__ L2out, int BH,
-    int N, int Npad) {
+    const float* __restrict__ LSE, float* __restrict__ Dout, float* __restrict__ L2out,
+    const BwdArgs a) {
+  const int BH = a.BH, N = a.Nq, Npad = a.Npad;
   constexpr int kPer = D / 8;                         // threads per row (8 bf16 each)
   constexpr int kRowsPerPass = kPrepThreads / kPer;   // rows covered by one pass
   const int part = threadIdx.x % kPer;
@@ -108,7 +154,7 @@ __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(
     if (row >= total) continue;
     const int bh = static_cast<int>(row / Npad);
     const int r = static_cast<int>(row % Npad);
-    if (r < N) {
+    if (r < row_limit(a, bh)) {
       const size_t off = (static_cast<size_t>(bh) * N + r) * D + part * 8;
       const uint4 a = *reinterpret_cast<const uint4*>(O + off);
       const uint4 b = *reinterpret_cast<const uint4*>(dO + off);
@@ -132,30 +178,11 @@ __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(
       const int bh = static_cast<int>(row / Npad);
       const int r = static_cast<int>(row % Npad);
       Dout[row] = -acc[k];
-      L2out[row] = r < N ? -LSE[static_cast<size_t>(bh) * N + r] * kLog2e : -INFINITY;
+      L2out[row] = r < row_limit(a, bh) ? -LSE[static_cast<size_t>(bh) * N + r] * kLog2e
+                                        : -INFINITY;
     }
   }
 }
-
-struct BwdArgs {
-  unsigned int* err;
-  __nv_bfloat16* dQ;
-  __nv_bfloat16* dK;
-  __nv_bfloat16* dV;
-  const float* Dpad;   // [BH][Npad]: -D
-  const float* L2pad;  // [BH][Npad]: -LSE * log2(e)
-  int BH;
-  int Nq;           // query rows per head (Q, O, dO, dQ, LSE)
-  int Nk;           // key rows per head (K, V, dK, dV)
-  int off;          // causal: Nk - Nq, the position of query row 0 among the keys
-  int Npad;         // Nq rounded up to whole tiles
-  int n_qt;         // ceil(Nq / 128)
-  int n_kt;         // ceil(Nk / 128)
-  int total_units;  // this kernel's units: BH * n_kt (dK/dV) or BH * n_qt (dQ)
-  int causal;
-  float scale;
-  float scale_log2;
-};
 
 // Convert 32 fp32 accumulator columns (times `mul`) to bf16 and store them to a row.
 __device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t* v, float mul) {
@@ -264,17 +291,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t tdV = tmem, tdK = tmem + D, tS = tmem + 2 * D, tdP = tmem + 2 * D + 128;
 
-  auto unit = [&](int w, int& bh, int& j, int& i0) {
+  // unit w: key tile j of head bh, meeting query tiles i0 .. i0 + m - 1 of its sequence
+  // (m = 0: the tile lies past the sequence's keys, or the sequence has no queries)
+  auto unit = [&](int w, int& bh, int& j, int& i0, int& m, int& lk, int& off) {
     if (args.causal) {
       j = w / args.BH;  // key tile 0 meets every query tile: heaviest first
       bh = w % args.BH;
-      // first query tile with a row whose position reaches key j*128
-      i0 = j * kTile > args.off ? (j * kTile - args.off) / kTile : 0;
     } else {
       bh = w / args.n_kt;
       j = w % args.n_kt;
-      i0 = 0;
     }
+    int lq;
+    seq_lengths(args, bh, lq, lk);
+    off = lk - lq;  // position of query row 0 among the keys
+    i0 = 0;
+    if (j * kTile >= lk || lq == 0) {
+      m = 0;
+      return;
+    }
+    // causal: first query tile with a row whose position reaches key j*128
+    if (args.causal && j * kTile > off) i0 = (j * kTile - off) / kTile;
+    m = (lq + kTile - 1) / kTile - i0;
   };
   auto qslot = [&](int s) -> uint32_t { return base + L::kQ0 + s * L::kTileBytes; };
   auto doslot = [&](int s) -> uint32_t { return base + L::kDO0 + s * L::kDOSlotBytes; };
@@ -287,10 +324,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     int q_issued[L::kQStages] = {}, d_issued[L::kDOStages] = {};
     uint32_t q_phase[L::kQStages] = {}, d_phase[L::kDOStages] = {};
     bool ok = true;
+    int live = 0;  // 1 when the unit just processed had work: units counts only those
     for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
-         w = snake_unit(++r), ++units) {
-      int bh, j, i0;
-      unit(w, bh, j, i0);
+         w = snake_unit(++r), units += live) {
+      int bh, j, i0, m, lk, off;
+      unit(w, bh, j, i0, m, lk, off);
+      live = m > 0;
+      if (!live) continue;
       if (units > 0) ok = wait_warp(bar(L::kBarKVEmpty), (units - 1) & 1);
       if (!ok) break;
       mbar_arrive_expect_tx_elect(bar(L::kBarKVFull), 2 * L::kTileBytes);
@@ -299,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d_elect(base + L::kV + c * L::kBoxBytes, &tmV, bar(L::kBarKVFull), c * 64, j * kTile, bh);
       }
       ++kv_loads;
-      for (int i = i0; ok && i < args.n_qt; ++i) {
+      for (int i = i0; ok && i < i0 + m; ++i) {
         ok = wait_warp(bar(L::kBarQEmpty + qs), qph ^ 1);
         if (!ok) break;
         mbar_arrive_expect_tx_elect(bar(L::kBarQFull + qs), L::kTileBytes);
@@ -378,11 +418,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       issue_ss(tdP, dV0, doslot(slot), bar(L::kBarDPFull));
       return true;
     };
+    int live = 0;
     for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
-         w = snake_unit(++r), ++units) {
-      int bh, j, i0;
-      unit(w, bh, j, i0);
-      const int m = args.n_qt - i0;
+         w = snake_unit(++r), units += live) {
+      int bh, j, i0, m, lk, off;
+      unit(w, bh, j, i0, m, lk, off);
+      live = m > 0;
+      if (!live) continue;
       ok = wait_warp(bar(L::kBarKVFull), units & 1);
       int curq = 0, curd = 0;
       if (ok) ok = next_s(curq);
@@ -429,11 +471,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     int stage = 0, units = 0, s_cnt = 0, dp_cnt = 0;
     uint32_t phase = 0;
     bool ok = true;
+    int live = 0;
     for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
-         w = snake_unit(++r), ++units) {
-      int bh, j, i0;
-      unit(w, bh, j, i0);
-      for (int i = i0; i < args.n_qt; ++i) {
+         w = snake_unit(++r), units += live) {
+      int bh, j, i0, m, lk, off;
+      unit(w, bh, j, i0, m, lk, off);
+      live = m > 0;
+      if (!live) continue;
+      for (int i = i0; i < i0 + m; ++i) {
         // this tile's L2 and D rows sit in its dO slot
         const uint8_t* sb = smem + L::kDO0 + stage * L::kDOSlotBytes;
         const float* sL = reinterpret_cast<const float*>(sb + L::kSlotL) + col0;
@@ -452,7 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld32(tS + lane_off + col0 + c * 32, &r[c * 32]);
           tmem_wait_ld();
           // causal: key j*128+row is hidden from query i*128+col when col < row + delta
-          const int delta = (j - i) * kTile - args.off;
+          const int delta = (j - i) * kTile - off;
           const bool diag = args.causal && delta > -kTile;
           const uint64_t scale2 = f32x2(args.scale_log2, args.scale_log2);
 #pragma unroll
@@ -514,16 +559,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const int kv_row = j * kTile + row;
-      const size_t off = (static_cast<size_t>(bh) * args.Nk + kv_row) * D;
+      const size_t orow = (static_cast<size_t>(bh) * args.Nk + kv_row) * D;
 #pragma unroll 1
       for (int c = g * (D / 64); c < (g + 1) * (D / 64); ++c) {
         uint32_t v[32];
         tmem_ld32(tdV + lane_off + c * 32, v);
         tmem_wait_ld();
-        if (kv_row < args.Nk) store_row32(args.dV + off + c * 32, v, 1.f);
+        if (kv_row < lk) store_row32(args.dV + orow + c * 32, v, 1.f);
         tmem_ld32(tdK + lane_off + c * 32, v);
         tmem_wait_ld();
-        if (kv_row < args.Nk) store_row32(args.dK + off + c * 32, v, args.scale);
+        if (kv_row < lk) store_row32(args.dK + orow + c * 32, v, args.scale);
       }
       warp_arrive(bar(L::kBarAccFree));
     }
@@ -631,17 +676,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   // dP products can start as soon as the element-wise warps have read this tile's.
   const uint32_t tdQ = tmem, tS = tmem + 128, tdP = tmem + 256, tdS = tmem + 384;
 
-  auto unit = [&](int w, int& bh, int& i, int& m) {
+  // unit w: query tile i of head bh, meeting key tiles 0 .. m - 1 of its sequence
+  // (m = 0: the tile lies past the sequence's queries, or the sequence has no keys)
+  auto unit = [&](int w, int& bh, int& i, int& m, int& lq, int& lk, int& off) {
     if (args.causal) {
       i = args.n_qt - 1 - w / args.BH;  // last query tile meets the most key tiles
       bh = w % args.BH;
-      // key tiles up to the one holding the position of the tile's last row
-      m = min((i * kTile + kTile - 1 + args.off) / kTile + 1, args.n_kt);
     } else {
       bh = w / args.n_qt;
       i = w % args.n_qt;
-      m = args.n_kt;
     }
+    seq_lengths(args, bh, lq, lk);
+    off = lk - lq;
+    if (i * kTile >= lq || lk == 0) {
+      m = 0;
+      return;
+    }
+    const int n_kv = (lk + kTile - 1) / kTile;
+    // causal: key tiles up to the one holding the position of the tile's last row
+    m = args.causal ? min((i * kTile + kTile - 1 + off) / kTile + 1, n_kv) : n_kv;
   };
 
   if (warp >= kWarpTMA) regs_dec<kRegsControl>();
@@ -653,10 +706,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       int k_issued[L::kKStages] = {}, v_issued[L::kVStages] = {};
       uint32_t k_phase[L::kKStages] = {}, v_phase[L::kVStages] = {};
       bool ok = true;
+      int live = 0;  // 1 when the unit just processed had work: units counts only those
       for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
-         w = snake_unit(++r), ++units) {
-        int bh, i, m;
-        unit(w, bh, i, m);
+         w = snake_unit(++r), units += live) {
+        int bh, i, m, lq, lk, off;
+        unit(w, bh, i, m, lq, lk, off);
+        live = m > 0;
+        if (!live) continue;
         if (units > 0) ok = wait_warp(bar(L::kBarQEmpty), (units - 1) & 1);
         if (!ok) break;
         mbar_arrive_expect_tx_elect(bar(L::kBarQFull), 2 * L::kTileBytes);
@@ -728,10 +784,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       int dpfree_cnt = 0;
+      int live = 0;
       for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
-         w = snake_unit(++r), ++units) {
-        int bh, i, m;
-        unit(w, bh, i, m);
+         w = snake_unit(++r), units += live) {
+        int bh, i, m, lq, lk, off;
+        unit(w, bh, i, m, lq, lk, off);
+        live = m > 0;
+        if (!live) continue;
         ok = wait_warp(bar(L::kBarQFull), units & 1);
         if (ok) ok = wait_warp(bar(L::kBarKFull + kc), kcph);
         if (!ok) break;
@@ -798,10 +857,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>((warp % 4) * 32) << 16;
     int units = 0, s_cnt = 0, dp_cnt = 0, dq_cnt = 0;
     bool ok = true;
+    int live = 0;
     for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
-         w = snake_unit(++r), ++units) {
-      int bh, i, m;
-      unit(w, bh, i, m);
+         w = snake_unit(++r), units += live) {
+      int bh, i, m, lq, lk, off;
+      unit(w, bh, i, m, lq, lk, off);
+      live = m > 0;
+      if (!live) continue;
       const int q_row = i * kTile + row;
       const size_t prow = static_cast<size_t>(bh) * args.Npad + q_row;  // q_row < Npad
       const float nl2row = args.L2pad[prow];   // -LSE * log2(e) of this query row
@@ -823,9 +885,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int kv0 = j * kTile + col0;
           // a ragged last key tile, or (causal) keys past the position of the tile's
           // first row
-          const bool need_mask = (kv0 + kCols > args.Nk) ||
-                                 (args.causal && kv0 + kCols - 1 > i * kTile + args.off);
-          const int lim = args.causal ? min(args.Nk, q_row + args.off + 1) : args.Nk;
+          const bool need_mask = (kv0 + kCols > lk) ||
+                                 (args.causal && kv0 + kCols - 1 > i * kTile + off);
+          const int lim = args.causal ? min(lk, q_row + off + 1) : lk;
           const uint64_t scale2 = f32x2(args.scale_log2, args.scale_log2);
           const uint64_t nl2 = f32x2(nl2row, nl2row);
 #pragma unroll
@@ -877,13 +939,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const size_t off = (static_cast<size_t>(bh) * args.Nq + q_row) * D;
+      const size_t orow = (static_cast<size_t>(bh) * args.Nq + q_row) * D;
 #pragma unroll 1
       for (int c = g * (D / 64); c < (g + 1) * (D / 64); ++c) {
         uint32_t v[32];
         tmem_ld32(tdQ + lane_off + c * 32, v);
         tmem_wait_ld();
-        if (q_row < args.Nq) store_row32(args.dQ + off + c * 32, v, args.scale);
+        if (q_row < lq) store_row32(args.dQ + orow + c * 32, v, args.scale);
       }
       warp_arrive(bar(L::kBarAccFree));
     }
@@ -910,9 +972,11 @@ cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUten
   a.dK = static_cast<__nv_bfloat16*>(dK);
   a.dV = static_cast<__nv_bfloat16*>(dV);
   a.BH = p.BH;
+  a.seqlens_q = p.seqlens_q;
+  a.seqlens_k = p.seqlens_k;
+  a.H = p.H;
   a.Nq = p.N;
   a.Nk = p.Nk;
-  a.off = p.Nk - p.N;
   a.n_qt = (p.N + kTile - 1) / kTile;
   a.n_kt = (p.Nk + kTile - 1) / kTile;
   a.Npad = a.n_qt * kTile;
@@ -931,7 +995,7 @@ cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUten
   bwd_prep_kernel<D><<<static_cast<unsigned>((rows + rows_per_block - 1) / rows_per_block),
                        kPrepThreads, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO), LSE, Dpad,
-      L2pad, p.BH, p.N, a.Npad);
+      L2pad, a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if ((e = trace_mark(p, 1, stream)) != cudaSuccess) return e;
 

@@ -139,8 +139,6 @@ bool overlaps(const void* a, size_t a_bytes, const void* b, size_t b_bytes) {
   return x < y + b_bytes && y < x + a_bytes;
 }
 
-bool overlaps(const void* a, const void* b, size_t bytes) { return overlaps(a, bytes, b, bytes); }
-
 // Checks shared by every call: Nq query rows and Nk key rows per head (Nk == Nq for
 // the entry points without the _qk suffix).  Sets *noop when there is nothing to
 // compute.
@@ -245,8 +243,37 @@ fa_status check_bwd_args(const void* Q, const void* K, const void* V, const void
   return FA_OK;
 }
 
+fa::Problem make_problem(int B, int H, int Nq, int Nk, int d, float scale, int causal,
+                         const DeviceInfo& dev, const int* seqlens_q = nullptr,
+                         const int* seqlens_k = nullptr) {
+  fa::Problem p{};
+  p.BH = B * H;
+  p.N = Nq;
+  p.Nk = Nk;
+  p.d = d;
+  p.scale = scale;
+  p.causal = causal;
+  p.err = dev.err;
+  p.seqlens_q = seqlens_q;
+  p.seqlens_k = seqlens_k;
+  p.H = H;
+  p.trace = g_n_trace ? g_trace : nullptr;
+  p.n_trace = g_n_trace;
+  return p;
+}
+
+// Per-sequence length arrays of the padded-batch calls: both given, 4-byte aligned.
+fa_status check_seqlens(const int* seqlens_q, const int* seqlens_k) {
+  if (seqlens_q == nullptr || seqlens_k == nullptr)
+    return fail(FA_ERR_INVALID_ARG, "seqlens_q and seqlens_k are required");
+  if ((reinterpret_cast<uintptr_t>(seqlens_q) | reinterpret_cast<uintptr_t>(seqlens_k)) & 3u)
+    return fail(FA_ERR_INVALID_ARG, "seqlens_q and seqlens_k must be 4-byte aligned");
+  return FA_OK;
+}
+
 fa_status fwd_impl(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
-                   int H, int Nq, int Nk, int d, float scale, int causal, cudaStream_t stream) {
+                   int H, int Nq, int Nk, int d, float scale, int causal, cudaStream_t stream,
+                   const int* seqlens_q = nullptr, const int* seqlens_k = nullptr) {
   g_last_error[0] = '\0';
   bool noop = false;
   FA_TRY(check_fwd_args(Q, K, V, O, LSE, B, H, Nq, Nk, d, scale, causal, 2, &noop));
@@ -259,8 +286,7 @@ fa_status fwd_impl(const void* Q, const void* K, const void* V, void* O, float* 
   FA_TRY(make_tmap(&tmQ, Q, BH, Nq, d));
   FA_TRY(make_tmap(&tmK, K, BH, Nk, d));
   FA_TRY(make_tmap(&tmV, V, BH, Nk, d));
-  fa::Problem p{BH, Nq, Nk, d, scale, causal, dev.err, g_n_trace ? g_trace : nullptr,
-                g_n_trace};
+  const fa::Problem p = make_problem(B, H, Nq, Nk, d, scale, causal, dev, seqlens_q, seqlens_k);
   cudaError_t e = fa::launch_fwd_sm100(tmQ, tmK, tmV, O, LSE, p, dev.num_sms, stream);
   if (e != cudaSuccess) return cuda_fail(e, "launching the forward kernel");
   return FA_OK;
@@ -269,7 +295,8 @@ fa_status fwd_impl(const void* Q, const void* K, const void* V, void* O, float* 
 fa_status bwd_impl(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                    const float* LSE, void* dQ, void* dK, void* dV, int B, int H, int Nq, int Nk,
                    int d, float scale, int causal, void* workspace, size_t workspace_bytes,
-                   cudaStream_t stream) {
+                   cudaStream_t stream, const int* seqlens_q = nullptr,
+                   const int* seqlens_k = nullptr) {
   g_last_error[0] = '\0';
   bool noop = false;
   FA_TRY(check_bwd_args(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, Nq, Nk, d, scale, causal,
@@ -288,8 +315,7 @@ fa_status bwd_impl(const void* Q, const void* K, const void* V, const void* O, c
   float* ws = static_cast<float*>(workspace);
   FA_TRY(make_row_tmap(&tmD, ws, BH, Npad));
   FA_TRY(make_row_tmap(&tmL2, ws + static_cast<size_t>(BH) * Npad, BH, Npad));
-  fa::Problem p{BH, Nq, Nk, d, scale, causal, dev.err, g_n_trace ? g_trace : nullptr,
-                g_n_trace};
+  const fa::Problem p = make_problem(B, H, Nq, Nk, d, scale, causal, dev, seqlens_q, seqlens_k);
   cudaError_t e = fa::launch_bwd_sm100(tmQ, tmK, tmV, tmdO, tmL2, tmD, O, dO, LSE, dQ, dK, dV,
                                        ws, p, dev.num_sms, stream);
   if (e != cudaSuccess) return cuda_fail(e, "launching the backward kernels");
@@ -336,6 +362,15 @@ fa_status fa_fwd_qk(const void* Q, const void* K, const void* V, void* O, float*
   return fwd_impl(Q, K, V, O, LSE, B, H, Nq, Nk, d, scale, causal, stream);
 }
 
+fa_status fa_fwd_varlen(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                        const int* seqlens_q, const int* seqlens_k, int B, int H, int Nq,
+                        int Nk, int d, float scale, int causal, cudaStream_t stream) {
+  g_last_error[0] = '\0';
+  if (B > 0 && H > 0 && Nq > 0) FA_TRY(check_seqlens(seqlens_q, seqlens_k));
+  return fwd_impl(Q, K, V, O, LSE, B, H, Nq, Nk, d, scale, causal, stream, seqlens_q,
+                  seqlens_k);
+}
+
 fa_status fa_fwd_f32(const float* Q, const float* K, const float* V, float* O, float* LSE,
                      int B, int H, int N, int d, float scale, int causal,
                      cudaStream_t stream) {
@@ -345,8 +380,7 @@ fa_status fa_fwd_f32(const float* Q, const float* K, const float* V, float* O, f
   if (noop) return FA_OK;  // empty problem: the pointers are never used (may be NULL)
   DeviceInfo dev;
   FA_TRY(device_info(&dev));
-  fa::Problem p{B * H, N, N, d, scale, causal, dev.err, g_n_trace ? g_trace : nullptr,
-                g_n_trace};
+  const fa::Problem p = make_problem(B, H, N, N, d, scale, causal, dev);
   cudaError_t e = fa::launch_fwd_f32(Q, K, V, O, LSE, p, stream);
   if (e != cudaSuccess) return cuda_fail(e, "launching the float32 forward kernel");
   return FA_OK;
@@ -376,6 +410,17 @@ fa_status fa_bwd_qk(const void* Q, const void* K, const void* V, const void* O, 
                   workspace_bytes, stream);
 }
 
+fa_status fa_bwd_varlen(const void* Q, const void* K, const void* V, const void* O,
+                        const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                        const int* seqlens_q, const int* seqlens_k, int B, int H, int Nq,
+                        int Nk, int d, float scale, int causal, void* workspace,
+                        size_t workspace_bytes, cudaStream_t stream) {
+  g_last_error[0] = '\0';
+  if (B > 0 && H > 0 && Nq > 0) FA_TRY(check_seqlens(seqlens_q, seqlens_k));
+  return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, Nq, Nk, d, scale, causal, workspace,
+                  workspace_bytes, stream, seqlens_q, seqlens_k);
+}
+
 fa_status fa_bwd_f32(const float* Q, const float* K, const float* V, const float* O,
                      const float* dO, const float* LSE, float* dQ, float* dK, float* dV, int B,
                      int H, int N, int d, float scale, int causal, void* workspace,
@@ -387,8 +432,7 @@ fa_status fa_bwd_f32(const float* Q, const float* K, const float* V, const float
   if (noop) return FA_OK;  // empty problem: the pointers are never used (may be NULL)
   DeviceInfo dev;
   FA_TRY(device_info(&dev));
-  fa::Problem p{B * H, N, N, d, scale, causal, dev.err, g_n_trace ? g_trace : nullptr,
-                g_n_trace};
+  const fa::Problem p = make_problem(B, H, N, N, d, scale, causal, dev);
   cudaError_t e = fa::launch_bwd_f32(Q, K, V, O, dO, LSE, dQ, dK, dV,
                                      static_cast<float*>(workspace), p, stream);
   if (e != cudaSuccess) return cuda_fail(e, "launching the float32 backward kernels");
@@ -408,6 +452,11 @@ fa_status fa_check_device_error(cudaStream_t stream) {
     const unsigned int zero = 0;
     e = cudaMemcpy(dev.err, &zero, sizeof(zero), cudaMemcpyHostToDevice);
     if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+    if (word & 4u)
+      return fail(FA_ERR_INVALID_ARG,
+                  "a per-sequence length was negative, above the padded length, or (causal) "
+                  "had more queries than keys; that sequence was skipped (error word 0x%x)",
+                  word);
     if (word & 2u)
       return fail(FA_ERR_CUDA,
                   "a kernel found its dynamic shared memory misaligned and did no work "

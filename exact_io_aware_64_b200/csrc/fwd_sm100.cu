@@ -38,6 +38,10 @@
 //     last row's position; only tiles that cross a row's limit, and a ragged last key
 //     tile, need element masks.  Rows past Nq (ragged last query tile) are computed on
 //     zero-filled Q and never stored.
+//   * Padded batches: with per-sequence lengths (seqlens_q[b], seqlens_k[b] <= Nq, Nk)
+//     sequence b uses its first seqlens_q[b] query and seqlens_k[b] key rows, with the
+//     same alignment rule; units past a sequence's queries have no work and every role
+//     skips them.  Key rows past a sequence's length are masked like a ragged tail.
 #include <cfloat>
 #include <cstdint>
 
@@ -97,10 +101,12 @@ struct FwdArgs {
   unsigned int* err;  // library error word (wait timeouts)
   __nv_bfloat16* O;
   float* LSE;
+  const int* seqlens_q;  // [B] per-sequence query rows, or null (all Nq)
+  const int* seqlens_k;  // [B] per-sequence key rows, or null (all Nk)
+  int H;
   int BH;
-  int Nq;           // query rows per head
-  int Nk;           // key rows per head
-  int off;          // causal: Nk - Nq, the position of query row 0
+  int Nq;           // query rows per head (padded length with seqlens)
+  int Nk;           // key rows per head (padded length with seqlens)
   int causal;
   int n_units;      // units per (batch, head) = ceil(Nq / 256)
   int total_units;  // BH * n_units
@@ -108,7 +114,8 @@ struct FwdArgs {
 };
 
 struct UnitInfo {
-  int bh, u, n0, n1;
+  int bh, u, n0, n1;  // n_t: key tiles of query tile t (0: no work)
+  int lq, lk, off;    // the sequence's query rows, key rows, position of query row 0
 };
 
 __device__ __forceinline__ UnitInfo unit_info(int w, const FwdArgs& a) {
@@ -121,12 +128,26 @@ __device__ __forceinline__ UnitInfo unit_info(int w, const FwdArgs& a) {
     r.bh = w / a.n_units;
     r.u = w % a.n_units;
   }
-  const int n_kv = (a.Nk + kBN - 1) / kBN;
+  r.lq = a.Nq;
+  r.lk = a.Nk;
+  if (a.seqlens_q != nullptr) {
+    const int b = r.bh / a.H;
+    r.lq = a.seqlens_q[b];
+    r.lk = a.seqlens_k[b];
+    if (r.lq < 0 || r.lq > a.Nq || r.lk < 0 || r.lk > a.Nk || (a.causal && r.lq > r.lk)) {
+      if (threadIdx.x == 0) atomicOr(a.err, kErrBadLength);
+      r.lq = 0;  // the sequence is skipped
+      r.lk = 0;
+    }
+  }
+  r.off = r.lk - r.lq;
+  const int n_kv = (r.lk + kBN - 1) / kBN;
   const int qt0 = 2 * r.u, qt1 = 2 * r.u + 1;
-  const bool valid1 = qt1 * kBM < a.Nq;
+  const bool valid0 = r.lk > 0 && qt0 * kBM < r.lq;
+  const bool valid1 = r.lk > 0 && qt1 * kBM < r.lq;
   // causal: key tiles up to the one holding the position of the tile's last row
-  auto n_causal = [&](int qt) { return min((qt * kBM + kBM - 1 + a.off) / kBN + 1, n_kv); };
-  r.n0 = a.causal ? n_causal(qt0) : n_kv;
+  auto n_causal = [&](int qt) { return min((qt * kBM + kBM - 1 + r.off) / kBN + 1, n_kv); };
+  r.n0 = valid0 ? (a.causal ? n_causal(qt0) : n_kv) : 0;
   r.n1 = valid1 ? (a.causal ? n_causal(qt1) : n_kv) : 0;
   return r;
 }
@@ -204,6 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int s = 0; s < L::kStages; ++s) issued[s] = 0, issued_phase[s] = 0;
       for (int r = 0, w = snake_unit(0); ok && w < args.total_units; w = snake_unit(++r)) {
         const UnitInfo ui = unit_info(w, args);
+        if (ui.n0 == 0) continue;  // no query rows in this unit (every role skips it)
         for (int t = 0; t < 2 && ok; ++t) {
           if (t == 1 && ui.n1 == 0) break;
           if (q_uses[t] > 0)
@@ -290,6 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       for (int r = 0, w = snake_unit(0); ok && w < args.total_units; w = snake_unit(++r)) {
         const UnitInfo ui = unit_info(w, args);
+        if (ui.n0 == 0) continue;  // no query rows in this unit
         const int nt[2] = {ui.n0, ui.n1};
         const int n = max(ui.n0, ui.n1);
         for (int t = 0; t < 2 && ok; ++t)
@@ -372,10 +395,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kv0 = j * kBN;
         // a ragged last key tile, or (causal) a tile whose last key lies past the
         // position of the tile's first row
-        const bool need_mask = (kv0 + kBN > args.Nk) ||
-                               (args.causal && kv0 + kBN - 1 > qt * kBM + args.off);
+        const bool need_mask = (kv0 + kBN > ui.lk) ||
+                               (args.causal && kv0 + kBN - 1 > qt * kBM + ui.off);
         if (need_mask) {
-          const int lim = args.causal ? min(args.Nk, q_row + args.off + 1) : args.Nk;
+          const int lim = args.causal ? min(ui.lk, q_row + ui.off + 1) : ui.lk;
 #pragma unroll
           for (int c = 0; c < kBN; ++c)
             if (kv0 + c >= lim) s[c] = -INFINITY;
@@ -462,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < D / 32; ++c) tmem_ld32(tOrow + c * 32, &ov[c * 32]);
       tmem_wait_ld();
       warp_arrive(bar(L::kBarOFree + t));
-      if (q_row < args.Nq) {
+      if (q_row < ui.lq) {
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t pk[16];
@@ -476,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
         }
       }
-      if (args.LSE != nullptr && q_row < args.Nq)
+      if (args.LSE != nullptr && q_row < ui.lq)
         args.LSE[static_cast<size_t>(bh) * args.Nq + q_row] =
             (m + __log2f(l)) * 0.69314718055994531f;
     }
@@ -500,9 +523,11 @@ cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUten
   a.O = static_cast<__nv_bfloat16*>(O);
   a.LSE = LSE;
   a.BH = p.BH;
+  a.seqlens_q = p.seqlens_q;
+  a.seqlens_k = p.seqlens_k;
+  a.H = p.H;
   a.Nq = p.N;
   a.Nk = p.Nk;
-  a.off = p.Nk - p.N;
   a.causal = p.causal;
   a.n_units = (p.N + 2 * kBM - 1) / (2 * kBM);
   a.total_units = p.BH * a.n_units;

@@ -19,6 +19,11 @@ struct Problem {
   float scale;
   int causal;
   unsigned int* err;  // device address of the library's error word
+  // padded batches: per-sequence lengths [B] on the device (both null otherwise); H
+  // heads per sequence, so head bh belongs to sequence bh / H
+  const int* seqlens_q;
+  const int* seqlens_k;
+  int H;
   // optional kernel-boundary events (fa_trace_events): trace[0] before the first kernel,
   // trace[k] after the k-th; n_trace entries
   cudaEvent_t* trace;

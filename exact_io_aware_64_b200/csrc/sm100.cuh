@@ -72,6 +72,7 @@ constexpr uint32_t kSpinCheck = 256;
 // dynamic shared memory not aligned as its layout requires (it then does no work).
 constexpr unsigned int kErrWaitTimeout = 1u;
 constexpr unsigned int kErrSmemAlign = 2u;
+constexpr unsigned int kErrBadLength = 4u;  // a per-sequence length out of range
 
 // Wait until the phase with the given parity has completed.  Returns false if the time
 // limit runs out (then it also sets kErrWaitTimeout in *err and raises *abort so the

@@ -103,6 +103,26 @@ FA_API fa_status fa_fwd_qk(const void* Q, const void* K, const void* V, void* O,
                            cudaStream_t stream);
 
 /*
+ * Forward pass over a padded batch of sequences of different lengths (no counterpart on
+ * the pages; the queries of each sequence are aligned with the end of its keys as in
+ * fa_fwd_qk).  Tensors are padded to common lengths:
+ *   Q, O [B,H,Nq,d] bf16;  K, V [B,H,Nk,d] bf16;  LSE [B,H,Nq] float32 or NULL
+ *   seqlens_q, seqlens_k: device int32 arrays [B], 4-byte aligned, required; sequence b
+ *     uses its first seqlens_q[b] query rows and seqlens_k[b] key rows
+ *     (0 <= seqlens_q[b] <= Nq, 0 <= seqlens_k[b] <= Nk, and causal needs
+ *     seqlens_q[b] <= seqlens_k[b]).
+ * Rows past a sequence's query length (in O and LSE) are not written.  A sequence with no
+ * queries or no keys is skipped.  Padding rows of K and V must hold finite values (their
+ * probabilities are zero, and 0 times a NaN is a NaN).  The lengths are read on the
+ * device: one out of range makes the kernel skip that sequence and makes
+ * fa_check_device_error report FA_ERR_INVALID_ARG.  Otherwise as fa_fwd_qk.
+ */
+FA_API fa_status fa_fwd_varlen(const void* Q, const void* K, const void* V, void* O,
+                               float* LSE, const int* seqlens_q, const int* seqlens_k, int B,
+                               int H, int Nq, int Nk, int d, float scale, int causal,
+                               cudaStream_t stream);
+
+/*
  * Forward pass with float32 inputs and outputs, computed in float32 on the CUDA cores
  * (same definition and arguments as fa_fwd).
  */
@@ -146,6 +166,21 @@ FA_API fa_status fa_bwd_qk(const void* Q, const void* K, const void* V, const vo
                            const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
                            int B, int H, int Nq, int Nk, int d, float scale, int causal,
                            void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Backward pass over a padded batch (the gradient of fa_fwd_varlen, same lengths).
+ *   Q, O, dO, dQ [B,H,Nq,d] bf16;  K, V, dK, dV [B,H,Nk,d] bf16;  LSE [B,H,Nq] float32
+ *   workspace: fa_bwd_workspace_bytes(B,H,Nq,d) bytes
+ * Rows past a sequence's lengths (dQ past seqlens_q[b], dK and dV past seqlens_k[b]) are
+ * not written.  Padding rows of Q, K, V, O and dO must hold finite values.  Lengths as
+ * for fa_fwd_varlen; otherwise as fa_bwd_qk.
+ */
+FA_API fa_status fa_bwd_varlen(const void* Q, const void* K, const void* V, const void* O,
+                               const void* dO, const float* LSE, void* dQ, void* dK,
+                               void* dV, const int* seqlens_q, const int* seqlens_k, int B,
+                               int H, int Nq, int Nk, int d, float scale, int causal,
+                               void* workspace, size_t workspace_bytes,
+                               cudaStream_t stream);
 
 /*
  * Backward pass, float32: the same computation as fa_bwd with float32 inputs, outputs

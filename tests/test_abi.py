@@ -178,3 +178,21 @@ def test_qk_validation(lib):
     assert bwd(100, 1000, ws_bytes=need - 4) == binding.FA_ERR_INVALID_ARG
     assert bwd(100, 1000, ws_bytes=need) != binding.FA_ERR_INVALID_ARG
     assert bwd(100, 1000, dk=G + 2 * 100 * 64 * 2 - 16) == binding.FA_ERR_INVALID_ARG
+
+
+def test_varlen_validation(lib):
+    """fa_fwd_varlen / fa_bwd_varlen: the length arrays are required (values are checked on
+    the device); the padded shapes follow the fa_fwd_qk rules."""
+    SQ, SK = 0xB00000, 0xC00000
+    def fwd(sq=SQ, sk=SK, Nq=64, Nk=64, causal=1):
+        return lib.fa_fwd_varlen(A, B_, C, D_, E, sq, sk, 2, 2, Nq, Nk, 64, 0.1, causal, None)
+
+    assert fwd(sq=0) == binding.FA_ERR_INVALID_ARG
+    assert fwd(sk=0) == binding.FA_ERR_INVALID_ARG
+    assert fwd(sq=SQ + 2) == binding.FA_ERR_INVALID_ARG      # misaligned
+    assert fwd(Nq=128, Nk=64) == binding.FA_ERR_INVALID_ARG   # causal: padded Nq <= Nk
+    assert fwd(Nq=0, sq=0, sk=0) == binding.FA_OK             # empty: no-op
+    F, G, H_, I, J = 0x600000, 0x700000, 0x800000, 0x900000, 0xA00000
+    st = lib.fa_bwd_varlen(A, B_, C, D_, E, F, G, H_, I, 0, SK, 2, 2, 64, 64, 64, 0.1, 1, J,
+                           1 << 20, None)
+    assert st == binding.FA_ERR_INVALID_ARG
