@@ -53,11 +53,21 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def library_digest() -> str:
+KERNEL_SOURCES = {
+    "fwd_sm100_kernel": ("fwd_sm100.cu", "sm100.cuh"),
+    "bwd_prep_kernel": ("bwd_sm100.cu", "sm100.cuh"),
+    "bwd_dkdv_kernel": ("bwd_sm100.cu", "sm100.cuh"),
+    "bwd_dq_kernel": ("bwd_sm100.cu", "sm100.cuh"),
+}
+
+
+def kernel_digest(kernel: str) -> str:
+    """Hash of the sources that define `kernel` (its translation unit and the sm_100a
+    primitives it includes)."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_io_aware_64_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -65,14 +75,14 @@ def library_digest() -> str:
 
 def recorded_traffic(kernel: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on the
-    current kernel sources; otherwise None."""
+    kernel's current sources; otherwise None."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
-    if not os.path.exists(p):
+    if not os.path.exists(p) or kernel not in KERNEL_SOURCES:
         return None
     with open(p) as f:
         d = json.load(f)
     e = d.get(kernel)
-    if not e or e.get("source_digest") != library_digest():
+    if not e or e.get("source_digest") != kernel_digest(kernel):
         return None
     return e.get("bytes_per_launch")
 
