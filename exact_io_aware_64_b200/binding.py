@@ -46,6 +46,7 @@ SIGNATURES = {
                        _i, _f, _i, _vp, _sz, _vp], _i),
     "fa_bwd_f32": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp,
                     _sz, _vp], _i),
+    "fa_merge": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp], _i),
     "fa_bwd_noalloc": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i,
                         _vp], _i),
     "fa_bwd_noalloc_max_scratch_bytes": ([], _sz),
@@ -312,6 +313,27 @@ def bwd_varlen(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, O: torch.Tenso
                                  _ptr(workspace), ws_bytes, _stream_handle(stream))
     _check("fa_bwd_varlen", st)
     return dQ, dK, dV
+
+
+def merge(O_acc: torch.Tensor, LSE_acc: torch.Tensor, O_part: torch.Tensor,
+          LSE_part: torch.Tensor, O_out: Optional[torch.Tensor] = None,
+          stream: Optional[torch.cuda.Stream] = None):
+    """Merge a partial result over a block of keys into a float32 accumulator in place
+    through ``fa_merge``.  O_acc [B, H, N, d] float32, LSE_acc [B, H, N] float32 (-inf:
+    empty), O_part [B, H, N, d] bf16, LSE_part [B, H, N] float32; O_out, if given, gets
+    the merged O as bf16.  Returns (O_acc, LSE_acc)."""
+    B, H, N, d = O_acc.shape
+    _check_bhnd("O_acc", O_acc, (B, H, N, d), torch.float32)
+    _check_bhnd("LSE_acc", LSE_acc, (B, H, N), torch.float32)
+    _check_bhnd("O_part", O_part, (B, H, N, d), torch.bfloat16)
+    _check_bhnd("LSE_part", LSE_part, (B, H, N), torch.float32)
+    if O_out is not None:
+        _check_bhnd("O_out", O_out, (B, H, N, d), torch.bfloat16)
+    with torch.cuda.device(O_acc.device):
+        st = lib().fa_merge(_ptr(O_acc), _ptr(LSE_acc), _ptr(O_part), _ptr(LSE_part),
+                            _ptr(O_out), B, H, N, d, _stream_handle(stream))
+    _check("fa_merge", st)
+    return O_acc, LSE_acc
 
 
 class trace_kernels:

@@ -439,6 +439,37 @@ fa_status fa_bwd_f32(const float* Q, const float* K, const float* V, const float
   return FA_OK;
 }
 
+fa_status fa_merge(float* O_acc, float* LSE_acc, const void* O_part, const float* LSE_part,
+                   void* O_out, int B, int H, int N, int d, cudaStream_t stream) {
+  g_last_error[0] = '\0';
+  bool noop = false;
+  FA_TRY(check_common(B, H, N, N, d, 1.f, 0, &noop));
+  if (noop) return FA_OK;  // empty problem: the pointers are never used (may be NULL)
+  FA_TRY(check_ptr(O_acc, "O_acc"));
+  FA_TRY(check_ptr(O_part, "O_part"));
+  if (O_out != nullptr) FA_TRY(check_ptr(O_out, "O_out"));
+  if (LSE_acc == nullptr || LSE_part == nullptr)
+    return fail(FA_ERR_INVALID_ARG, "LSE_acc and LSE_part are required");
+  if ((reinterpret_cast<uintptr_t>(LSE_acc) | reinterpret_cast<uintptr_t>(LSE_part)) & 3u)
+    return fail(FA_ERR_INVALID_ARG, "LSE_acc and LSE_part must be 4-byte aligned");
+  const size_t rows = static_cast<size_t>(B) * H * N;
+  const size_t acc_b = rows * d * 4, part_b = rows * d * 2, lse_b = rows * 4;
+  if (overlaps(O_acc, acc_b, O_part, part_b) || overlaps(O_acc, acc_b, LSE_part, lse_b) ||
+      overlaps(LSE_acc, lse_b, O_part, part_b) || overlaps(LSE_acc, lse_b, LSE_part, lse_b) ||
+      overlaps(O_acc, acc_b, LSE_acc, lse_b))
+    return fail(FA_ERR_INVALID_ARG, "the accumulator overlaps the partial result");
+  if (O_out != nullptr &&
+      (overlaps(O_out, part_b, O_acc, acc_b) || overlaps(O_out, part_b, LSE_acc, lse_b) ||
+       overlaps(O_out, part_b, LSE_part, lse_b)))
+    return fail(FA_ERR_INVALID_ARG, "O_out overlaps the accumulator");
+  DeviceInfo dev;
+  FA_TRY(device_info(&dev));
+  const fa::Problem p = make_problem(B, H, N, N, d, 1.f, 0, dev);
+  cudaError_t e = fa::launch_merge(O_acc, LSE_acc, O_part, LSE_part, O_out, p, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "launching the merge kernel");
+  return FA_OK;
+}
+
 fa_status fa_check_device_error(cudaStream_t stream) {
   g_last_error[0] = '\0';
   cudaError_t e = cudaStreamSynchronize(stream);

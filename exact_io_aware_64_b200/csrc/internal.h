@@ -64,4 +64,10 @@ cudaError_t launch_bwd_f32(const float* Q, const float* K, const float* V, const
                            const float* dO, const float* LSE, float* dQ, float* dK, float* dV,
                            float* workspace, const Problem& p, cudaStream_t stream);
 
+// Merge of a partial attention result (O_part bf16, LSE_part) into a float32 accumulator
+// (O_acc, LSE_acc), optionally writing the merged O as bf16 to O_out; [BH][N] rows.
+cudaError_t launch_merge(float* O_acc, float* LSE_acc, const void* O_part,
+                         const float* LSE_part, void* O_out, const Problem& p,
+                         cudaStream_t stream);
+
 }  // namespace fa

@@ -199,6 +199,27 @@ FA_API fa_status fa_bwd_f32(const float* Q, const float* K, const float* V, cons
                             void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Merge a partial attention result into an accumulator ("FlashAttention, simplified",
+ * "The trick": the rescale-and-add step of the online softmax, applied to two results
+ * over disjoint key sets, as context-parallel attention needs when each GPU holds a
+ * block of the keys).  With m = max(LSE_acc, LSE_part) and w = exp(LSE - m):
+ *   O_acc <- (w_acc O_acc + w_part O_part) / (w_acc + w_part)
+ *   LSE_acc <- m + log(w_acc + w_part)
+ *   O_acc    in/out: [B,H,N,d] float32 (rows whose LSE_acc is -inf are empty; their
+ *                    values are ignored)
+ *   LSE_acc  in/out: [B,H,N] float32 natural-log normalisers (-inf: no keys yet)
+ *   O_part   in    : [B,H,N,d] bf16, e.g. fa_fwd / fa_fwd_qk over one key block
+ *   LSE_part in    : [B,H,N] float32 from the same call (-inf: an empty block)
+ *   O_out    out   : [B,H,N,d] bf16, the merged O rounded once; may be NULL
+ * A row empty on both sides stays empty (O 0, LSE -inf).  Pointers 16-byte aligned (LSE
+ * arrays 4-byte); the accumulator must not overlap the partial result.  One kernel on
+ * `stream`, one warp per row.
+ */
+FA_API fa_status fa_merge(float* O_acc, float* LSE_acc, const void* O_part,
+                          const float* LSE_part, void* O_out, int B, int H, int N, int d,
+                          cudaStream_t stream);
+
+/*
  * fa_bwd for callers that cannot allocate device memory (no counterpart on the pages:
  * it is a property of this library, not of the method).  Same arguments and result as
  * fa_bwd, without the workspace: the scratch is a fixed array inside the library,

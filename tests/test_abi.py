@@ -196,3 +196,20 @@ def test_varlen_validation(lib):
     st = lib.fa_bwd_varlen(A, B_, C, D_, E, F, G, H_, I, 0, SK, 2, 2, 64, 64, 64, 0.1, 1, J,
                            1 << 20, None)
     assert st == binding.FA_ERR_INVALID_ARG
+
+
+def test_merge_validation(lib):
+    O_acc, L_acc, O_p, L_p, O_out = 0x100000, 0x200000, 0x300000, 0x400000, 0x500000
+
+    def call(oa=O_acc, la=L_acc, op=O_p, lp=L_p, oo=O_out, N=16, d=64):
+        return lib.fa_merge(oa, la, op, lp, oo, 1, 2, N, d, None)
+
+    assert call(N=0, oa=0, la=0, op=0, lp=0) == binding.FA_OK   # empty: no-op
+    assert call(la=0) == binding.FA_ERR_INVALID_ARG
+    assert call(op=0) == binding.FA_ERR_INVALID_ARG
+    assert call(oa=O_acc + 8) == binding.FA_ERR_INVALID_ARG    # misaligned
+    assert call(lp=L_p + 2) == binding.FA_ERR_INVALID_ARG
+    assert call(d=96) == binding.FA_ERR_UNSUPPORTED
+    assert call(op=O_acc + 64) == binding.FA_ERR_INVALID_ARG   # accumulator overlaps part
+    assert call(oo=O_acc) == binding.FA_ERR_INVALID_ARG        # output overlaps accumulator
+    assert call(oo=0) != binding.FA_ERR_INVALID_ARG            # no bf16 output is fine
