@@ -47,6 +47,7 @@ SIGNATURES = {
     "fa_bwd_f32": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp,
                     _sz, _vp], _i),
     "fa_merge": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp], _i),
+    "fa_accumulate": ([_vp, _vp, _vp, _sz, _vp], _i),
     "fa_bwd_noalloc": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i,
                         _vp], _i),
     "fa_bwd_noalloc_max_scratch_bytes": ([], _sz),
@@ -334,6 +335,26 @@ def merge(O_acc: torch.Tensor, LSE_acc: torch.Tensor, O_part: torch.Tensor,
                             _ptr(O_out), B, H, N, d, _stream_handle(stream))
     _check("fa_merge", st)
     return O_acc, LSE_acc
+
+
+def accumulate(acc: torch.Tensor, part: torch.Tensor, out: Optional[torch.Tensor] = None,
+               stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """acc += part (float32 += bf16, same shape, contiguous) through ``fa_accumulate``;
+    ``out``, if given, receives acc rounded to bf16.  Returns acc."""
+    if acc.dtype != torch.float32 or part.dtype != torch.bfloat16:
+        raise ValueError("acc must be float32 and part bfloat16")
+    if acc.shape != part.shape or (out is not None and out.shape != acc.shape):
+        raise ValueError("acc, part and out must have the same shape")
+    for name, t in (("acc", acc), ("part", part), ("out", out)):
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if out is not None and out.dtype != torch.bfloat16:
+        raise ValueError("out must be bfloat16")
+    with torch.cuda.device(acc.device):
+        st = lib().fa_accumulate(_ptr(acc), _ptr(part), _ptr(out), acc.numel(),
+                                 _stream_handle(stream))
+    _check("fa_accumulate", st)
+    return acc
 
 
 class trace_kernels:

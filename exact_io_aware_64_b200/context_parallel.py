@@ -1,5 +1,5 @@
-"""Context-parallel attention forward: the sequence split across ranks, key/value blocks
-passed around a ring, partial results merged.
+"""Context-parallel attention: the sequence split across ranks, key/value blocks passed
+around a ring, partial results merged (forward) and gradients accumulated (backward).
 
 Rank r of W holds tokens [r*L, (r+1)*L) of every sequence: its queries Q_r and its keys
 and values K_r, V_r ([B, H, L, d], bf16).  Over W steps each rank computes attention of
@@ -10,11 +10,19 @@ partial results).  Under causal masking a block from an earlier rank is visible 
 the rank's own block needs the causal mask, and blocks from later ranks are skipped
 (they are still forwarded).
 
+The backward walks the same ring.  ``fa_bwd`` on one key block, given the global O and
+LSE of the forward, yields exactly that block's share of the gradients (its
+probabilities are the global ones restricted to the block), so each rank adds its dQ
+share in float32 (``fa_accumulate``) and the block's dK and dV shares travel with the
+block, in float32 accumulators, until every rank has added its part; one more hop takes
+them home.
+
 The exchange is torch.distributed point-to-point (NCCL between GPUs): at every step the
 send of the current block to rank r+1 and the receive of the next one from rank r-1 are
-posted before the step's attention, so the transfer overlaps it.  This forward path is
-exercised on one GPU by ``blockwise_forward`` (the same blocks and merges without the
-exchange) and its exchange schedule with gloo ranks on CPU.
+posted before the step's attention, so the transfer overlaps it (in the backward the
+gradient accumulators follow once the step has added to them).  ``blockwise_forward``
+and ``blockwise_backward`` run the same blocks, merges and accumulations on one device
+without the exchange; the exchange schedule is tested with gloo ranks on CPU.
 """
 from __future__ import annotations
 
@@ -46,6 +54,16 @@ def _default_fwd():
 def _default_merge():
     from . import binding
     return binding.merge
+
+
+def _default_bwd():
+    from . import binding
+    return binding.bwd
+
+
+def _default_accumulate():
+    from . import binding
+    return binding.accumulate
 
 
 def _accumulator(q: torch.Tensor) -> Tuple[torch.Tensor, torch.Tensor]:
@@ -114,3 +132,83 @@ def ring_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool
         if i + 1 < world:
             cur_k, cur_v = nk, nv
     return O, LSE_acc
+
+
+def _to_bf16(acc: torch.Tensor, like: torch.Tensor, accumulate: Callable) -> torch.Tensor:
+    """acc rounded to like's dtype (a zero added through the accumulate call)."""
+    out = torch.empty(acc.shape, dtype=like.dtype, device=acc.device)
+    accumulate(acc, torch.zeros(acc.shape, dtype=like.dtype, device=acc.device), out=out)
+    return out
+
+
+def blockwise_backward(qs, ks, vs, Os, dOs, LSEs, causal: bool, scale: Optional[float] = None,
+                       bwd: Optional[Callable] = None, accumulate: Optional[Callable] = None):
+    """Every rank's gradients with all chunks at hand (lists indexed by rank): the ring's
+    block backwards and accumulations in the ring's order (step by step, and within a
+    step rank by rank, so each block's accumulators receive their shares in the order
+    the ring delivers them), without the exchange.  Os and LSEs are the forward's global
+    results.  Returns lists (dQ, dK, dV) indexed by rank, in the inputs' dtype."""
+    bwd = bwd or _default_bwd()
+    accumulate = accumulate or _default_accumulate()
+    world = len(qs)
+    dQ = [torch.zeros(q.shape, dtype=torch.float32, device=q.device) for q in qs]
+    dK = [torch.zeros(k.shape, dtype=torch.float32, device=k.device) for k in ks]
+    dV = [torch.zeros(v.shape, dtype=torch.float32, device=v.device) for v in vs]
+    plans = [_plan(r, world, causal)[0] for r in range(world)]
+    for i in range(world):
+        for r in range(world):
+            src, kind = plans[r][i]
+            if kind is None:
+                continue
+            gq, gk, gv = bwd(qs[r], ks[src], vs[src], Os[r], dOs[r], LSEs[r], scale=scale,
+                             causal=(kind == "causal"))
+            accumulate(dQ[r], gq)
+            accumulate(dK[src], gk)
+            accumulate(dV[src], gv)
+    return ([_to_bf16(a, qs[r], accumulate) for r, a in enumerate(dQ)],
+            [_to_bf16(a, ks[r], accumulate) for r, a in enumerate(dK)],
+            [_to_bf16(a, vs[r], accumulate) for r, a in enumerate(dV)])
+
+
+def ring_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, O: torch.Tensor,
+                  dO: torch.Tensor, LSE: torch.Tensor, causal: bool,
+                  scale: Optional[float] = None, group=None, bwd: Optional[Callable] = None,
+                  accumulate: Optional[Callable] = None):
+    """This rank's (dQ, dK, dV) for ``ring_forward``'s output: O and LSE are what it
+    returned, dO the gradient of O; every rank calls it with its own chunk."""
+    import torch.distributed as dist
+    bwd = bwd or _default_bwd()
+    accumulate = accumulate or _default_accumulate()
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    to_global = (lambda r: r) if group is None else (lambda r: dist.get_global_rank(group, r))
+    nxt, prv = to_global((rank + 1) % world), to_global((rank - 1) % world)
+    steps, _ = _plan(rank, world, causal)
+    dQ = torch.zeros(q.shape, dtype=torch.float32, device=q.device)
+    cur_k, cur_v = k.contiguous(), v.contiguous()
+    cur_dk = torch.zeros(k.shape, dtype=torch.float32, device=k.device)
+    cur_dv = torch.zeros(v.shape, dtype=torch.float32, device=v.device)
+    for i, (src, kind) in enumerate(steps):
+        kv_reqs = []
+        if i + 1 < world:
+            nk, nv = torch.empty_like(cur_k), torch.empty_like(cur_v)
+            kv_reqs = [dist.isend(cur_k, nxt, group=group), dist.isend(cur_v, nxt, group=group),
+                       dist.irecv(nk, prv, group=group), dist.irecv(nv, prv, group=group)]
+        if kind is not None:
+            gq, gk, gv = bwd(q, cur_k, cur_v, O, dO, LSE, scale=scale,
+                             causal=(kind == "causal"))
+            accumulate(dQ, gq)
+            accumulate(cur_dk, gk)
+            accumulate(cur_dv, gv)
+        # the block's gradient accumulators move on with it (after this step's share);
+        # after the last step they go home: the block held now belongs to rank + 1
+        ndk, ndv = torch.empty_like(cur_dk), torch.empty_like(cur_dv)
+        g_reqs = [dist.isend(cur_dk, nxt, group=group), dist.isend(cur_dv, nxt, group=group),
+                  dist.irecv(ndk, prv, group=group), dist.irecv(ndv, prv, group=group)]
+        for rq in kv_reqs + g_reqs:
+            rq.wait()
+        cur_dk, cur_dv = ndk, ndv
+        if i + 1 < world:
+            cur_k, cur_v = nk, nv
+    return _to_bf16(dQ, q, accumulate), _to_bf16(cur_dk, k, accumulate), \
+        _to_bf16(cur_dv, v, accumulate)

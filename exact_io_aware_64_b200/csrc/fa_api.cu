@@ -470,6 +470,26 @@ fa_status fa_merge(float* O_acc, float* LSE_acc, const void* O_part, const float
   return FA_OK;
 }
 
+fa_status fa_accumulate(float* acc, const void* part, void* out, size_t n,
+                        cudaStream_t stream) {
+  g_last_error[0] = '\0';
+  if (n == 0) return FA_OK;
+  if (n % 8 != 0) return fail(FA_ERR_INVALID_ARG, "n=%zu is not a multiple of 8", n);
+  if (n >= (size_t(1) << 40)) return fail(FA_ERR_INVALID_ARG, "n=%zu is too large", n);
+  FA_TRY(check_ptr(acc, "acc"));
+  FA_TRY(check_ptr(part, "part"));
+  if (out != nullptr) FA_TRY(check_ptr(out, "out"));
+  if (overlaps(acc, n * 4, part, n * 2) ||
+      (out != nullptr && (overlaps(out, n * 2, acc, n * 4) || overlaps(out, n * 2, part, n * 2))))
+    return fail(FA_ERR_INVALID_ARG, "acc, part and out must not overlap");
+  DeviceInfo dev;
+  FA_TRY(device_info(&dev));
+  const fa::Problem p = make_problem(1, 1, 1, 1, 64, 1.f, 0, dev);
+  cudaError_t e = fa::launch_accumulate(acc, part, out, static_cast<long long>(n), p, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "launching the accumulate kernel");
+  return FA_OK;
+}
+
 fa_status fa_check_device_error(cudaStream_t stream) {
   g_last_error[0] = '\0';
   cudaError_t e = cudaStreamSynchronize(stream);

@@ -70,4 +70,9 @@ cudaError_t launch_merge(float* O_acc, float* LSE_acc, const void* O_part,
                          const float* LSE_part, void* O_out, const Problem& p,
                          cudaStream_t stream);
 
+// acc[i] += part[i] (float32 += bf16) for n elements, n a multiple of 8; out[i] =
+// bf16(acc[i]) when out is not null.
+cudaError_t launch_accumulate(float* acc, const void* part, void* out, long long n,
+                              const Problem& p, cudaStream_t stream);
+
 }  // namespace fa

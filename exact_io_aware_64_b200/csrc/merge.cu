@@ -10,6 +10,9 @@
 //
 // Mapping: one warp per query row, each lane holding d / 32 consecutive elements; the
 // accumulator is float32 so that a chain of merges rounds to bf16 only once, at the end.
+//
+// The same file holds the float32 accumulation of gradients over key blocks that the
+// context-parallel backward needs (acc += part, with a final bf16 copy).
 #include <cmath>
 #include <cstdint>
 
@@ -81,6 +84,35 @@ __global__ void __launch_bounds__(kRowsPerBlock * 32)
   if (lane == 0) Lacc[row] = lnew;
 }
 
+// acc[i] += part[i] for n elements (float32 += bf16), 8 per thread with 16-byte loads of
+// the bf16 operand; out[i] = bf16(acc[i]) when out is given.  n is a multiple of 8.
+__global__ void __launch_bounds__(256)
+    accumulate_kernel(float* __restrict__ acc, const __nv_bfloat16* __restrict__ part,
+                      __nv_bfloat16* __restrict__ out, long long n8) {
+  const long long i = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x;
+  if (i >= n8) return;
+  const uint4 pv = reinterpret_cast<const uint4*>(part)[i];
+  float4* a4 = reinterpret_cast<float4*>(acc) + 2 * i;
+  float4 a0 = a4[0], a1 = a4[1];
+  const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&pv);
+  const float2 f0 = __bfloat1622float2(p2[0]), f1 = __bfloat1622float2(p2[1]);
+  const float2 f2 = __bfloat1622float2(p2[2]), f3 = __bfloat1622float2(p2[3]);
+  a0.x += f0.x, a0.y += f0.y, a0.z += f1.x, a0.w += f1.y;
+  a1.x += f2.x, a1.y += f2.y, a1.z += f3.x, a1.w += f3.y;
+  a4[0] = a0;
+  a4[1] = a1;
+  if (out != nullptr) {
+    uint4 o;
+    const __nv_bfloat162 o0 = __floats2bfloat162_rn(a0.x, a0.y), o1 = __floats2bfloat162_rn(a0.z, a0.w);
+    const __nv_bfloat162 o2 = __floats2bfloat162_rn(a1.x, a1.y), o3 = __floats2bfloat162_rn(a1.z, a1.w);
+    o.x = *reinterpret_cast<const uint32_t*>(&o0);
+    o.y = *reinterpret_cast<const uint32_t*>(&o1);
+    o.z = *reinterpret_cast<const uint32_t*>(&o2);
+    o.w = *reinterpret_cast<const uint32_t*>(&o3);
+    reinterpret_cast<uint4*>(out)[i] = o;
+  }
+}
+
 template <int D>
 cudaError_t launch_d(float* Oacc, float* Lacc, const void* Opart, const float* Lpart,
                      void* Oout, const Problem& p, cudaStream_t stream) {
@@ -96,6 +128,17 @@ cudaError_t launch_d(float* Oacc, float* Lacc, const void* Opart, const float* L
 }
 
 }  // namespace
+
+cudaError_t launch_accumulate(float* acc, const void* part, void* out, long long n,
+                              const Problem& p, cudaStream_t stream) {
+  const long long n8 = n / 8;
+  cudaError_t e = trace_mark(p, 0, stream);
+  if (e != cudaSuccess) return e;
+  accumulate_kernel<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, stream>>>(
+      acc, static_cast<const __nv_bfloat16*>(part), static_cast<__nv_bfloat16*>(out), n8);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  return trace_mark(p, 1, stream);
+}
 
 cudaError_t launch_merge(float* Oacc, float* Lacc, const void* Opart, const float* Lpart,
                          void* Oout, const Problem& p, cudaStream_t stream) {

@@ -220,6 +220,18 @@ FA_API fa_status fa_merge(float* O_acc, float* LSE_acc, const void* O_part,
                           cudaStream_t stream);
 
 /*
+ * Accumulate a bf16 partial result into float32: acc[i] += part[i] for i < n, and
+ * out[i] = bf16(acc[i]) when out is not NULL.  The context-parallel backward sums the
+ * gradient contributions of several key blocks with it (each block's dQ on the query's
+ * GPU, each block's dK and dV as the block travels around the ring).
+ *   acc  in/out: n float32;  part in: n bf16;  out: n bf16 or NULL
+ * n a multiple of 8; pointers 16-byte aligned and not overlapping; one kernel on
+ * `stream`.  n == 0 is a no-op.
+ */
+FA_API fa_status fa_accumulate(float* acc, const void* part, void* out, size_t n,
+                               cudaStream_t stream);
+
+/*
  * fa_bwd for callers that cannot allocate device memory (no counterpart on the pages:
  * it is a property of this library, not of the method).  Same arguments and result as
  * fa_bwd, without the workspace: the scratch is a fixed array inside the library,

@@ -213,3 +213,13 @@ def test_merge_validation(lib):
     assert call(op=O_acc + 64) == binding.FA_ERR_INVALID_ARG   # accumulator overlaps part
     assert call(oo=O_acc) == binding.FA_ERR_INVALID_ARG        # output overlaps accumulator
     assert call(oo=0) != binding.FA_ERR_INVALID_ARG            # no bf16 output is fine
+
+
+def test_accumulate_validation(lib):
+    acc, part, out = 0x100000, 0x200000, 0x300000
+    assert lib.fa_accumulate(0, 0, 0, 0, None) == binding.FA_OK          # n = 0: no-op
+    assert lib.fa_accumulate(acc, part, out, 12, None) == binding.FA_ERR_INVALID_ARG  # not /8
+    assert lib.fa_accumulate(0, part, out, 16, None) == binding.FA_ERR_INVALID_ARG
+    assert lib.fa_accumulate(acc + 4, part, out, 16, None) == binding.FA_ERR_INVALID_ARG
+    assert lib.fa_accumulate(acc, acc + 32, 0, 16, None) == binding.FA_ERR_INVALID_ARG  # overlap
+    assert lib.fa_accumulate(acc, part, acc + 16, 16, None) == binding.FA_ERR_INVALID_ARG

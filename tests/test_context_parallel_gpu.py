@@ -81,3 +81,42 @@ def test_blockwise_forward_every_rank(causal):
             sl = slice(r * L, (r + 1) * L)
             assert_bf16_close(to64(O[0, h]), refs[h][0][sl], f"rank {r} O h={h}")
             assert_lse_close(to64(LSE[0, h]), refs[h][1][sl], f"rank {r} LSE h={h}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_blockwise_backward_every_rank(causal):
+    """The emulated 4-rank ring's backward: block backwards with the global O and LSE,
+    accumulated in float32 in the ring's order, give the gradients of attention over the
+    whole sequence (with D formed from the bf16 output, as fa_bwd does)."""
+    from parity import assert_bf16_close_scaled
+    W, B, H, L, d = 4, 1, 2, 384, 128
+    ins = inputs.make_inputs(B, H, W * L, d, seed=64, with_dO=True)
+    q, k, v, do = (ins[n].cuda() for n in ("Q", "K", "V", "dO"))
+    chunks = lambda t: [t[:, :, s * L:(s + 1) * L].contiguous() for s in range(W)]  # noqa: E731
+    qs, ks, vs, dos = chunks(q), chunks(k), chunks(v), chunks(do)
+    scale = d ** -0.5
+    fw = [cp.blockwise_forward(qs[r], ks, vs, r, causal, scale=scale) for r in range(W)]
+    Os, LSEs = [f[0] for f in fw], [f[1] for f in fw]
+    dQs, dKs, dVs = cp.blockwise_backward(qs, ks, vs, Os, dos, LSEs, causal, scale=scale)
+    binding.check_device_error()
+    O_full = torch.cat(Os, dim=2)
+    for h in range(H):
+        ref = oracle.attention_bwd_head(to64(ins["Q"][0, h]), to64(ins["K"][0, h]),
+                                        to64(ins["V"][0, h]), to64(ins["dO"][0, h]), scale,
+                                        causal, O_given=to64(O_full[0, h]))
+        for r in range(W):
+            sl = slice(r * L, (r + 1) * L)
+            for got, rf, name in ((dQs[r], ref[0], "dQ"), (dKs[r], ref[1], "dK"),
+                                  (dVs[r], ref[2], "dV")):
+                assert_bf16_close_scaled(to64(got[0, h]), rf[sl], f"rank {r} {name} h={h}")
+
+
+def test_accumulate():
+    acc = torch.randn(1000, 8, device="cuda")
+    part = torch.randn(1000, 8, device="cuda").to(torch.bfloat16)
+    out = torch.empty(1000, 8, dtype=torch.bfloat16, device="cuda")
+    ref = acc.double() + part.double()
+    binding.accumulate(acc, part, out=out)
+    torch.cuda.synchronize()
+    assert torch.equal(acc, (ref).float())
+    assert torch.equal(out, acc.to(torch.bfloat16))
