@@ -272,6 +272,10 @@ def run_gpu(args, w):
 
     fwd_ms = span(0, 1)
     bwd_ms = span(2, 5) if with_bwd else 0.0
+    # per-step device time (first kernel start to last kernel end of each step)
+    per_step = sorted(m[0].elapsed_time(m[5 if with_bwd else 1]) for m in marks)
+    pct = statistics.quantiles(per_step, n=10) if len(per_step) > 1 else per_step * 9
+    step_pct = {"p10": pct[0], "p50": statistics.median(per_step), "p90": pct[-1]}
     f_fwd = traffic.fwd_flops(B, H, N, d, w.causal)
     f_bwd = traffic.bwd_flops(B, H, N, d, w.causal) if with_bwd else 0.0
     # per kernel: mean launch time and algorithmic work (FLOPs credited to that kernel,
@@ -408,7 +412,7 @@ def run_gpu(args, w):
                    "step": "fa_fwd + fa_bwd" if with_bwd else "fa_fwd",
                    "l2": "inputs larger than L2 (no flush)",
                    "parallelism": f"replicas x{world} (independent heads per GPU)"},
-        "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+        "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "step_ms_percentiles": step_pct,
         "fwd_tflops": f_fwd / (fwd_ms * 1e-3) / 1e12,
         "bwd_tflops": (f_bwd / (bwd_ms * 1e-3) / 1e12) if with_bwd else None,
         "roofline": {"kernel": dom_name, "bound": "tensor", "achieved": achieved,

@@ -48,6 +48,7 @@ SIGNATURES = {
                     _sz, _vp], _i),
     "fa_merge": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp], _i),
     "fa_accumulate": ([_vp, _vp, _vp, _sz, _vp], _i),
+    "fa_selftest_timeout": ([ctypes.c_longlong, _vp], _i),
     "fa_bwd_noalloc": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i,
                         _vp], _i),
     "fa_bwd_noalloc_max_scratch_bytes": ([], _sz),

@@ -490,6 +490,18 @@ fa_status fa_accumulate(float* acc, const void* part, void* out, size_t n,
   return FA_OK;
 }
 
+fa_status fa_selftest_timeout(long long limit_cycles, cudaStream_t stream) {
+  g_last_error[0] = '\0';
+  if (limit_cycles < 0 || limit_cycles > (1ll << 34))
+    return fail(FA_ERR_INVALID_ARG, "limit_cycles=%lld out of range (0 .. 2^34)", limit_cycles);
+  DeviceInfo dev;
+  FA_TRY(device_info(&dev));
+  const fa::Problem p = make_problem(1, 1, 1, 1, 64, 1.f, 0, dev);
+  cudaError_t e = fa::launch_timeout_probe(limit_cycles, p, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "launching the timeout probe");
+  return FA_OK;
+}
+
 fa_status fa_check_device_error(cudaStream_t stream) {
   g_last_error[0] = '\0';
   cudaError_t e = cudaStreamSynchronize(stream);

@@ -75,4 +75,9 @@ cudaError_t launch_merge(float* O_acc, float* LSE_acc, const void* O_part,
 cudaError_t launch_accumulate(float* acc, const void* part, void* out, long long n,
                               const Problem& p, cudaStream_t stream);
 
+// One warp waiting on an mbarrier nothing arrives on, giving up after limit_cycles with
+// the kernels' timeout error (a check of the failure path).
+cudaError_t launch_timeout_probe(long long limit_cycles, const Problem& p,
+                                 cudaStream_t stream);
+
 }  // namespace fa

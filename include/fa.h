@@ -275,6 +275,16 @@ FA_API const char* fa_status_string(fa_status status);
 FA_API const char* fa_last_error_message(void);
 
 /*
+ * Check of the failure path (no counterpart on the pages): launches one warp that waits
+ * on an mbarrier nothing arrives on, in the same bounded loop as the kernels' pipeline
+ * waits but giving up after limit_cycles SM cycles (0 .. 2^34; e.g. 2e7, about 10 ms).
+ * It then sets the timeout bit of the library's error word and returns, so the next
+ * fa_check_device_error reports FA_ERR_TIMEOUT and clears it; the CUDA context stays
+ * usable.  Asynchronous on `stream`.
+ */
+FA_API fa_status fa_selftest_timeout(long long limit_cycles, cudaStream_t stream);
+
+/*
  * Synchronises `stream`, then reports and clears the device-side error word that the
  * kernels set when a pipeline wait exceeds its time limit (FA_ERR_TIMEOUT) or when a
  * kernel finds its shared memory misaligned and skips its work (FA_ERR_CUDA), or

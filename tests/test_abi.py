@@ -223,3 +223,8 @@ def test_accumulate_validation(lib):
     assert lib.fa_accumulate(acc + 4, part, out, 16, None) == binding.FA_ERR_INVALID_ARG
     assert lib.fa_accumulate(acc, acc + 32, 0, 16, None) == binding.FA_ERR_INVALID_ARG  # overlap
     assert lib.fa_accumulate(acc, part, acc + 16, 16, None) == binding.FA_ERR_INVALID_ARG
+
+
+def test_selftest_timeout_validation(lib):
+    assert lib.fa_selftest_timeout(-1, None) == binding.FA_ERR_INVALID_ARG
+    assert lib.fa_selftest_timeout(1 << 35, None) == binding.FA_ERR_INVALID_ARG
