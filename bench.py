@@ -53,6 +53,12 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+KERNEL_NAMES_BF16 = ("fwd_sm100_kernel", "bwd_prep_kernel", "bwd_dkdv_kernel", "bwd_dq_kernel")
+KERNEL_NAMES_F32 = ("fwd_f32_kernel", "bwd_f32_prep_kernel", "bwd_f32_dkdv_kernel",
+                    "bwd_f32_dq_kernel")
+# float32 FMA on the CUDA cores: 148 SMs x 128 lanes x 2 FLOP per clock at 1965 MHz
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
 KERNEL_SOURCES = {
     "fwd_sm100_kernel": ("fwd_sm100.cu", "sm100.cuh"),
     "bwd_prep_kernel": ("bwd_sm100.cu", "sm100.cuh"),
@@ -222,8 +228,10 @@ def run_gpu(args, w):
     dev = torch.device("cuda", local)
     B, H, N, d = w.B, w.H, w.N, w.d
     with_bwd = not args.fwd_only
+    f32 = w.dtype == "f32"
     ins = fa_inputs.make_inputs(B, H, N, d, fa_dist.replica_seed(w.seed, info), sigma_qk=w.sigma_qk,
-                                sigma_v=w.sigma_v, with_dO=True, device=str(dev))
+                                sigma_v=w.sigma_v, with_dO=True, device=str(dev),
+                                dtype=torch.float32 if f32 else torch.bfloat16)
     q, k, v, do = ins["Q"], ins["K"], ins["V"], ins["dO"]
     O = torch.empty_like(q)
     LSE = torch.empty((B, H, N), device=dev, dtype=torch.float32)
@@ -280,13 +288,14 @@ def run_gpu(args, w):
     f_bwd = traffic.bwd_flops(B, H, N, d, w.causal) if with_bwd else 0.0
     # per kernel: mean launch time and algorithmic work (FLOPs credited to that kernel,
     # or bytes for the bandwidth-bound preparation)
-    kernels = {"fwd_sm100_kernel": {"ms": fwd_ms, "flops": f_fwd}}
+    kn = KERNEL_NAMES_F32 if f32 else KERNEL_NAMES_BF16
+    kernels = {kn[0]: {"ms": fwd_ms, "flops": f_fwd}}
     if with_bwd:
         half = 0.5 if w.causal else 1.0
-        kernels["bwd_prep_kernel"] = {"ms": span(2, 3),
-                                      "bytes": traffic.bwd_prep_bytes(B, H, N, d)}
-        kernels["bwd_dkdv_kernel"] = {"ms": span(3, 4), "flops": 8.0 * B * H * N * N * d * half}
-        kernels["bwd_dq_kernel"] = {"ms": span(4, 5), "flops": 2.0 * B * H * N * N * d * half}
+        kernels[kn[1]] = {"ms": span(2, 3),
+                          "bytes": traffic.bwd_prep_bytes(B, H, N, d, 4 if f32 else 2)}
+        kernels[kn[2]] = {"ms": span(3, 4), "flops": 8.0 * B * H * N * N * d * half}
+        kernels[kn[3]] = {"ms": span(4, 5), "flops": 2.0 * B * H * N * N * d * half}
     for kinfo in kernels.values():
         if "flops" in kinfo:
             kinfo["tflops"] = kinfo["flops"] / (kinfo["ms"] * 1e-3) / 1e12
@@ -402,11 +411,18 @@ def run_gpu(args, w):
     dom_name = max(kernels, key=lambda k: kernels[k]["ms"])
     dom = kernels[dom_name]
     peak = peaks.get("bf16_tflops_sustained" if args.sustained_peak else "bf16_tflops")
+    bound, peak_source = "tensor", (f"{peak_src} "
+                                    f"{'sustained' if args.sustained_peak else 'burst'} bf16")
+    if f32:
+        # the float32 path runs on the CUDA cores: nominal FMA rate at the maximum clock
+        peak, bound = FP32_ALU_TFLOPS, "alu"
+        peak_source = "derived: 148 SMs x 128 FP32 lanes x 2 FLOP x 1965 MHz"
     achieved = dom["tflops"]
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32" if f32 else "bf16",
         "data": "synthetic",
         "config": {"workload": w.name, "B": B, "H": H, "N": N, "d": d, "causal": w.causal,
                    "step": "fa_fwd + fa_bwd" if with_bwd else "fa_fwd",
@@ -415,11 +431,9 @@ def run_gpu(args, w):
         "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "step_ms_percentiles": step_pct,
         "fwd_tflops": f_fwd / (fwd_ms * 1e-3) / 1e12,
         "bwd_tflops": (f_bwd / (bwd_ms * 1e-3) / 1e12) if with_bwd else None,
-        "roofline": {"kernel": dom_name, "bound": "tensor", "achieved": achieved,
+        "roofline": {"kernel": dom_name, "bound": bound, "achieved": achieved,
                      "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                     "peak_source": f"{peak_src} "
-                                    f"{'sustained' if args.sustained_peak else 'burst'} bf16",
-                     "traffic": recorded_traffic(dom_name)},
+                     "peak_source": peak_source, "traffic": recorded_traffic(dom_name)},
         "kernels": kernels,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
@@ -561,8 +575,6 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     w = fa_inputs.WORKLOADS[args.workload]
-    if w.dtype != "bf16":
-        ap.error("the benchmark runs the bf16 path")
     if args.impl == "reference":
         return run_reference(args, w)
     if args.sweep:
