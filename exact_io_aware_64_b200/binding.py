@@ -36,6 +36,8 @@ SIGNATURES = {
     "fa_fwd_qk": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _vp], _i),
     "fa_fwd_varlen": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _vp],
                       _i),
+    "fa_fwd_packed": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _i,
+                       _vp], _i),
     "fa_fwd_f32": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp], _i),
     "fa_bwd_workspace_bytes": ([_i, _i, _i, _i], _sz),
     "fa_bwd": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _sz,
@@ -44,6 +46,8 @@ SIGNATURES = {
                    _sz, _vp], _i),
     "fa_bwd_varlen": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
                        _i, _f, _i, _vp, _sz, _vp], _i),
+    "fa_bwd_packed": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
+                       _i, _i, _i, _f, _i, _vp, _sz, _vp], _i),
     "fa_bwd_f32": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp,
                     _sz, _vp], _i),
     "fa_merge": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp], _i),
@@ -314,6 +318,88 @@ def bwd_varlen(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, O: torch.Tenso
                                  B, H, Nq, Nk, d, float(scale), int(bool(causal)),
                                  _ptr(workspace), ws_bytes, _stream_handle(stream))
     _check("fa_bwd_varlen", st)
+    return dQ, dK, dV
+
+
+def _check_packed(name: str, t: torch.Tensor, tokens: int, H: int, d: int) -> None:
+    _check_bhnd(name, t, (tokens, H, d), torch.bfloat16)
+
+
+def _check_cu(cu_q: torch.Tensor, cu_k: torch.Tensor, device) -> int:
+    for name, t in (("cu_seqlens_q", cu_q), ("cu_seqlens_k", cu_k)):
+        if not t.is_cuda or t.device != device or t.dtype != torch.int32 or t.dim() != 1 \
+                or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous int32 CUDA vector on the inputs' device")
+    if cu_q.numel() != cu_k.numel() or cu_q.numel() < 1:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both have B+1 entries")
+    return cu_q.numel() - 1
+
+
+def fwd_packed(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, cu_seqlens_q: torch.Tensor,
+               cu_seqlens_k: torch.Tensor, max_seqlen_q: int, max_seqlen_k: int,
+               scale: Optional[float] = None, causal: bool = False,
+               O: Optional[torch.Tensor] = None, LSE: Optional[torch.Tensor] = None,
+               stream: Optional[torch.cuda.Stream] = None):
+    """Forward over a packed batch through ``fa_fwd_packed``: Q [total_q, H, d], K and V
+    [total_k, H, d] (bf16), sequences delimited by the int32 start arrays (B+1 entries).
+    Returns (O [total_q, H, d], LSE [H, total_q])."""
+    total_q, H, d = Q.shape
+    total_k = K.shape[0]
+    _check_packed("Q", Q, total_q, H, d)
+    for name, t in (("K", K), ("V", V)):
+        _check_packed(name, t, total_k, H, d)
+    B = _check_cu(cu_seqlens_q, cu_seqlens_k, Q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    O = torch.zeros_like(Q) if O is None else O
+    LSE = torch.full((H, total_q), float("-inf"), device=Q.device) if LSE is None else LSE
+    _check_packed("O", O, total_q, H, d)
+    _check_bhnd("LSE", LSE, (H, total_q), torch.float32)
+    with torch.cuda.device(Q.device):
+        st = lib().fa_fwd_packed(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE),
+                                 _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), B, H, int(max_seqlen_q),
+                                 int(max_seqlen_k), total_q, total_k, d, float(scale),
+                                 int(bool(causal)), _stream_handle(stream))
+    _check("fa_fwd_packed", st)
+    return O, LSE
+
+
+def bwd_packed(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, O: torch.Tensor,
+               dO: torch.Tensor, LSE: torch.Tensor, cu_seqlens_q: torch.Tensor,
+               cu_seqlens_k: torch.Tensor, max_seqlen_q: int, max_seqlen_k: int,
+               scale: Optional[float] = None, causal: bool = False,
+               dQ: Optional[torch.Tensor] = None, dK: Optional[torch.Tensor] = None,
+               dV: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+               stream: Optional[torch.cuda.Stream] = None):
+    """Backward over a packed batch through ``fa_bwd_packed`` (the gradient of
+    ``fwd_packed`` with the same start arrays).  Returns (dQ, dK, dV)."""
+    total_q, H, d = Q.shape
+    total_k = K.shape[0]
+    for name, t in (("Q", Q), ("O", O), ("dO", dO)):
+        _check_packed(name, t, total_q, H, d)
+    for name, t in (("K", K), ("V", V)):
+        _check_packed(name, t, total_k, H, d)
+    _check_bhnd("LSE", LSE, (H, total_q), torch.float32)
+    B = _check_cu(cu_seqlens_q, cu_seqlens_k, Q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dQ = torch.zeros_like(Q) if dQ is None else dQ
+    dK = torch.zeros_like(K) if dK is None else dK
+    dV = torch.zeros_like(V) if dV is None else dV
+    _check_packed("dQ", dQ, total_q, H, d)
+    for name, t in (("dK", dK), ("dV", dV)):
+        _check_packed(name, t, total_k, H, d)
+    need = workspace_bytes(B, H, int(max_seqlen_q), d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), device=Q.device, dtype=torch.uint8)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    with torch.cuda.device(Q.device):
+        st = lib().fa_bwd_packed(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _ptr(LSE),
+                                 _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(cu_seqlens_q),
+                                 _ptr(cu_seqlens_k), B, H, int(max_seqlen_q), int(max_seqlen_k),
+                                 total_q, total_k, d, float(scale), int(bool(causal)),
+                                 _ptr(workspace), ws_bytes, _stream_handle(stream))
+    _check("fa_bwd_packed", st)
     return dQ, dK, dV
 
 

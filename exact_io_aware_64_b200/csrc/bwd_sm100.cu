@@ -84,6 +84,10 @@ struct BwdArgs {
   unsigned int* err;
   const int* seqlens_q;  // [B] per-sequence query rows, or null (all Nq)
   const int* seqlens_k;  // [B] per-sequence key rows, or null (all Nk)
+  const int* cu_q;       // packed layout: [B+1] first query token of each sequence, or null
+  const int* cu_k;       // packed layout: [B+1] first key token of each sequence
+  int total_q;           // packed layout: query tokens of all sequences
+  int total_k;
   int H;
   __nv_bfloat16* dQ;
   __nv_bfloat16* dK;
@@ -102,27 +106,54 @@ struct BwdArgs {
   float scale_log2;
 };
 
-// The lengths of head bh's sequence: (Nq, Nk), or its entries of seqlens_q / seqlens_k.
-// A length out of range sets kErrBadLength and skips the sequence: (0, 0).
-__device__ __forceinline__ void seq_lengths(const BwdArgs& a, int bh, int& lq, int& lk) {
+// Head bh's sequence: its query and key row counts (Nq, Nk, or its entries of
+// seqlens_q / seqlens_k, or the differences of cu_q / cu_k) and, in the packed layout,
+// its first query and key tokens (0 otherwise).  A sequence out of range sets
+// kErrBadLength and is skipped: (0, 0).
+__device__ __forceinline__ void seq_info(const BwdArgs& a, int bh, int& lq, int& lk, int& tq0,
+                                         int& tk0) {
   lq = a.Nq;
   lk = a.Nk;
-  if (a.seqlens_q == nullptr) return;
-  const int b = bh / a.H;
-  lq = a.seqlens_q[b];
-  lk = a.seqlens_k[b];
-  if (lq < 0 || lq > a.Nq || lk < 0 || lk > a.Nk || (a.causal && lq > lk)) {
+  tq0 = 0;
+  tk0 = 0;
+  bool bad = false;
+  if (a.cu_q != nullptr) {
+    const int b = bh / a.H;
+    tq0 = a.cu_q[b];
+    tk0 = a.cu_k[b];
+    lq = a.cu_q[b + 1] - tq0;
+    lk = a.cu_k[b + 1] - tk0;
+    bad = tq0 < 0 || tq0 + lq > a.total_q || tk0 < 0 || tk0 + lk > a.total_k;
+  } else if (a.seqlens_q != nullptr) {
+    const int b = bh / a.H;
+    lq = a.seqlens_q[b];
+    lk = a.seqlens_k[b];
+  } else {
+    return;
+  }
+  if (bad || lq < 0 || lq > a.Nq || lk < 0 || lk > a.Nk || (a.causal && lq > lk)) {
     atomicOr(a.err, kErrBadLength);
     lq = 0;
     lk = 0;
   }
 }
 
-// Query rows of head bh that hold data (the rest of the padded length is padding).
-__device__ __forceinline__ int row_limit(const BwdArgs& a, int bh) {
-  int lq, lk;
-  seq_lengths(a, bh, lq, lk);
-  return lq;
+// Element offset of row `row` of head bh in a query-side ([BH][Nq][d] or packed
+// [tokens][H][d]) tensor, t0 the sequence's first token in the packed layout.
+__device__ __forceinline__ size_t q_row_offset(const BwdArgs& a, int bh, int t0, int row,
+                                               int D) {
+  return a.cu_q != nullptr ? (static_cast<size_t>(t0 + row) * a.H + bh % a.H) * D
+                           : (static_cast<size_t>(bh) * a.Nq + row) * D;
+}
+__device__ __forceinline__ size_t k_row_offset(const BwdArgs& a, int bh, int t0, int row,
+                                               int D) {
+  return a.cu_q != nullptr ? (static_cast<size_t>(t0 + row) * a.H + bh % a.H) * D
+                           : (static_cast<size_t>(bh) * a.Nk + row) * D;
+}
+// Index of row `row` of head bh in LSE ([BH][Nq], or [H][total_q] when packed).
+__device__ __forceinline__ size_t lse_index(const BwdArgs& a, int bh, int t0, int row) {
+  return a.cu_q != nullptr ? static_cast<size_t>(bh % a.H) * a.total_q + t0 + row
+                           : static_cast<size_t>(bh) * a.Nq + row;
 }
 
 // ------------------------------------------------------------------ 1. preparation
@@ -139,7 +170,7 @@ __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(
     const __nv_bfloat16* __restrict__ O, const __nv_bfloat16* __restrict__ dO,
     const float* __restrict__ LSE, float* __restrict__ Dout, float* __restrict__ L2out,
     const BwdArgs a) {
-  const int BH = a.BH, N = a.Nq, Npad = a.Npad;
+  const int BH = a.BH, Npad = a.Npad;
   constexpr int kPer = D / 8;                         // threads per row (8 bf16 each)
   constexpr int kRowsPerPass = kPrepThreads / kPer;   // rows covered by one pass
   const int part = threadIdx.x % kPer;
@@ -154,8 +185,10 @@ __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(
     if (row >= total) continue;
     const int bh = static_cast<int>(row / Npad);
     const int r = static_cast<int>(row % Npad);
-    if (r < row_limit(a, bh)) {
-      const size_t off = (static_cast<size_t>(bh) * N + r) * D + part * 8;
+    int lq, lk, tq0, tk0;
+    seq_info(a, bh, lq, lk, tq0, tk0);
+    if (r < lq) {
+      const size_t off = q_row_offset(a, bh, tq0, r, D) + part * 8;
       const uint4 a = *reinterpret_cast<const uint4*>(O + off);
       const uint4 b = *reinterpret_cast<const uint4*>(dO + off);
       const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
@@ -177,9 +210,10 @@ __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(
     if (part == 0 && row < total) {
       const int bh = static_cast<int>(row / Npad);
       const int r = static_cast<int>(row % Npad);
+      int lq, lk, tq0, tk0;
+      seq_info(a, bh, lq, lk, tq0, tk0);
       Dout[row] = -acc[k];
-      L2out[row] = r < row_limit(a, bh) ? -LSE[static_cast<size_t>(bh) * N + r] * kLog2e
-                                        : -INFINITY;
+      L2out[row] = r < lq ? -LSE[lse_index(a, bh, tq0, r)] * kLog2e : -INFINITY;
     }
   }
 }
@@ -259,6 +293,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto wait_warp = [&](uint32_t b, uint32_t parity) -> bool {
     return __all_sync(0xffffffffu, mbar_wait(b, parity, abort_flag, args.err));
   };
+  // TMA coordinates of row `row` of head bh's queries (t0 = tq0) or keys (t0 = tk0):
+  // (row, head) in the [BH][N][d] maps, (head, first token + row) in the packed maps
+  const bool packed = args.cu_q != nullptr;
+  auto tma_y = [&](int bh, int row) { return packed ? bh % args.H : row; };
+  auto tma_z = [&](int bh, int t0, int row) { return packed ? t0 + row : bh; };
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -293,7 +332,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // unit w: key tile j of head bh, meeting query tiles i0 .. i0 + m - 1 of its sequence
   // (m = 0: the tile lies past the sequence's keys, or the sequence has no queries)
-  auto unit = [&](int w, int& bh, int& j, int& i0, int& m, int& lk, int& off) {
+  auto unit = [&](int w, int& bh, int& j, int& i0, int& m, int& lk, int& off, int& tq0,
+                  int& tk0) {
     if (args.causal) {
       j = w / args.BH;  // key tile 0 meets every query tile: heaviest first
       bh = w % args.BH;
@@ -302,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       j = w % args.n_kt;
     }
     int lq;
-    seq_lengths(args, bh, lq, lk);
+    seq_info(args, bh, lq, lk, tq0, tk0);
     off = lk - lq;  // position of query row 0 among the keys
     i0 = 0;
     if (j * kTile >= lk || lq == 0) {
@@ -327,16 +367,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     int live = 0;  // 1 when the unit just processed had work: units counts only those
     for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
          w = snake_unit(++r), units += live) {
-      int bh, j, i0, m, lk, off;
-      unit(w, bh, j, i0, m, lk, off);
+      int bh, j, i0, m, lk, off, tq0, tk0;
+      unit(w, bh, j, i0, m, lk, off, tq0, tk0);
       live = m > 0;
       if (!live) continue;
       if (units > 0) ok = wait_warp(bar(L::kBarKVEmpty), (units - 1) & 1);
       if (!ok) break;
       mbar_arrive_expect_tx_elect(bar(L::kBarKVFull), 2 * L::kTileBytes);
       for (int c = 0; c < D / 64; ++c) {
-        tma_load_3d_elect(base + L::kK + c * L::kBoxBytes, &tmK, bar(L::kBarKVFull), c * 64, j * kTile, bh);
-        tma_load_3d_elect(base + L::kV + c * L::kBoxBytes, &tmV, bar(L::kBarKVFull), c * 64, j * kTile, bh);
+        tma_load_3d_elect(base + L::kK + c * L::kBoxBytes, &tmK, bar(L::kBarKVFull), c * 64,
+                          tma_y(bh, j * kTile), tma_z(bh, tk0, j * kTile));
+        tma_load_3d_elect(base + L::kV + c * L::kBoxBytes, &tmV, bar(L::kBarKVFull), c * 64,
+                          tma_y(bh, j * kTile), tma_z(bh, tk0, j * kTile));
       }
       ++kv_loads;
       for (int i = i0; ok && i < i0 + m; ++i) {
@@ -345,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx_elect(bar(L::kBarQFull + qs), L::kTileBytes);
         for (int c = 0; c < D / 64; ++c)
           tma_load_3d_elect(qslot(qs) + c * L::kBoxBytes, &tmQ, bar(L::kBarQFull + qs), c * 64,
-                            i * kTile, bh);
+                            tma_y(bh, i * kTile), tma_z(bh, tq0, i * kTile));
         q_issued[qs] = 1;
         q_phase[qs] = qph;
         if (++qs == L::kQStages) qs = 0, qph ^= 1;
@@ -354,7 +396,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t fb = bar(L::kBarDOFull + ds);
         mbar_arrive_expect_tx_elect(fb, L::kTileBytes + 1024);
         for (int c = 0; c < D / 64; ++c)
-          tma_load_3d_elect(doslot(ds) + c * L::kBoxBytes, &tmdO, fb, c * 64, i * kTile, bh);
+          tma_load_3d_elect(doslot(ds) + c * L::kBoxBytes, &tmdO, fb, c * 64,
+                            tma_y(bh, i * kTile), tma_z(bh, tq0, i * kTile));
         tma_load_3d_elect(doslot(ds) + L::kSlotL, &tmL2, fb, i * kTile, bh, 0);
         tma_load_3d_elect(doslot(ds) + L::kSlotD, &tmD, fb, i * kTile, bh, 0);
         d_issued[ds] = 1;
@@ -421,8 +464,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int live = 0;
     for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
          w = snake_unit(++r), units += live) {
-      int bh, j, i0, m, lk, off;
-      unit(w, bh, j, i0, m, lk, off);
+      int bh, j, i0, m, lk, off, tq0, tk0;
+      unit(w, bh, j, i0, m, lk, off, tq0, tk0);
       live = m > 0;
       if (!live) continue;
       ok = wait_warp(bar(L::kBarKVFull), units & 1);
@@ -474,8 +517,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int live = 0;
     for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
          w = snake_unit(++r), units += live) {
-      int bh, j, i0, m, lk, off;
-      unit(w, bh, j, i0, m, lk, off);
+      int bh, j, i0, m, lk, off, tq0, tk0;
+      unit(w, bh, j, i0, m, lk, off, tq0, tk0);
       live = m > 0;
       if (!live) continue;
       for (int i = i0; i < i0 + m; ++i) {
@@ -559,7 +602,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const int kv_row = j * kTile + row;
-      const size_t orow = (static_cast<size_t>(bh) * args.Nk + kv_row) * D;
+      const size_t orow = k_row_offset(args, bh, tk0, kv_row, D);
 #pragma unroll 1
       for (int c = g * (D / 64); c < (g + 1) * (D / 64); ++c) {
         uint32_t v[32];
@@ -640,6 +683,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto wait_warp = [&](uint32_t b, uint32_t parity) -> bool {
     return __all_sync(0xffffffffu, mbar_wait(b, parity, abort_flag, args.err));
   };
+  // TMA coordinates of row `row` of head bh's queries (t0 = tq0) or keys (t0 = tk0):
+  // (row, head) in the [BH][N][d] maps, (head, first token + row) in the packed maps
+  const bool packed = args.cu_q != nullptr;
+  auto tma_y = [&](int bh, int row) { return packed ? bh % args.H : row; };
+  auto tma_z = [&](int bh, int t0, int row) { return packed ? t0 + row : bh; };
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -678,7 +726,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // unit w: query tile i of head bh, meeting key tiles 0 .. m - 1 of its sequence
   // (m = 0: the tile lies past the sequence's queries, or the sequence has no keys)
-  auto unit = [&](int w, int& bh, int& i, int& m, int& lq, int& lk, int& off) {
+  auto unit = [&](int w, int& bh, int& i, int& m, int& lq, int& lk, int& off, int& tq0,
+                  int& tk0) {
     if (args.causal) {
       i = args.n_qt - 1 - w / args.BH;  // last query tile meets the most key tiles
       bh = w % args.BH;
@@ -686,7 +735,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bh = w / args.n_qt;
       i = w % args.n_qt;
     }
-    seq_lengths(args, bh, lq, lk);
+    seq_info(args, bh, lq, lk, tq0, tk0);
     off = lk - lq;
     if (i * kTile >= lq || lk == 0) {
       m = 0;
@@ -709,16 +758,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       int live = 0;  // 1 when the unit just processed had work: units counts only those
       for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
          w = snake_unit(++r), units += live) {
-        int bh, i, m, lq, lk, off;
-        unit(w, bh, i, m, lq, lk, off);
+        int bh, i, m, lq, lk, off, tq0, tk0;
+        unit(w, bh, i, m, lq, lk, off, tq0, tk0);
         live = m > 0;
         if (!live) continue;
         if (units > 0) ok = wait_warp(bar(L::kBarQEmpty), (units - 1) & 1);
         if (!ok) break;
         mbar_arrive_expect_tx_elect(bar(L::kBarQFull), 2 * L::kTileBytes);
         for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d_elect(base + L::kQ + c * L::kBoxBytes, &tmQ, bar(L::kBarQFull), c * 64, i * kTile, bh);
-          tma_load_3d_elect(base + L::kDO + c * L::kBoxBytes, &tmdO, bar(L::kBarQFull), c * 64, i * kTile, bh);
+          tma_load_3d_elect(base + L::kQ + c * L::kBoxBytes, &tmQ, bar(L::kBarQFull), c * 64,
+                            tma_y(bh, i * kTile), tma_z(bh, tq0, i * kTile));
+          tma_load_3d_elect(base + L::kDO + c * L::kBoxBytes, &tmdO, bar(L::kBarQFull), c * 64,
+                            tma_y(bh, i * kTile), tma_z(bh, tq0, i * kTile));
         }
         ++q_loads;
         for (int j = 0; ok && j < m; ++j) {
@@ -727,7 +778,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx_elect(bar(L::kBarKFull + ks), L::kTileBytes);
           for (int c = 0; c < D / 64; ++c)
             tma_load_3d_elect(base + L::kK0 + ks * L::kTileBytes + c * L::kBoxBytes, &tmK,
-                              bar(L::kBarKFull + ks), c * 64, j * kTile, bh);
+                              bar(L::kBarKFull + ks), c * 64, tma_y(bh, j * kTile),
+                              tma_z(bh, tk0, j * kTile));
           k_issued[ks] = 1;
           k_phase[ks] = kph;
           if (++ks == L::kKStages) ks = 0, kph ^= 1;
@@ -736,7 +788,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx_elect(bar(L::kBarVFull + vs), L::kTileBytes);
           for (int c = 0; c < D / 64; ++c)
             tma_load_3d_elect(base + L::kV0 + vs * L::kTileBytes + c * L::kBoxBytes, &tmV,
-                              bar(L::kBarVFull + vs), c * 64, j * kTile, bh);
+                              bar(L::kBarVFull + vs), c * 64, tma_y(bh, j * kTile),
+                              tma_z(bh, tk0, j * kTile));
           v_issued[vs] = 1;
           v_phase[vs] = vph;
           if (++vs == L::kVStages) vs = 0, vph ^= 1;
@@ -787,8 +840,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int live = 0;
       for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
          w = snake_unit(++r), units += live) {
-        int bh, i, m, lq, lk, off;
-        unit(w, bh, i, m, lq, lk, off);
+        int bh, i, m, lq, lk, off, tq0, tk0;
+        unit(w, bh, i, m, lq, lk, off, tq0, tk0);
         live = m > 0;
         if (!live) continue;
         ok = wait_warp(bar(L::kBarQFull), units & 1);
@@ -860,8 +913,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int live = 0;
     for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
          w = snake_unit(++r), units += live) {
-      int bh, i, m, lq, lk, off;
-      unit(w, bh, i, m, lq, lk, off);
+      int bh, i, m, lq, lk, off, tq0, tk0;
+      unit(w, bh, i, m, lq, lk, off, tq0, tk0);
       live = m > 0;
       if (!live) continue;
       const int q_row = i * kTile + row;
@@ -939,7 +992,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const size_t orow = (static_cast<size_t>(bh) * args.Nq + q_row) * D;
+      const size_t orow = q_row_offset(args, bh, tq0, q_row, D);
 #pragma unroll 1
       for (int c = g * (D / 64); c < (g + 1) * (D / 64); ++c) {
         uint32_t v[32];
@@ -974,6 +1027,10 @@ cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUten
   a.BH = p.BH;
   a.seqlens_q = p.seqlens_q;
   a.seqlens_k = p.seqlens_k;
+  a.cu_q = p.cu_q;
+  a.cu_k = p.cu_k;
+  a.total_q = p.total_q;
+  a.total_k = p.total_k;
   a.H = p.H;
   a.Nq = p.N;
   a.Nk = p.Nk;

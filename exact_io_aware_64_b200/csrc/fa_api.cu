@@ -113,6 +113,26 @@ fa_status make_tmap(CUtensorMap* tm, const void* ptr, int BH, int N, int d) {
   return FA_OK;
 }
 
+// Packed [tokens][H][d] bf16 viewed as a 3-D tensor {d, H, tokens}; boxes of 64
+// elements x 1 head x 128 tokens, which land in shared memory exactly like the 64 x 128
+// boxes above (128 rows of 128 bytes, 128-byte swizzle).  Tokens past the end read as
+// zeros.
+fa_status make_tmap_packed(CUtensorMap* tm, const void* ptr, int tokens, int H, int d) {
+  auto fn = encode_fn();
+  if (!fn) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(tokens)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                           static_cast<cuuint64_t>(H) * static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return FA_OK;
+}
+
 // [BH][rows] float32 (a per-row statistic padded to whole tiles) viewed as a 3-D tensor
 // [1][BH][rows] with boxes of 128 rows, no swizzle.
 fa_status make_row_tmap(CUtensorMap* tm, const float* ptr, int BH, int rows) {
@@ -245,8 +265,13 @@ fa_status check_bwd_args(const void* Q, const void* K, const void* V, const void
 
 fa::Problem make_problem(int B, int H, int Nq, int Nk, int d, float scale, int causal,
                          const DeviceInfo& dev, const int* seqlens_q = nullptr,
-                         const int* seqlens_k = nullptr) {
+                         const int* seqlens_k = nullptr, const int* cu_q = nullptr,
+                         const int* cu_k = nullptr, int total_q = 0, int total_k = 0) {
   fa::Problem p{};
+  p.cu_q = cu_q;
+  p.cu_k = cu_k;
+  p.total_q = total_q;
+  p.total_k = total_k;
   p.BH = B * H;
   p.N = Nq;
   p.Nk = Nk;
@@ -322,6 +347,26 @@ fa_status bwd_impl(const void* Q, const void* K, const void* V, const void* O, c
   return FA_OK;
 }
 
+// Checks of the packed-layout calls: lengths, totals and the start-token arrays.
+fa_status check_packed(const int* cu_q, const int* cu_k, int B, int H, int max_q, int max_k,
+                       int total_q, int total_k, int d, float scale, int causal, bool* noop) {
+  FA_TRY(check_common(B, H, max_q, max_k, d, scale, causal, noop));
+  if (total_q < 0 || total_k < 0)
+    return fail(FA_ERR_INVALID_ARG, "token totals must be non-negative");
+  const long long h = H;
+  if (h * total_q >= (1ll << 31) || h * total_k >= (1ll << 31))
+    return fail(FA_ERR_INVALID_ARG, "H * tokens is too large");
+  if (*noop || total_q == 0) {
+    *noop = true;
+    return FA_OK;
+  }
+  if (cu_q == nullptr || cu_k == nullptr)
+    return fail(FA_ERR_INVALID_ARG, "cu_seqlens_q and cu_seqlens_k are required");
+  if ((reinterpret_cast<uintptr_t>(cu_q) | reinterpret_cast<uintptr_t>(cu_k)) & 3u)
+    return fail(FA_ERR_INVALID_ARG, "cu_seqlens_q and cu_seqlens_k must be 4-byte aligned");
+  return FA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -369,6 +414,104 @@ fa_status fa_fwd_varlen(const void* Q, const void* K, const void* V, void* O, fl
   if (B > 0 && H > 0 && Nq > 0) FA_TRY(check_seqlens(seqlens_q, seqlens_k));
   return fwd_impl(Q, K, V, O, LSE, B, H, Nq, Nk, d, scale, causal, stream, seqlens_q,
                   seqlens_k);
+}
+
+fa_status fa_fwd_packed(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                        const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int H,
+                        int max_seqlen_q, int max_seqlen_k, int total_q, int total_k, int d,
+                        float scale, int causal, cudaStream_t stream) {
+  g_last_error[0] = '\0';
+  bool noop = false;
+  FA_TRY(check_packed(cu_seqlens_q, cu_seqlens_k, B, H, max_seqlen_q, max_seqlen_k, total_q,
+                      total_k, d, scale, causal, &noop));
+  if (noop) return FA_OK;
+  FA_TRY(check_ptr(Q, "Q"));
+  FA_TRY(check_ptr(K, "K"));
+  FA_TRY(check_ptr(V, "V"));
+  FA_TRY(check_ptr(O, "O"));
+  if (LSE != nullptr && (reinterpret_cast<uintptr_t>(LSE) & 3u))
+    return fail(FA_ERR_INVALID_ARG, "LSE is not 4-byte aligned");
+  const size_t qb = static_cast<size_t>(total_q) * H * d * 2;
+  const size_t kb = static_cast<size_t>(total_k) * H * d * 2;
+  if (overlaps(O, qb, Q, qb) || overlaps(O, qb, K, kb) || overlaps(O, qb, V, kb))
+    return fail(FA_ERR_INVALID_ARG, "O overlaps an input");
+  DeviceInfo dev;
+  FA_TRY(device_info(&dev));
+  FA_TRY(require_sm100(dev));
+  CUtensorMap tmQ, tmK, tmV;
+  FA_TRY(make_tmap_packed(&tmQ, Q, total_q, H, d));
+  FA_TRY(make_tmap_packed(&tmK, K, total_k, H, d));
+  FA_TRY(make_tmap_packed(&tmV, V, total_k, H, d));
+  const fa::Problem p = make_problem(B, H, max_seqlen_q, max_seqlen_k, d, scale, causal, dev,
+                                     nullptr, nullptr, cu_seqlens_q, cu_seqlens_k, total_q,
+                                     total_k);
+  cudaError_t e = fa::launch_fwd_sm100(tmQ, tmK, tmV, O, LSE, p, dev.num_sms, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "launching the forward kernel");
+  return FA_OK;
+}
+
+fa_status fa_bwd_packed(const void* Q, const void* K, const void* V, const void* O,
+                        const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                        const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int H,
+                        int max_seqlen_q, int max_seqlen_k, int total_q, int total_k, int d,
+                        float scale, int causal, void* workspace, size_t workspace_bytes,
+                        cudaStream_t stream) {
+  g_last_error[0] = '\0';
+  bool noop = false;
+  FA_TRY(check_packed(cu_seqlens_q, cu_seqlens_k, B, H, max_seqlen_q, max_seqlen_k, total_q,
+                      total_k, d, scale, causal, &noop));
+  if (noop) return FA_OK;
+  FA_TRY(check_ptr(Q, "Q"));
+  FA_TRY(check_ptr(K, "K"));
+  FA_TRY(check_ptr(V, "V"));
+  FA_TRY(check_ptr(O, "O"));
+  FA_TRY(check_ptr(dO, "dO"));
+  FA_TRY(check_ptr(LSE, "LSE"));
+  FA_TRY(check_ptr(dQ, "dQ"));
+  FA_TRY(check_ptr(dK, "dK"));
+  FA_TRY(check_ptr(dV, "dV"));
+  const size_t need = fa_bwd_workspace_bytes(B, H, max_seqlen_q, d);
+  FA_TRY(check_ptr(workspace, "workspace"));
+  if (workspace_bytes < need)
+    return fail(FA_ERR_INVALID_ARG, "workspace has %zu bytes, %zu needed", workspace_bytes,
+                need);
+  const size_t qb = static_cast<size_t>(total_q) * H * d * 2;
+  const size_t kb = static_cast<size_t>(total_k) * H * d * 2;
+  struct Buf {
+    const void* p;
+    size_t n;
+  };
+  const Buf ins[5] = {{Q, qb}, {K, kb}, {V, kb}, {O, qb}, {dO, qb}};
+  const Buf outs[3] = {{dQ, qb}, {dK, kb}, {dV, kb}};
+  for (const Buf& o : outs) {
+    for (const Buf& in : ins)
+      if (overlaps(o.p, o.n, in.p, in.n))
+        return fail(FA_ERR_INVALID_ARG, "a gradient overlaps an input");
+    if (overlaps(o.p, o.n, workspace, need))
+      return fail(FA_ERR_INVALID_ARG, "a gradient overlaps the workspace");
+  }
+  if (overlaps(dQ, qb, dK, kb) || overlaps(dQ, qb, dV, kb) || overlaps(dK, kb, dV, kb))
+    return fail(FA_ERR_INVALID_ARG, "gradients overlap each other");
+  DeviceInfo dev;
+  FA_TRY(device_info(&dev));
+  FA_TRY(require_sm100(dev));
+  const int BH = B * H;
+  CUtensorMap tmQ, tmK, tmV, tmdO, tmL2, tmD;
+  FA_TRY(make_tmap_packed(&tmQ, Q, total_q, H, d));
+  FA_TRY(make_tmap_packed(&tmK, K, total_k, H, d));
+  FA_TRY(make_tmap_packed(&tmV, V, total_k, H, d));
+  FA_TRY(make_tmap_packed(&tmdO, dO, total_q, H, d));
+  const int Npad = fa::bwd_padded_rows(max_seqlen_q);
+  float* ws = static_cast<float*>(workspace);
+  FA_TRY(make_row_tmap(&tmD, ws, BH, Npad));
+  FA_TRY(make_row_tmap(&tmL2, ws + static_cast<size_t>(BH) * Npad, BH, Npad));
+  const fa::Problem p = make_problem(B, H, max_seqlen_q, max_seqlen_k, d, scale, causal, dev,
+                                     nullptr, nullptr, cu_seqlens_q, cu_seqlens_k, total_q,
+                                     total_k);
+  cudaError_t e = fa::launch_bwd_sm100(tmQ, tmK, tmV, tmdO, tmL2, tmD, O, dO, LSE, dQ, dK, dV,
+                                       ws, p, dev.num_sms, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "launching the backward kernels");
+  return FA_OK;
 }
 
 fa_status fa_fwd_f32(const float* Q, const float* K, const float* V, float* O, float* LSE,

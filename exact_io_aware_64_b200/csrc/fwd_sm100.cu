@@ -42,6 +42,10 @@
 //     sequence b uses its first seqlens_q[b] query and seqlens_k[b] key rows, with the
 //     same alignment rule; units past a sequence's queries have no work and every role
 //     skips them.  Key rows past a sequence's length are masked like a ragged tail.
+//   * Packed layout: tensors [tokens, H, d] with sequence b's tokens from cu_q[b] (keys
+//     cu_k[b]); the tensor maps address (column, head, token), so a tile is 128 tokens of
+//     one head from the sequence's first token on.  Tile rows past the sequence hold the
+//     next sequence's tokens: masked as keys, not stored as queries.
 #include <cfloat>
 #include <cstdint>
 
@@ -103,6 +107,10 @@ struct FwdArgs {
   float* LSE;
   const int* seqlens_q;  // [B] per-sequence query rows, or null (all Nq)
   const int* seqlens_k;  // [B] per-sequence key rows, or null (all Nk)
+  const int* cu_q;       // packed layout: [B+1] first query token of each sequence, or null
+  const int* cu_k;       // packed layout: [B+1] first key token of each sequence
+  int total_q;           // packed layout: query tokens of all sequences
+  int total_k;
   int H;
   int BH;
   int Nq;           // query rows per head (padded length with seqlens)
@@ -116,6 +124,7 @@ struct FwdArgs {
 struct UnitInfo {
   int bh, u, n0, n1;  // n_t: key tiles of query tile t (0: no work)
   int lq, lk, off;    // the sequence's query rows, key rows, position of query row 0
+  int h, tq0, tk0;    // head; packed layout: the sequence's first query and key token
 };
 
 __device__ __forceinline__ UnitInfo unit_info(int w, const FwdArgs& a) {
@@ -130,7 +139,22 @@ __device__ __forceinline__ UnitInfo unit_info(int w, const FwdArgs& a) {
   }
   r.lq = a.Nq;
   r.lk = a.Nk;
-  if (a.seqlens_q != nullptr) {
+  r.h = r.bh % a.H;
+  r.tq0 = 0;
+  r.tk0 = 0;
+  if (a.cu_q != nullptr) {
+    const int b = r.bh / a.H;
+    r.tq0 = a.cu_q[b];
+    r.tk0 = a.cu_k[b];
+    r.lq = a.cu_q[b + 1] - r.tq0;
+    r.lk = a.cu_k[b + 1] - r.tk0;
+    if (r.tq0 < 0 || r.lq < 0 || r.lq > a.Nq || r.tq0 + r.lq > a.total_q || r.tk0 < 0 ||
+        r.lk < 0 || r.lk > a.Nk || r.tk0 + r.lk > a.total_k || (a.causal && r.lq > r.lk)) {
+      if (threadIdx.x == 0) atomicOr(a.err, kErrBadLength);
+      r.lq = 0;  // the sequence is skipped
+      r.lk = 0;
+    }
+  } else if (a.seqlens_q != nullptr) {
     const int b = r.bh / a.H;
     r.lq = a.seqlens_q[b];
     r.lk = a.seqlens_k[b];
@@ -175,6 +199,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto wait_warp = [&](uint32_t b, uint32_t parity) -> bool {
     return __all_sync(0xffffffffu, mbar_wait(b, parity, abort_flag, args.err));
   };
+  // TMA coordinates of row `row` of a unit's queries (t0 = tq0) or keys (t0 = tk0):
+  // (row, head) in the [BH][N][d] maps, (head, first token + row) in the packed maps
+  const bool packed = args.cu_q != nullptr;
+  auto tma_y = [&](const UnitInfo& ui, int row) { return packed ? ui.h : row; };
+  auto tma_z = [&](const UnitInfo& ui, int t0, int row) { return packed ? t0 + row : ui.bh; };
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -235,7 +264,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx_elect(qb, L::kTileBytes);
           const uint32_t dst = base + (t == 0 ? L::kQ0 : L::kQ1);
           for (int c = 0; c < D / 64; ++c)
-            tma_load_3d_elect(dst + c * L::kBoxBytes, &tmQ, qb, c * 64, (2 * ui.u + t) * kBM, ui.bh);
+            tma_load_3d_elect(dst + c * L::kBoxBytes, &tmQ, qb, c * 64,
+                              tma_y(ui, (2 * ui.u + t) * kBM), tma_z(ui, ui.tq0, (2 * ui.u + t) * kBM));
           ++q_uses[t];
         }
         const int n = max(ui.n0, ui.n1);
@@ -248,7 +278,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t dst = base + L::kRing + stage * L::kTileBytes;
             const CUtensorMap* tm = kv == 0 ? &tmK : &tmV;
             for (int c = 0; c < D / 64; ++c)
-              tma_load_3d_elect(dst + c * L::kBoxBytes, tm, fb, c * 64, j * kBN, ui.bh);
+              tma_load_3d_elect(dst + c * L::kBoxBytes, tm, fb, c * 64, tma_y(ui, j * kBN),
+                                tma_z(ui, ui.tk0, j * kBN));
             issued[stage] = 1;
             issued_phase[stage] = phase;
             if (++stage == L::kStages) stage = 0, phase ^= 1;
@@ -477,7 +508,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const float inv_l = 1.f / l;
       const int bh = ui.bh;
-      __nv_bfloat16* orow = args.O + (static_cast<size_t>(bh) * args.Nq + q_row) * D;
+      __nv_bfloat16* orow =
+          args.O + (packed ? (static_cast<size_t>(ui.tq0 + q_row) * args.H + ui.h) * D
+                           : (static_cast<size_t>(bh) * args.Nq + q_row) * D);
       // take the whole O row into registers first, so the MMA warp may start the next
       // unit's first P V product while this row is being converted and stored
       uint32_t ov[D];
@@ -500,7 +533,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (args.LSE != nullptr && q_row < ui.lq)
-        args.LSE[static_cast<size_t>(bh) * args.Nq + q_row] =
+        args.LSE[packed ? static_cast<size_t>(ui.h) * args.total_q + ui.tq0 + q_row
+                        : static_cast<size_t>(bh) * args.Nq + q_row] =
             (m + __log2f(l)) * 0.69314718055994531f;
     }
   }
@@ -525,6 +559,10 @@ cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUten
   a.BH = p.BH;
   a.seqlens_q = p.seqlens_q;
   a.seqlens_k = p.seqlens_k;
+  a.cu_q = p.cu_q;
+  a.cu_k = p.cu_k;
+  a.total_q = p.total_q;
+  a.total_k = p.total_k;
   a.H = p.H;
   a.Nq = p.N;
   a.Nk = p.Nk;

@@ -24,6 +24,13 @@ struct Problem {
   const int* seqlens_q;
   const int* seqlens_k;
   int H;
+  // packed layout ([tokens, H, d] tensors, LSE [H, tokens]): per-sequence start tokens
+  // [B+1] on the device (both null otherwise) and the token totals; N and Nk are then
+  // the longest sequence's query and key counts
+  const int* cu_q;
+  const int* cu_k;
+  int total_q;
+  int total_k;
   // optional kernel-boundary events (fa_trace_events): trace[0] before the first kernel,
   // trace[k] after the k-th; n_trace entries
   cudaEvent_t* trace;

@@ -123,6 +123,29 @@ FA_API fa_status fa_fwd_varlen(const void* Q, const void* K, const void* V, void
                                cudaStream_t stream);
 
 /*
+ * Forward pass over a packed batch of sequences of different lengths (no counterpart on
+ * the pages; queries aligned with the end of their sequence's keys as in fa_fwd_qk).
+ * The tokens of all sequences are stored one after another, with no padding:
+ *   Q, O [total_q, H, d] bf16;  K, V [total_k, H, d] bf16;  LSE [H, total_q] float32
+ *     or NULL
+ *   cu_seqlens_q, cu_seqlens_k: device int32 arrays [B+1], 4-byte aligned, required;
+ *     sequence b has queries cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1 and keys
+ *     cu_seqlens_k[b] .. cu_seqlens_k[b+1]-1 (non-decreasing, ending at total_q and
+ *     total_k)
+ *   max_seqlen_q, max_seqlen_k: at least the longest sequence's query and key counts
+ *     (they size the work grid); causal needs max_seqlen_q <= max_seqlen_k and each
+ *     sequence's queries <= its keys.
+ * A sequence with no queries or no keys is skipped (its rows are not written).  The
+ * start arrays are read on the device: a sequence out of range is skipped and reported
+ * by fa_check_device_error as FA_ERR_INVALID_ARG.  Otherwise as fa_fwd_qk.
+ */
+FA_API fa_status fa_fwd_packed(const void* Q, const void* K, const void* V, void* O,
+                               float* LSE, const int* cu_seqlens_q, const int* cu_seqlens_k,
+                               int B, int H, int max_seqlen_q, int max_seqlen_k, int total_q,
+                               int total_k, int d, float scale, int causal,
+                               cudaStream_t stream);
+
+/*
  * Forward pass with float32 inputs and outputs, computed in float32 on the CUDA cores
  * (same definition and arguments as fa_fwd).
  */
@@ -181,6 +204,20 @@ FA_API fa_status fa_bwd_varlen(const void* Q, const void* K, const void* V, cons
                                int H, int Nq, int Nk, int d, float scale, int causal,
                                void* workspace, size_t workspace_bytes,
                                cudaStream_t stream);
+
+/*
+ * Backward pass over a packed batch (the gradient of fa_fwd_packed, same start arrays).
+ *   Q, O, dO, dQ [total_q, H, d] bf16;  K, V, dK, dV [total_k, H, d] bf16;
+ *   LSE [H, total_q] float32
+ *   workspace: fa_bwd_workspace_bytes(B, H, max_seqlen_q, d) bytes
+ * Otherwise as fa_bwd_varlen.
+ */
+FA_API fa_status fa_bwd_packed(const void* Q, const void* K, const void* V, const void* O,
+                               const void* dO, const float* LSE, void* dQ, void* dK,
+                               void* dV, const int* cu_seqlens_q, const int* cu_seqlens_k,
+                               int B, int H, int max_seqlen_q, int max_seqlen_k, int total_q,
+                               int total_k, int d, float scale, int causal, void* workspace,
+                               size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * Backward pass, float32: the same computation as fa_bwd with float32 inputs, outputs

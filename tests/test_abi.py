@@ -228,3 +228,22 @@ def test_accumulate_validation(lib):
 def test_selftest_timeout_validation(lib):
     assert lib.fa_selftest_timeout(-1, None) == binding.FA_ERR_INVALID_ARG
     assert lib.fa_selftest_timeout(1 << 35, None) == binding.FA_ERR_INVALID_ARG
+
+
+def test_packed_validation(lib):
+    CQ, CK = 0xB00000, 0xC00000
+
+    def fwd(cq=CQ, ck=CK, maxq=64, maxk=64, tq=100, tk=100, causal=1):
+        return lib.fa_fwd_packed(A, B_, C, D_, E, cq, ck, 2, 2, maxq, maxk, tq, tk, 64, 0.1,
+                                 causal, None)
+
+    assert fwd(tq=0, cq=0, ck=0) == binding.FA_OK             # no tokens: no-op
+    assert fwd(cq=0) == binding.FA_ERR_INVALID_ARG
+    assert fwd(ck=CK + 2) == binding.FA_ERR_INVALID_ARG       # misaligned
+    assert fwd(maxq=128, maxk=64) == binding.FA_ERR_INVALID_ARG  # causal: max_q <= max_k
+    assert fwd(tq=-1) == binding.FA_ERR_INVALID_ARG
+    F, G, H_, I, J = 0x600000, 0x700000, 0x800000, 0x900000, 0xA00000
+    need = binding.workspace_bytes(2, 2, 64, 64)
+    st = lib.fa_bwd_packed(A, B_, C, D_, E, F, G, H_, I, CQ, CK, 2, 2, 64, 64, 100, 100, 64,
+                           0.1, 1, J, need - 4, None)
+    assert st == binding.FA_ERR_INVALID_ARG                   # workspace too small
