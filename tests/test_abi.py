@@ -247,3 +247,25 @@ def test_packed_validation(lib):
     st = lib.fa_bwd_packed(A, B_, C, D_, E, F, G, H_, I, CQ, CK, 2, 2, 64, 64, 100, 100, 64,
                            0.1, 1, J, need - 4, None)
     assert st == binding.FA_ERR_INVALID_ARG                   # workspace too small
+
+
+def test_binding_refuses_host_tensors():
+    """No CPU fallback: every entry point of the binding rejects tensors that are not on a
+    CUDA device before anything is computed."""
+    import torch
+    q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
+    lse = torch.zeros(1, 1, 8)
+    with pytest.raises(ValueError, match="CUDA"):
+        binding.fwd(q, q, q)
+    with pytest.raises(ValueError, match="CUDA"):
+        binding.bwd(q, q, q, q, q, lse)
+    with pytest.raises(ValueError, match="CUDA"):
+        binding.bwd_noalloc(q, q, q, q, q, lse)
+    with pytest.raises(ValueError, match="CUDA"):
+        binding.fwd_packed(q[0, 0].unsqueeze(1), q[0, 0].unsqueeze(1), q[0, 0].unsqueeze(1),
+                           torch.zeros(2, dtype=torch.int32), torch.zeros(2, dtype=torch.int32),
+                           8, 8)
+    with pytest.raises(ValueError):
+        binding.merge(torch.zeros(1, 1, 8, 64), lse, q, lse)
+    with pytest.raises(ValueError):
+        binding.accumulate(torch.zeros(8), torch.zeros(8, dtype=torch.bfloat16))
