@@ -20,14 +20,19 @@
  * Layout and types
  *   Q, K, V, O, dO, dQ, dK, dV: [B, H, N, d] contiguous row-major (d fastest).  bf16 in
  *   the bf16 calls (__nv_bfloat16, passed as void*), float in the _f32 calls.
- *   LSE: [B, H, N] float32.  All pointers are device pointers.
+ *   LSE: [B, H, N] float32.  All pointers are device pointers.  The _qk calls take Nq
+ *   query rows and Nk key rows, the _varlen calls padded batches with per-sequence
+ *   lengths, the _packed calls [tokens, H, d] tensors delimited by start arrays; each
+ *   declaration below gives its shapes.
  *   Arithmetic: bf16 inputs, float32 accumulation and softmax statistics; the bf16 calls
  *   round the probabilities (and dS in the backward) to bf16 before the second matrix
  *   product.  The _f32 calls compute in float32 throughout.
  *
  * Ownership and asynchrony
  *   The caller allocates and owns every buffer.  The library allocates no device memory
- *   and keeps no per-call state; it reads the device's SM count once per device.  Each
+ *   and keeps no per-call state; it reads the device's SM count once per device.  (Its
+ *   only device data of its own are an error word and the fixed scratch array of
+ *   fa_bwd_noalloc, both part of the loaded module.)  Each
  *   call validates its arguments on the host, enqueues kernels on `stream` and returns;
  *   the results are ready when `stream` reaches that point.  A return of FA_OK says the
  *   launch was accepted; errors raised while the kernels run are reported by
