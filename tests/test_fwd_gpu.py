@@ -70,12 +70,13 @@ def test_bf16_many_units_per_cta(causal):
     _full_check(ins, 0.125, causal)
 
 
-def _rows_check(w, rows_per_head=256, full_heads=((0, 0),), check_lse=True):
+def _rows_check(w, rows_per_head=256, full_heads=((0, 0),), check_lse=True, extra_rows=()):
     ins = inputs.make_workload_inputs(w)
     O, LSE = _run(ins, w.scale, w.causal)
     Q, K, V = (to64(ins[n]) for n in ("Q", "K", "V"))
     O64, LSE64 = to64(O), to64(LSE)
-    rows = np.array(inputs.sample_rows(w.N, rows_per_head, seed=1234))
+    rows = np.array(sorted(set(inputs.sample_rows(w.N, rows_per_head, seed=1234)) |
+                           set(extra_rows)))
     for b in range(w.B):
         for h in range(w.H):
             Or, LSEr, _ = oracle.attention_head(Q[b, h, rows], K[b, h], V[b, h], w.scale,
@@ -97,13 +98,24 @@ def test_workload_n4096_d64(name):
 
 
 def test_workload_n10000_ragged_tail():
+    # 512 seeded rows per head, the tile boundaries and the ragged last tile (16 rows),
+    # in all 32 heads; one head in full
     w = inputs.WORKLOADS["n10000_d128_causal"]
-    _rows_check(w, rows_per_head=384, full_heads=((0, 31),))
+    _rows_check(w, rows_per_head=512, full_heads=((0, 31),))
 
 
 def test_workload_n32768_large_logits():
+    # 512 seeded rows per head plus the whole first and last 128-row tiles, all 8 heads,
+    # with LSE (a full 32K x 32K head is left to the row checks: each row is exact alone)
     w = inputs.WORKLOADS["n32768_d128_causal_sigma3"]
-    _rows_check(w, rows_per_head=384, full_heads=())
+    _rows_check(w, rows_per_head=512, full_heads=(), extra_rows=range(128))
+
+
+def test_workload_n8192_forward():
+    # the benchmark workload's forward: O and LSE on 256 seeded rows of every head and
+    # one head in full
+    w = inputs.WORKLOADS["n8192_d128_causal_bwd"]
+    _rows_check(w, rows_per_head=256, full_heads=((1, 7),))
 
 
 def test_deterministic_and_in_bounds():
