@@ -39,6 +39,11 @@ SIGNATURES = {
     "fa_fwd_packed": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _i,
                        _vp], _i),
     "fa_fwd_f32": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp], _i),
+    "fa_fwd_f32_qk": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _vp], _i),
+    "fa_fwd_f32_varlen": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i,
+                           _vp], _i),
+    "fa_fwd_f32_packed": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f,
+                           _i, _vp], _i),
     "fa_bwd_workspace_bytes": ([_i, _i, _i, _i], _sz),
     "fa_bwd": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _sz,
                 _vp], _i),
@@ -50,6 +55,12 @@ SIGNATURES = {
                        _i, _i, _i, _f, _i, _vp, _sz, _vp], _i),
     "fa_bwd_f32": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp,
                     _sz, _vp], _i),
+    "fa_bwd_f32_qk": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i,
+                       _vp, _sz, _vp], _i),
+    "fa_bwd_f32_varlen": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i,
+                           _i, _i, _f, _i, _vp, _sz, _vp], _i),
+    "fa_bwd_f32_packed": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i,
+                           _i, _i, _i, _i, _f, _i, _vp, _sz, _vp], _i),
     "fa_merge": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp], _i),
     "fa_accumulate": ([_vp, _vp, _vp, _sz, _vp], _i),
     "fa_selftest_timeout": ([ctypes.c_longlong, _vp], _i),
@@ -118,12 +129,12 @@ def fwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, scale: Optional[float
         causal: bool = False, O: Optional[torch.Tensor] = None,
         LSE: Optional[torch.Tensor] = None, want_lse: bool = True,
         stream: Optional[torch.cuda.Stream] = None):
-    """Exact attention forward through ``fa_fwd`` (bf16), ``fa_fwd_qk`` (bf16, fewer
-    queries than keys) or ``fa_fwd_f32`` (float32).
+    """Exact attention forward through ``fa_fwd`` / ``fa_fwd_qk`` (bf16; the latter when
+    Nq != Nk) or ``fa_fwd_f32`` / ``fa_fwd_f32_qk`` (float32).
 
     Q: [B, H, Nq, d]; K, V: [B, H, Nk, d]; CUDA tensors, contiguous, all bf16 or all
     float32.  With Nq != Nk the queries are the last Nq of the Nk tokens (causal masking
-    aligned at the bottom right); the float32 path takes Nq == Nk only.
+    aligned at the bottom right).
     Returns (O, LSE); LSE is None when ``want_lse`` is False and none is passed.
     """
     B, H, Nq, d = Q.shape
@@ -134,8 +145,6 @@ def fwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, scale: Optional[float
     _check_bhnd("Q", Q, (B, H, Nq, d), dtype)
     for name, t in (("K", K), ("V", V)):
         _check_bhnd(name, t, (B, H, Nk, d), dtype)
-    if dtype == torch.float32 and Nq != Nk:
-        raise ValueError("the float32 path takes as many queries as keys")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if O is None:
@@ -146,10 +155,15 @@ def fwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, scale: Optional[float
     if LSE is not None:
         _check_bhnd("LSE", LSE, (B, H, Nq), torch.float32)
     with torch.cuda.device(Q.device):
-        if dtype == torch.float32:
+        if dtype == torch.float32 and Nq == Nk:
             name = "fa_fwd_f32"
             st = lib().fa_fwd_f32(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), B, H, Nq, d,
                                   float(scale), int(bool(causal)), _stream_handle(stream))
+        elif dtype == torch.float32:
+            name = "fa_fwd_f32_qk"
+            st = lib().fa_fwd_f32_qk(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), B, H, Nq,
+                                     Nk, d, float(scale), int(bool(causal)),
+                                     _stream_handle(stream))
         elif Nq == Nk:
             name = "fa_fwd"
             st = lib().fa_fwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), B, H, Nq, d,
@@ -172,8 +186,8 @@ def bwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, O: torch.Tensor,
         dK: Optional[torch.Tensor] = None, dV: Optional[torch.Tensor] = None,
         workspace: Optional[torch.Tensor] = None,
         stream: Optional[torch.cuda.Stream] = None):
-    """Exact attention backward through ``fa_bwd`` (bf16), ``fa_bwd_qk`` (bf16, fewer
-    queries than keys) or ``fa_bwd_f32`` (float32).
+    """Exact attention backward through ``fa_bwd`` / ``fa_bwd_qk`` (bf16; the latter when
+    Nq != Nk) or ``fa_bwd_f32`` / ``fa_bwd_f32_qk`` (float32).
 
     Q, O, dO: [B, H, Nq, d]; K, V: [B, H, Nk, d]; CUDA tensors, contiguous, all bf16 or
     all float32; LSE: [B, H, Nq] float32.  Returns (dQ, dK, dV) in the inputs' dtype."""
@@ -187,8 +201,6 @@ def bwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, O: torch.Tensor,
     for name, t in (("K", K), ("V", V)):
         _check_bhnd(name, t, (B, H, Nk, d), dtype)
     _check_bhnd("LSE", LSE, (B, H, Nq), torch.float32)
-    if dtype == torch.float32 and Nq != Nk:
-        raise ValueError("the float32 path takes as many queries as keys")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     dQ = torch.empty_like(Q) if dQ is None else dQ
@@ -205,9 +217,12 @@ def bwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, O: torch.Tensor,
             _ptr(dV))
     tail = (float(scale), int(bool(causal)), _ptr(workspace), ws_bytes, _stream_handle(stream))
     with torch.cuda.device(Q.device):
-        if dtype == torch.float32:
+        if dtype == torch.float32 and Nq == Nk:
             name = "fa_bwd_f32"
             st = lib().fa_bwd_f32(*ptrs, B, H, Nq, d, *tail)
+        elif dtype == torch.float32:
+            name = "fa_bwd_f32_qk"
+            st = lib().fa_bwd_f32_qk(*ptrs, B, H, Nq, Nk, d, *tail)
         elif Nq == Nk:
             name = "fa_bwd"
             st = lib().fa_bwd(*ptrs, B, H, Nq, d, *tail)
@@ -245,6 +260,12 @@ def bwd_noalloc(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, O: torch.Tens
     return dQ, dK, dV
 
 
+def _layout_dtype(Q: torch.Tensor) -> torch.dtype:
+    if Q.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("Q, K, V must be bfloat16 or float32")
+    return Q.dtype
+
+
 def _check_seqlens(seqlens_q: torch.Tensor, seqlens_k: torch.Tensor, B: int, device) -> None:
     for name, t in (("seqlens_q", seqlens_q), ("seqlens_k", seqlens_k)):
         if not t.is_cuda or t.device != device:
@@ -257,15 +278,17 @@ def fwd_varlen(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, seqlens_q: tor
                seqlens_k: torch.Tensor, scale: Optional[float] = None, causal: bool = False,
                O: Optional[torch.Tensor] = None, LSE: Optional[torch.Tensor] = None,
                stream: Optional[torch.cuda.Stream] = None):
-    """Forward over a padded batch through ``fa_fwd_varlen``: sequence b uses its first
-    seqlens_q[b] query rows of Q [B, H, Nq, d] and seqlens_k[b] key rows of K, V
-    [B, H, Nk, d] (bf16).  Rows of O and LSE past a sequence's length are not written
-    (outputs allocated here start as zeros and -inf).  Returns (O, LSE)."""
+    """Forward over a padded batch through ``fa_fwd_varlen`` (bf16) or
+    ``fa_fwd_f32_varlen`` (float32): sequence b uses its first seqlens_q[b] query rows of
+    Q [B, H, Nq, d] and seqlens_k[b] key rows of K, V [B, H, Nk, d].  Rows of O and LSE
+    past a sequence's length are not written (outputs allocated here start as zeros and
+    -inf).  Returns (O, LSE)."""
     B, H, Nq, d = Q.shape
     Nk = K.shape[2]
-    _check_bhnd("Q", Q, (B, H, Nq, d), torch.bfloat16)
+    dtype = _layout_dtype(Q)
+    _check_bhnd("Q", Q, (B, H, Nq, d), dtype)
     for name, t in (("K", K), ("V", V)):
-        _check_bhnd(name, t, (B, H, Nk, d), torch.bfloat16)
+        _check_bhnd(name, t, (B, H, Nk, d), dtype)
     _check_seqlens(seqlens_q, seqlens_k, B, Q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
@@ -273,13 +296,14 @@ def fwd_varlen(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, seqlens_q: tor
         O = torch.zeros_like(Q)
     if LSE is None:
         LSE = torch.full((B, H, Nq), float("-inf"), device=Q.device, dtype=torch.float32)
-    _check_bhnd("O", O, (B, H, Nq, d), torch.bfloat16)
+    _check_bhnd("O", O, (B, H, Nq, d), dtype)
     _check_bhnd("LSE", LSE, (B, H, Nq), torch.float32)
+    name = "fa_fwd_varlen" if dtype == torch.bfloat16 else "fa_fwd_f32_varlen"
     with torch.cuda.device(Q.device):
-        st = lib().fa_fwd_varlen(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), _ptr(seqlens_q),
-                                 _ptr(seqlens_k), B, H, Nq, Nk, d, float(scale),
-                                 int(bool(causal)), _stream_handle(stream))
-    _check("fa_fwd_varlen", st)
+        st = getattr(lib(), name)(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE),
+                                  _ptr(seqlens_q), _ptr(seqlens_k), B, H, Nq, Nk, d,
+                                  float(scale), int(bool(causal)), _stream_handle(stream))
+    _check(name, st)
     return O, LSE
 
 
@@ -289,15 +313,17 @@ def bwd_varlen(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, O: torch.Tenso
                dQ: Optional[torch.Tensor] = None, dK: Optional[torch.Tensor] = None,
                dV: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
                stream: Optional[torch.cuda.Stream] = None):
-    """Backward over a padded batch through ``fa_bwd_varlen`` (the gradient of
-    ``fwd_varlen`` with the same lengths).  Rows past a sequence's lengths are not
-    written (gradients allocated here start as zeros).  Returns (dQ, dK, dV)."""
+    """Backward over a padded batch through ``fa_bwd_varlen`` (bf16) or
+    ``fa_bwd_f32_varlen`` (float32), the gradient of ``fwd_varlen`` with the same lengths.
+    Rows past a sequence's lengths are not written (gradients allocated here start as
+    zeros).  Returns (dQ, dK, dV)."""
     B, H, Nq, d = Q.shape
     Nk = K.shape[2]
+    dtype = _layout_dtype(Q)
     for name, t in (("Q", Q), ("O", O), ("dO", dO)):
-        _check_bhnd(name, t, (B, H, Nq, d), torch.bfloat16)
+        _check_bhnd(name, t, (B, H, Nq, d), dtype)
     for name, t in (("K", K), ("V", V)):
-        _check_bhnd(name, t, (B, H, Nk, d), torch.bfloat16)
+        _check_bhnd(name, t, (B, H, Nk, d), dtype)
     _check_bhnd("LSE", LSE, (B, H, Nq), torch.float32)
     _check_seqlens(seqlens_q, seqlens_k, B, Q.device)
     if scale is None:
@@ -305,24 +331,27 @@ def bwd_varlen(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, O: torch.Tenso
     dQ = torch.zeros_like(Q) if dQ is None else dQ
     dK = torch.zeros_like(K) if dK is None else dK
     dV = torch.zeros_like(V) if dV is None else dV
-    _check_bhnd("dQ", dQ, (B, H, Nq, d), torch.bfloat16)
+    _check_bhnd("dQ", dQ, (B, H, Nq, d), dtype)
     for name, t in (("dK", dK), ("dV", dV)):
-        _check_bhnd(name, t, (B, H, Nk, d), torch.bfloat16)
+        _check_bhnd(name, t, (B, H, Nk, d), dtype)
     need = workspace_bytes(B, H, Nq, d)
     if workspace is None:
         workspace = torch.empty(max(need, 1), device=Q.device, dtype=torch.uint8)
     ws_bytes = workspace.numel() * workspace.element_size()
+    name = "fa_bwd_varlen" if dtype == torch.bfloat16 else "fa_bwd_f32_varlen"
     with torch.cuda.device(Q.device):
-        st = lib().fa_bwd_varlen(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _ptr(LSE),
-                                 _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(seqlens_q), _ptr(seqlens_k),
-                                 B, H, Nq, Nk, d, float(scale), int(bool(causal)),
-                                 _ptr(workspace), ws_bytes, _stream_handle(stream))
-    _check("fa_bwd_varlen", st)
+        st = getattr(lib(), name)(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _ptr(LSE),
+                                  _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(seqlens_q),
+                                  _ptr(seqlens_k), B, H, Nq, Nk, d, float(scale),
+                                  int(bool(causal)), _ptr(workspace), ws_bytes,
+                                  _stream_handle(stream))
+    _check(name, st)
     return dQ, dK, dV
 
 
-def _check_packed(name: str, t: torch.Tensor, tokens: int, H: int, d: int) -> None:
-    _check_bhnd(name, t, (tokens, H, d), torch.bfloat16)
+def _check_packed(name: str, t: torch.Tensor, tokens: int, H: int, d: int,
+                  dtype: torch.dtype = torch.bfloat16) -> None:
+    _check_bhnd(name, t, (tokens, H, d), dtype)
 
 
 def _check_cu(cu_q: torch.Tensor, cu_k: torch.Tensor, device) -> int:
@@ -340,27 +369,30 @@ def fwd_packed(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, cu_seqlens_q: 
                scale: Optional[float] = None, causal: bool = False,
                O: Optional[torch.Tensor] = None, LSE: Optional[torch.Tensor] = None,
                stream: Optional[torch.cuda.Stream] = None):
-    """Forward over a packed batch through ``fa_fwd_packed``: Q [total_q, H, d], K and V
-    [total_k, H, d] (bf16), sequences delimited by the int32 start arrays (B+1 entries).
+    """Forward over a packed batch through ``fa_fwd_packed`` (bf16) or
+    ``fa_fwd_f32_packed`` (float32): Q [total_q, H, d], K and V [total_k, H, d], sequences
+    delimited by the int32 start arrays (B+1 entries).
     Returns (O [total_q, H, d], LSE [H, total_q])."""
     total_q, H, d = Q.shape
     total_k = K.shape[0]
-    _check_packed("Q", Q, total_q, H, d)
+    dtype = _layout_dtype(Q)
+    _check_packed("Q", Q, total_q, H, d, dtype)
     for name, t in (("K", K), ("V", V)):
-        _check_packed(name, t, total_k, H, d)
+        _check_packed(name, t, total_k, H, d, dtype)
     B = _check_cu(cu_seqlens_q, cu_seqlens_k, Q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     O = torch.zeros_like(Q) if O is None else O
     LSE = torch.full((H, total_q), float("-inf"), device=Q.device) if LSE is None else LSE
-    _check_packed("O", O, total_q, H, d)
+    _check_packed("O", O, total_q, H, d, dtype)
     _check_bhnd("LSE", LSE, (H, total_q), torch.float32)
+    name = "fa_fwd_packed" if dtype == torch.bfloat16 else "fa_fwd_f32_packed"
     with torch.cuda.device(Q.device):
-        st = lib().fa_fwd_packed(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE),
-                                 _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), B, H, int(max_seqlen_q),
-                                 int(max_seqlen_k), total_q, total_k, d, float(scale),
-                                 int(bool(causal)), _stream_handle(stream))
-    _check("fa_fwd_packed", st)
+        st = getattr(lib(), name)(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE),
+                                  _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), B, H,
+                                  int(max_seqlen_q), int(max_seqlen_k), total_q, total_k, d,
+                                  float(scale), int(bool(causal)), _stream_handle(stream))
+    _check(name, st)
     return O, LSE
 
 
@@ -371,14 +403,16 @@ def bwd_packed(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, O: torch.Tenso
                dQ: Optional[torch.Tensor] = None, dK: Optional[torch.Tensor] = None,
                dV: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
                stream: Optional[torch.cuda.Stream] = None):
-    """Backward over a packed batch through ``fa_bwd_packed`` (the gradient of
-    ``fwd_packed`` with the same start arrays).  Returns (dQ, dK, dV)."""
+    """Backward over a packed batch through ``fa_bwd_packed`` (bf16) or
+    ``fa_bwd_f32_packed`` (float32), the gradient of ``fwd_packed`` with the same start
+    arrays.  Returns (dQ, dK, dV)."""
     total_q, H, d = Q.shape
     total_k = K.shape[0]
+    dtype = _layout_dtype(Q)
     for name, t in (("Q", Q), ("O", O), ("dO", dO)):
-        _check_packed(name, t, total_q, H, d)
+        _check_packed(name, t, total_q, H, d, dtype)
     for name, t in (("K", K), ("V", V)):
-        _check_packed(name, t, total_k, H, d)
+        _check_packed(name, t, total_k, H, d, dtype)
     _check_bhnd("LSE", LSE, (H, total_q), torch.float32)
     B = _check_cu(cu_seqlens_q, cu_seqlens_k, Q.device)
     if scale is None:
@@ -386,20 +420,22 @@ def bwd_packed(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, O: torch.Tenso
     dQ = torch.zeros_like(Q) if dQ is None else dQ
     dK = torch.zeros_like(K) if dK is None else dK
     dV = torch.zeros_like(V) if dV is None else dV
-    _check_packed("dQ", dQ, total_q, H, d)
+    _check_packed("dQ", dQ, total_q, H, d, dtype)
     for name, t in (("dK", dK), ("dV", dV)):
-        _check_packed(name, t, total_k, H, d)
+        _check_packed(name, t, total_k, H, d, dtype)
     need = workspace_bytes(B, H, int(max_seqlen_q), d)
     if workspace is None:
         workspace = torch.empty(max(need, 1), device=Q.device, dtype=torch.uint8)
     ws_bytes = workspace.numel() * workspace.element_size()
+    name = "fa_bwd_packed" if dtype == torch.bfloat16 else "fa_bwd_f32_packed"
     with torch.cuda.device(Q.device):
-        st = lib().fa_bwd_packed(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _ptr(LSE),
-                                 _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(cu_seqlens_q),
-                                 _ptr(cu_seqlens_k), B, H, int(max_seqlen_q), int(max_seqlen_k),
-                                 total_q, total_k, d, float(scale), int(bool(causal)),
-                                 _ptr(workspace), ws_bytes, _stream_handle(stream))
-    _check("fa_bwd_packed", st)
+        st = getattr(lib(), name)(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _ptr(LSE),
+                                  _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(cu_seqlens_q),
+                                  _ptr(cu_seqlens_k), B, H, int(max_seqlen_q),
+                                  int(max_seqlen_k), total_q, total_k, d, float(scale),
+                                  int(bool(causal)), _ptr(workspace), ws_bytes,
+                                  _stream_handle(stream))
+    _check(name, st)
     return dQ, dK, dV
 
 

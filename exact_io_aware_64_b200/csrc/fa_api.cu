@@ -367,6 +367,100 @@ fa_status check_packed(const int* cu_q, const int* cu_k, int B, int H, int max_q
   return FA_OK;
 }
 
+// Pointer and overlap checks of the packed-layout forward calls (elem = bytes per
+// element of Q, K, V, O).
+fa_status check_packed_fwd_ptrs(const void* Q, const void* K, const void* V, const void* O,
+                                const float* LSE, int H, int d, int total_q, int total_k,
+                                size_t elem) {
+  FA_TRY(check_ptr(Q, "Q"));
+  FA_TRY(check_ptr(K, "K"));
+  FA_TRY(check_ptr(V, "V"));
+  FA_TRY(check_ptr(O, "O"));
+  if (LSE != nullptr && (reinterpret_cast<uintptr_t>(LSE) & 3u))
+    return fail(FA_ERR_INVALID_ARG, "LSE is not 4-byte aligned");
+  const size_t qb = static_cast<size_t>(total_q) * H * d * elem;
+  const size_t kb = static_cast<size_t>(total_k) * H * d * elem;
+  if (overlaps(O, qb, Q, qb) || overlaps(O, qb, K, kb) || overlaps(O, qb, V, kb))
+    return fail(FA_ERR_INVALID_ARG, "O overlaps an input");
+  return FA_OK;
+}
+
+// Pointer, workspace and overlap checks of the packed-layout backward calls.
+fa_status check_packed_bwd_ptrs(const void* Q, const void* K, const void* V, const void* O,
+                                const void* dO, const float* LSE, const void* dQ,
+                                const void* dK, const void* dV, int H, int d, int total_q,
+                                int total_k, const void* workspace, size_t need,
+                                size_t workspace_bytes, size_t elem) {
+  FA_TRY(check_ptr(Q, "Q"));
+  FA_TRY(check_ptr(K, "K"));
+  FA_TRY(check_ptr(V, "V"));
+  FA_TRY(check_ptr(O, "O"));
+  FA_TRY(check_ptr(dO, "dO"));
+  FA_TRY(check_ptr(LSE, "LSE"));
+  FA_TRY(check_ptr(dQ, "dQ"));
+  FA_TRY(check_ptr(dK, "dK"));
+  FA_TRY(check_ptr(dV, "dV"));
+  FA_TRY(check_ptr(workspace, "workspace"));
+  if (workspace_bytes < need)
+    return fail(FA_ERR_INVALID_ARG, "workspace has %zu bytes, %zu needed", workspace_bytes,
+                need);
+  const size_t qb = static_cast<size_t>(total_q) * H * d * elem;
+  const size_t kb = static_cast<size_t>(total_k) * H * d * elem;
+  struct Buf {
+    const void* p;
+    size_t n;
+  };
+  const Buf ins[5] = {{Q, qb}, {K, kb}, {V, kb}, {O, qb}, {dO, qb}};
+  const Buf outs[3] = {{dQ, qb}, {dK, kb}, {dV, kb}};
+  for (const Buf& o : outs) {
+    for (const Buf& in : ins)
+      if (overlaps(o.p, o.n, in.p, in.n))
+        return fail(FA_ERR_INVALID_ARG, "a gradient overlaps an input");
+    if (overlaps(o.p, o.n, workspace, need))
+      return fail(FA_ERR_INVALID_ARG, "a gradient overlaps the workspace");
+  }
+  if (overlaps(dQ, qb, dK, kb) || overlaps(dQ, qb, dV, kb) || overlaps(dK, kb, dV, kb))
+    return fail(FA_ERR_INVALID_ARG, "gradients overlap each other");
+  return FA_OK;
+}
+
+// float32 forward, dense or padded layout (seqlens null: every row of every head).
+fa_status fwd_f32_impl(const float* Q, const float* K, const float* V, float* O, float* LSE,
+                       int B, int H, int Nq, int Nk, int d, float scale, int causal,
+                       cudaStream_t stream, const int* seqlens_q = nullptr,
+                       const int* seqlens_k = nullptr) {
+  g_last_error[0] = '\0';
+  bool noop = false;
+  FA_TRY(check_fwd_args(Q, K, V, O, LSE, B, H, Nq, Nk, d, scale, causal, 4, &noop));
+  if (noop) return FA_OK;  // empty problem: the pointers are never used (may be NULL)
+  DeviceInfo dev;
+  FA_TRY(device_info(&dev));
+  const fa::Problem p = make_problem(B, H, Nq, Nk, d, scale, causal, dev, seqlens_q, seqlens_k);
+  cudaError_t e = fa::launch_fwd_f32(Q, K, V, O, LSE, p, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "launching the float32 forward kernel");
+  return FA_OK;
+}
+
+// float32 backward, dense or padded layout.
+fa_status bwd_f32_impl(const float* Q, const float* K, const float* V, const float* O,
+                       const float* dO, const float* LSE, float* dQ, float* dK, float* dV,
+                       int B, int H, int Nq, int Nk, int d, float scale, int causal,
+                       void* workspace, size_t workspace_bytes, cudaStream_t stream,
+                       const int* seqlens_q = nullptr, const int* seqlens_k = nullptr) {
+  g_last_error[0] = '\0';
+  bool noop = false;
+  FA_TRY(check_bwd_args(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, Nq, Nk, d, scale, causal,
+                        workspace, workspace_bytes, 4, &noop));
+  if (noop) return FA_OK;  // empty problem: the pointers are never used (may be NULL)
+  DeviceInfo dev;
+  FA_TRY(device_info(&dev));
+  const fa::Problem p = make_problem(B, H, Nq, Nk, d, scale, causal, dev, seqlens_q, seqlens_k);
+  cudaError_t e = fa::launch_bwd_f32(Q, K, V, O, dO, LSE, dQ, dK, dV,
+                                     static_cast<float*>(workspace), p, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "launching the float32 backward kernels");
+  return FA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -425,16 +519,7 @@ fa_status fa_fwd_packed(const void* Q, const void* K, const void* V, void* O, fl
   FA_TRY(check_packed(cu_seqlens_q, cu_seqlens_k, B, H, max_seqlen_q, max_seqlen_k, total_q,
                       total_k, d, scale, causal, &noop));
   if (noop) return FA_OK;
-  FA_TRY(check_ptr(Q, "Q"));
-  FA_TRY(check_ptr(K, "K"));
-  FA_TRY(check_ptr(V, "V"));
-  FA_TRY(check_ptr(O, "O"));
-  if (LSE != nullptr && (reinterpret_cast<uintptr_t>(LSE) & 3u))
-    return fail(FA_ERR_INVALID_ARG, "LSE is not 4-byte aligned");
-  const size_t qb = static_cast<size_t>(total_q) * H * d * 2;
-  const size_t kb = static_cast<size_t>(total_k) * H * d * 2;
-  if (overlaps(O, qb, Q, qb) || overlaps(O, qb, K, kb) || overlaps(O, qb, V, kb))
-    return fail(FA_ERR_INVALID_ARG, "O overlaps an input");
+  FA_TRY(check_packed_fwd_ptrs(Q, K, V, O, LSE, H, d, total_q, total_k, 2));
   DeviceInfo dev;
   FA_TRY(device_info(&dev));
   FA_TRY(require_sm100(dev));
@@ -461,37 +546,9 @@ fa_status fa_bwd_packed(const void* Q, const void* K, const void* V, const void*
   FA_TRY(check_packed(cu_seqlens_q, cu_seqlens_k, B, H, max_seqlen_q, max_seqlen_k, total_q,
                       total_k, d, scale, causal, &noop));
   if (noop) return FA_OK;
-  FA_TRY(check_ptr(Q, "Q"));
-  FA_TRY(check_ptr(K, "K"));
-  FA_TRY(check_ptr(V, "V"));
-  FA_TRY(check_ptr(O, "O"));
-  FA_TRY(check_ptr(dO, "dO"));
-  FA_TRY(check_ptr(LSE, "LSE"));
-  FA_TRY(check_ptr(dQ, "dQ"));
-  FA_TRY(check_ptr(dK, "dK"));
-  FA_TRY(check_ptr(dV, "dV"));
   const size_t need = fa_bwd_workspace_bytes(B, H, max_seqlen_q, d);
-  FA_TRY(check_ptr(workspace, "workspace"));
-  if (workspace_bytes < need)
-    return fail(FA_ERR_INVALID_ARG, "workspace has %zu bytes, %zu needed", workspace_bytes,
-                need);
-  const size_t qb = static_cast<size_t>(total_q) * H * d * 2;
-  const size_t kb = static_cast<size_t>(total_k) * H * d * 2;
-  struct Buf {
-    const void* p;
-    size_t n;
-  };
-  const Buf ins[5] = {{Q, qb}, {K, kb}, {V, kb}, {O, qb}, {dO, qb}};
-  const Buf outs[3] = {{dQ, qb}, {dK, kb}, {dV, kb}};
-  for (const Buf& o : outs) {
-    for (const Buf& in : ins)
-      if (overlaps(o.p, o.n, in.p, in.n))
-        return fail(FA_ERR_INVALID_ARG, "a gradient overlaps an input");
-    if (overlaps(o.p, o.n, workspace, need))
-      return fail(FA_ERR_INVALID_ARG, "a gradient overlaps the workspace");
-  }
-  if (overlaps(dQ, qb, dK, kb) || overlaps(dQ, qb, dV, kb) || overlaps(dK, kb, dV, kb))
-    return fail(FA_ERR_INVALID_ARG, "gradients overlap each other");
+  FA_TRY(check_packed_bwd_ptrs(Q, K, V, O, dO, LSE, dQ, dK, dV, H, d, total_q, total_k,
+                               workspace, need, workspace_bytes, 2));
   DeviceInfo dev;
   FA_TRY(device_info(&dev));
   FA_TRY(require_sm100(dev));
@@ -517,13 +574,41 @@ fa_status fa_bwd_packed(const void* Q, const void* K, const void* V, const void*
 fa_status fa_fwd_f32(const float* Q, const float* K, const float* V, float* O, float* LSE,
                      int B, int H, int N, int d, float scale, int causal,
                      cudaStream_t stream) {
+  return fwd_f32_impl(Q, K, V, O, LSE, B, H, N, N, d, scale, causal, stream);
+}
+
+fa_status fa_fwd_f32_qk(const float* Q, const float* K, const float* V, float* O, float* LSE,
+                        int B, int H, int Nq, int Nk, int d, float scale, int causal,
+                        cudaStream_t stream) {
+  return fwd_f32_impl(Q, K, V, O, LSE, B, H, Nq, Nk, d, scale, causal, stream);
+}
+
+fa_status fa_fwd_f32_varlen(const float* Q, const float* K, const float* V, float* O,
+                            float* LSE, const int* seqlens_q, const int* seqlens_k, int B,
+                            int H, int Nq, int Nk, int d, float scale, int causal,
+                            cudaStream_t stream) {
+  g_last_error[0] = '\0';
+  if (B > 0 && H > 0 && Nq > 0) FA_TRY(check_seqlens(seqlens_q, seqlens_k));
+  return fwd_f32_impl(Q, K, V, O, LSE, B, H, Nq, Nk, d, scale, causal, stream, seqlens_q,
+                      seqlens_k);
+}
+
+fa_status fa_fwd_f32_packed(const float* Q, const float* K, const float* V, float* O,
+                            float* LSE, const int* cu_seqlens_q, const int* cu_seqlens_k,
+                            int B, int H, int max_seqlen_q, int max_seqlen_k, int total_q,
+                            int total_k, int d, float scale, int causal,
+                            cudaStream_t stream) {
   g_last_error[0] = '\0';
   bool noop = false;
-  FA_TRY(check_fwd_args(Q, K, V, O, LSE, B, H, N, N, d, scale, causal, 4, &noop));
-  if (noop) return FA_OK;  // empty problem: the pointers are never used (may be NULL)
+  FA_TRY(check_packed(cu_seqlens_q, cu_seqlens_k, B, H, max_seqlen_q, max_seqlen_k, total_q,
+                      total_k, d, scale, causal, &noop));
+  if (noop) return FA_OK;
+  FA_TRY(check_packed_fwd_ptrs(Q, K, V, O, LSE, H, d, total_q, total_k, 4));
   DeviceInfo dev;
   FA_TRY(device_info(&dev));
-  const fa::Problem p = make_problem(B, H, N, N, d, scale, causal, dev);
+  const fa::Problem p = make_problem(B, H, max_seqlen_q, max_seqlen_k, d, scale, causal, dev,
+                                     nullptr, nullptr, cu_seqlens_q, cu_seqlens_k, total_q,
+                                     total_k);
   cudaError_t e = fa::launch_fwd_f32(Q, K, V, O, LSE, p, stream);
   if (e != cudaSuccess) return cuda_fail(e, "launching the float32 forward kernel");
   return FA_OK;
@@ -568,14 +653,48 @@ fa_status fa_bwd_f32(const float* Q, const float* K, const float* V, const float
                      const float* dO, const float* LSE, float* dQ, float* dK, float* dV, int B,
                      int H, int N, int d, float scale, int causal, void* workspace,
                      size_t workspace_bytes, cudaStream_t stream) {
+  return bwd_f32_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, N, d, scale, causal,
+                      workspace, workspace_bytes, stream);
+}
+
+fa_status fa_bwd_f32_qk(const float* Q, const float* K, const float* V, const float* O,
+                        const float* dO, const float* LSE, float* dQ, float* dK, float* dV,
+                        int B, int H, int Nq, int Nk, int d, float scale, int causal,
+                        void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return bwd_f32_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, Nq, Nk, d, scale, causal,
+                      workspace, workspace_bytes, stream);
+}
+
+fa_status fa_bwd_f32_varlen(const float* Q, const float* K, const float* V, const float* O,
+                            const float* dO, const float* LSE, float* dQ, float* dK,
+                            float* dV, const int* seqlens_q, const int* seqlens_k, int B,
+                            int H, int Nq, int Nk, int d, float scale, int causal,
+                            void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  g_last_error[0] = '\0';
+  if (B > 0 && H > 0 && Nq > 0) FA_TRY(check_seqlens(seqlens_q, seqlens_k));
+  return bwd_f32_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, Nq, Nk, d, scale, causal,
+                      workspace, workspace_bytes, stream, seqlens_q, seqlens_k);
+}
+
+fa_status fa_bwd_f32_packed(const float* Q, const float* K, const float* V, const float* O,
+                            const float* dO, const float* LSE, float* dQ, float* dK,
+                            float* dV, const int* cu_seqlens_q, const int* cu_seqlens_k,
+                            int B, int H, int max_seqlen_q, int max_seqlen_k, int total_q,
+                            int total_k, int d, float scale, int causal, void* workspace,
+                            size_t workspace_bytes, cudaStream_t stream) {
   g_last_error[0] = '\0';
   bool noop = false;
-  FA_TRY(check_bwd_args(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, N, d, scale, causal,
-                        workspace, workspace_bytes, 4, &noop));
-  if (noop) return FA_OK;  // empty problem: the pointers are never used (may be NULL)
+  FA_TRY(check_packed(cu_seqlens_q, cu_seqlens_k, B, H, max_seqlen_q, max_seqlen_k, total_q,
+                      total_k, d, scale, causal, &noop));
+  if (noop) return FA_OK;
+  const size_t need = fa_bwd_workspace_bytes(B, H, max_seqlen_q, d);
+  FA_TRY(check_packed_bwd_ptrs(Q, K, V, O, dO, LSE, dQ, dK, dV, H, d, total_q, total_k,
+                               workspace, need, workspace_bytes, 4));
   DeviceInfo dev;
   FA_TRY(device_info(&dev));
-  const fa::Problem p = make_problem(B, H, N, N, d, scale, causal, dev);
+  const fa::Problem p = make_problem(B, H, max_seqlen_q, max_seqlen_k, d, scale, causal, dev,
+                                     nullptr, nullptr, cu_seqlens_q, cu_seqlens_k, total_q,
+                                     total_k);
   cudaError_t e = fa::launch_bwd_f32(Q, K, V, O, dO, LSE, dQ, dK, dV,
                                      static_cast<float*>(workspace), p, stream);
   if (e != cudaSuccess) return cuda_fail(e, "launching the float32 backward kernels");

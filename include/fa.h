@@ -159,6 +159,25 @@ FA_API fa_status fa_fwd_f32(const float* Q, const float* K, const float* V, floa
                      cudaStream_t stream);
 
 /*
+ * The float32 forward with Nq queries and Nk keys per head, over a padded batch, and
+ * over a packed batch: the same definitions, arguments, layouts, length rules and
+ * errors as fa_fwd_qk, fa_fwd_varlen and fa_fwd_packed, with float32 tensors (Q, K, V,
+ * O) and float32 arithmetic on the CUDA cores.  Any sm_100 device.
+ */
+FA_API fa_status fa_fwd_f32_qk(const float* Q, const float* K, const float* V, float* O,
+                               float* LSE, int B, int H, int Nq, int Nk, int d, float scale,
+                               int causal, cudaStream_t stream);
+FA_API fa_status fa_fwd_f32_varlen(const float* Q, const float* K, const float* V, float* O,
+                                   float* LSE, const int* seqlens_q, const int* seqlens_k,
+                                   int B, int H, int Nq, int Nk, int d, float scale,
+                                   int causal, cudaStream_t stream);
+FA_API fa_status fa_fwd_f32_packed(const float* Q, const float* K, const float* V, float* O,
+                                   float* LSE, const int* cu_seqlens_q,
+                                   const int* cu_seqlens_k, int B, int H, int max_seqlen_q,
+                                   int max_seqlen_k, int total_q, int total_k, int d,
+                                   float scale, int causal, cudaStream_t stream);
+
+/*
  * Bytes of scratch that fa_bwd (and fa_bwd_f32) needs for given sizes: two float32 per query row
  * (D_i = sum_k dO_ik O_ik and LSE_i * log2(e)), rows padded to a multiple of 128,
  * rounded up to 256 bytes: 8 * B * H * ceil(N/128) * 128.  Grows as B*H*N, never as N^2.
@@ -239,6 +258,33 @@ FA_API fa_status fa_bwd_f32(const float* Q, const float* K, const float* V, cons
                             const float* dO, const float* LSE, float* dQ, float* dK,
                             float* dV, int B, int H, int N, int d, float scale, int causal,
                             void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * The float32 backward with Nq queries and Nk keys per head, over a padded batch, and
+ * over a packed batch: the gradients of fa_fwd_f32_qk, fa_fwd_f32_varlen and
+ * fa_fwd_f32_packed, with the arguments, layouts, workspace sizes and rules of
+ * fa_bwd_qk, fa_bwd_varlen and fa_bwd_packed and float32 tensors.  D goes to the first
+ * 4*B*H*Nq (packed: 4*B*H*max_seqlen_q) bytes of the workspace.  Rows past a sequence's
+ * lengths are not written.  Otherwise as fa_bwd_f32.
+ */
+FA_API fa_status fa_bwd_f32_qk(const float* Q, const float* K, const float* V, const float* O,
+                               const float* dO, const float* LSE, float* dQ, float* dK,
+                               float* dV, int B, int H, int Nq, int Nk, int d, float scale,
+                               int causal, void* workspace, size_t workspace_bytes,
+                               cudaStream_t stream);
+FA_API fa_status fa_bwd_f32_varlen(const float* Q, const float* K, const float* V,
+                                   const float* O, const float* dO, const float* LSE,
+                                   float* dQ, float* dK, float* dV, const int* seqlens_q,
+                                   const int* seqlens_k, int B, int H, int Nq, int Nk, int d,
+                                   float scale, int causal, void* workspace,
+                                   size_t workspace_bytes, cudaStream_t stream);
+FA_API fa_status fa_bwd_f32_packed(const float* Q, const float* K, const float* V,
+                                   const float* O, const float* dO, const float* LSE,
+                                   float* dQ, float* dK, float* dV, const int* cu_seqlens_q,
+                                   const int* cu_seqlens_k, int B, int H, int max_seqlen_q,
+                                   int max_seqlen_k, int total_q, int total_k, int d,
+                                   float scale, int causal, void* workspace,
+                                   size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * Merge a partial attention result into an accumulator ("FlashAttention, simplified",

@@ -269,3 +269,51 @@ def test_binding_refuses_host_tensors():
         binding.merge(torch.zeros(1, 1, 8, 64), lse, q, lse)
     with pytest.raises(ValueError):
         binding.accumulate(torch.zeros(8), torch.zeros(8, dtype=torch.bfloat16))
+
+
+def test_f32_layout_validation(lib):
+    """The float32 Nq != Nk, padded and packed calls follow the bf16 rules, with 4-byte
+    elements in the size and overlap checks."""
+    F, G, H_, I, J = 0x600000, 0x700000, 0x800000, 0x900000, 0xA00000
+    SQ, SK = 0xB00000, 0xC00000
+
+    def fwd_qk(Nq, Nk, causal=1, o=D_):
+        return lib.fa_fwd_f32_qk(A, B_, C, o, E, 1, 2, Nq, Nk, 64, 0.1, causal, None)
+
+    assert fwd_qk(0, 5) == binding.FA_OK
+    assert fwd_qk(4, 0) == binding.FA_ERR_INVALID_ARG
+    assert fwd_qk(8, 4, causal=1) == binding.FA_ERR_INVALID_ARG
+    assert fwd_qk(8, 4, causal=0) != binding.FA_ERR_INVALID_ARG
+    # K holds 2 heads x 64 rows x 64 float32: O just past it does not overlap, 16 B less does
+    assert fwd_qk(16, 64, o=B_ + 2 * 64 * 64 * 4) != binding.FA_ERR_INVALID_ARG
+    assert fwd_qk(16, 64, o=B_ + 2 * 64 * 64 * 4 - 16) == binding.FA_ERR_INVALID_ARG
+
+    def bwd_qk(Nq, Nk, ws_bytes=1 << 20, dk=H_):
+        return lib.fa_bwd_f32_qk(A, B_, C, D_, E, F, G, dk, I, 1, 2, Nq, Nk, 64, 0.1, 1, J,
+                                 ws_bytes, None)
+
+    assert bwd_qk(5, 3) == binding.FA_ERR_INVALID_ARG
+    need = binding.workspace_bytes(1, 2, 100, 64)
+    assert bwd_qk(100, 1000, ws_bytes=need - 4) == binding.FA_ERR_INVALID_ARG
+    assert bwd_qk(100, 1000, ws_bytes=need) != binding.FA_ERR_INVALID_ARG
+    assert bwd_qk(100, 1000, dk=G + 2 * 100 * 64 * 4 - 16) == binding.FA_ERR_INVALID_ARG
+
+    assert lib.fa_fwd_f32_varlen(A, B_, C, D_, E, 0, SK, 2, 2, 64, 64, 64, 0.1, 1,
+                                 None) == binding.FA_ERR_INVALID_ARG
+    assert lib.fa_fwd_f32_varlen(A, B_, C, D_, E, SQ, SK, 2, 2, 128, 64, 64, 0.1, 1,
+                                 None) == binding.FA_ERR_INVALID_ARG
+    assert lib.fa_bwd_f32_varlen(A, B_, C, D_, E, F, G, H_, I, SQ, 0, 2, 2, 64, 64, 64, 0.1,
+                                 1, J, 1 << 20, None) == binding.FA_ERR_INVALID_ARG
+
+    def fwd_packed(cq=SQ, ck=SK, tq=100, tk=100, o=D_):
+        return lib.fa_fwd_f32_packed(A, B_, C, o, E, cq, ck, 2, 2, 64, 64, tq, tk, 64, 0.1, 1,
+                                     None)
+
+    assert fwd_packed(tq=0, cq=0, ck=0) == binding.FA_OK
+    assert fwd_packed(cq=0) == binding.FA_ERR_INVALID_ARG
+    # Q holds 100 tokens x 2 heads x 64 float32
+    assert fwd_packed(o=A + 100 * 2 * 64 * 4 - 16) == binding.FA_ERR_INVALID_ARG
+    need = binding.workspace_bytes(2, 2, 64, 64)
+    st = lib.fa_bwd_f32_packed(A, B_, C, D_, E, F, G, H_, I, SQ, SK, 2, 2, 64, 64, 100, 100,
+                               64, 0.1, 1, J, need - 4, None)
+    assert st == binding.FA_ERR_INVALID_ARG

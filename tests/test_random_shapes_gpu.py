@@ -1,7 +1,7 @@
 """Seeded random shapes: forward and backward against the oracle on problems drawn at
 random (query and key counts with offsets that are not multiples of the tile, both head
-sizes and masks, logit scales from flat to peaked), so that no mask or tail rule is
-only exercised at hand-picked sizes.  Every case is fixed by its seed."""
+sizes and masks, logit scales from flat to peaked; bf16 and float32), so that no mask or
+tail rule is only exercised at hand-picked sizes.  Every case is fixed by its seed."""
 import numpy as np
 import pytest
 import torch
@@ -63,25 +63,30 @@ def test_random_shape(seed):
 
 @pytest.mark.parametrize("seed", range(8))
 def test_random_shape_f32(seed):
-    """The float32 path (square problems only) at random lengths, heads and masks."""
+    """The float32 path at random query and key counts, heads and masks."""
     rng = np.random.default_rng(20000 + seed)
     d = int(rng.choice([64, 128]))
     causal = bool(rng.integers(2))
-    N = int(rng.integers(1, 400))
+    Nk = int(rng.integers(1, 400))
+    Nq = int(rng.integers(1, Nk + 1)) if causal else int(rng.integers(1, 400))
     H = int(rng.integers(1, 3))
-    ins = inputs.make_inputs(1, H, N, d, seed=9900 + seed, dtype=torch.float32, with_dO=True)
+    a = inputs.make_inputs(1, H, Nq, d, seed=9900 + seed, dtype=torch.float32, with_dO=True)
+    b = inputs.make_inputs(1, H, Nk, d, seed=9950 + seed, dtype=torch.float32)
     scale = d ** -0.5
-    q, k, v, do = (ins[n].cuda() for n in ("Q", "K", "V", "dO"))
+    q, do = a["Q"].cuda(), a["dO"].cuda()
+    k, v = b["K"].cuda(), b["V"].cuda()
     O, LSE = binding.fwd(q, k, v, scale=scale, causal=causal)
     dQ, dK, dV = binding.bwd(q, k, v, O, do, LSE, scale=scale, causal=causal)
     binding.check_device_error()
     assert O.dtype == torch.float32 and dQ.dtype == torch.float32
-    what = f"f32 seed={seed} d={d} causal={causal} N={N}"
+    pos = oracle.chunk_positions(Nq, Nk) if causal else None
+    what = f"f32 seed={seed} d={d} causal={causal} Nq={Nq} Nk={Nk}"
     for h in range(H):
-        args = [to64(ins[n][0, h]) for n in ("Q", "K", "V", "dO")]
-        rO, rL, _ = oracle.attention_head(args[0], args[1], args[2], scale, causal)
+        Qh, Gh = to64(a["Q"][0, h]), to64(a["dO"][0, h])
+        Kh, Vh = to64(b["K"][0, h]), to64(b["V"][0, h])
+        rO, rL, _ = oracle.attention_head(Qh, Kh, Vh, scale, causal, pos)
         assert_f32_close(to64(O[0, h]), rO, "O " + what)
         assert_lse_close(to64(LSE[0, h]), rL, "LSE " + what)
-        ref = oracle.attention_bwd_head(*args, scale, causal)
+        ref = oracle.attention_bwd_head(Qh, Kh, Vh, Gh, scale, causal, q_index=pos)
         for k_, name, got in ((0, "dQ", dQ), (1, "dK", dK), (2, "dV", dV)):
             assert_f32_close(to64(got[0, h]), ref[k_], f"{name} {what}")
