@@ -15,7 +15,9 @@ Rank 0 prints one JSON line.  Besides the contract keys it carries:
   e2e           the same metric with host buffers: pinned host -> device copies of the
                 inputs, fa_fwd, fa_bwd and device -> host copies of the results, all
                 inside the timed region; pipelined over three streams (uploads, compute,
-                downloads), with the one-stream figure beside it ("serial")
+                downloads), with the one-stream figure beside it ("serial") and the
+                time of the same copies alone, both directions at once
+                ("copy_floor_ms": no pipelined step can be faster)
   clocks        SM clocks and throttle reasons sampled during the timed region
 """
 from __future__ import annotations
@@ -329,7 +331,9 @@ def run_gpu(args, w):
     fa_dist.barrier(info)
     e0, e1 = ev(), ev()
     e0.record(stream)
-    e2e_steps = max(2, min(args.steps, 10))
+    # enough steps that the pipelined figure below is not dominated by filling and
+    # draining its three-stage pipeline
+    e2e_steps = max(2, min(args.steps, 30))
     for _ in range(e2e_steps):
         e2e_step()
     e1.record(stream)
@@ -400,6 +404,31 @@ def run_gpu(args, w):
     e2e_ms = fa_dist.max_over_ranks(p0.elapsed_time(p1) / e2e_steps, info, device=str(dev))
     e2e_value = fa_dist.aggregate_throughput(f_fwd + f_bwd, e2e_ms * 1e-3, info) / 1e12
     serial_value = fa_dist.aggregate_throughput(f_fwd + f_bwd, serial_ms * 1e-3, info) / 1e12
+
+    # (c) the copy floor of (b): one step's uploads and downloads, both directions at once
+    # on the same streams, with no compute.  No pipelined step can be faster.
+    di0, dout0, ho0 = sets[0]
+
+    def copies():
+        with torch.cuda.stream(s_up):
+            for n, t in di0.items():
+                t.copy_(hin[n], non_blocking=True)
+        with torch.cuda.stream(s_down):
+            for n, t in dout0.items():
+                ho0[n].copy_(t, non_blocking=True)
+
+    copies()
+    torch.cuda.synchronize()
+    c0, c1 = ev(), ev()
+    c0.record(s_up)
+    s_down.wait_event(c0)
+    copy_reps = 5
+    for _ in range(copy_reps):
+        copies()
+    s_down.wait_stream(s_up)
+    c1.record(s_down)
+    torch.cuda.synchronize()
+    copy_ms = fa_dist.max_over_ranks(c0.elapsed_time(c1) / copy_reps, info, device=str(dev))
     del sets
 
     if rank != 0:
@@ -438,6 +467,7 @@ def run_gpu(args, w):
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "mode": "pipelined: uploads, compute and downloads on three streams",
+                "copy_floor_ms": copy_ms, "frac_of_copy_floor": copy_ms / e2e_ms,
                 "serial": {"value": serial_value, "ms_per_step": serial_ms}},
         "gpu_launches": args.steps * (1 + (3 if with_bwd else 0)),
         "clocks": clocks.summary(),
