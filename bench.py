@@ -297,10 +297,14 @@ def run_gpu(args, w):
         kernels[kn[1]] = {"ms": span(2, 3),
                           "bytes": traffic.bwd_prep_bytes(B, H, N, d, 4 if f32 else 2)}
         kernels[kn[2]] = {"ms": span(3, 4), "flops": 8.0 * B * H * N * N * d * half}
-        kernels[kn[3]] = {"ms": span(4, 5), "flops": 2.0 * B * H * N * N * d * half}
+        # credited: the dQ product; executed: the S and dP recomputes as well
+        kernels[kn[3]] = {"ms": span(4, 5), "flops": 2.0 * B * H * N * N * d * half,
+                          "executed_flops": 6.0 * B * H * N * N * d * half}
     for kinfo in kernels.values():
         if "flops" in kinfo:
             kinfo["tflops"] = kinfo["flops"] / (kinfo["ms"] * 1e-3) / 1e12
+        if "executed_flops" in kinfo:
+            kinfo["executed_tflops"] = kinfo["executed_flops"] / (kinfo["ms"] * 1e-3) / 1e12
         else:
             kinfo["gbs"] = kinfo["bytes"] / (kinfo["ms"] * 1e-3) / 1e9
     value = fa_dist.aggregate_throughput(f_fwd + f_bwd, ms * 1e-3, info) / 1e12
@@ -460,6 +464,9 @@ def run_gpu(args, w):
         "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "step_ms_percentiles": step_pct,
         "fwd_tflops": f_fwd / (fwd_ms * 1e-3) / 1e12,
         "bwd_tflops": (f_bwd / (bwd_ms * 1e-3) / 1e12) if with_bwd else None,
+        # tensor-core work the split backward executes (its dQ kernel recomputes S and dP)
+        "bwd_executed_tflops": (traffic.bwd_executed_flops(B, H, N, d, w.causal)
+                                / (bwd_ms * 1e-3) / 1e12) if with_bwd else None,
         "roofline": {"kernel": dom_name, "bound": bound, "achieved": achieved,
                      "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": peak_source, "traffic": recorded_traffic(dom_name)},

@@ -41,6 +41,14 @@ def bwd_flops(B: int, H: int, N: int, d: int, causal: bool) -> float:
     return f / 2 if causal else f
 
 
+def bwd_executed_flops(B: int, H: int, N: int, d: int, causal: bool) -> float:
+    """Tensor-core FLOPs the split backward actually executes: the dK/dV kernel's four
+    products (S, dP, dV, dK) and the dQ kernel's three (S and dP again, then dQ),
+    14 B H N^2 d, halved when causal.  The credited figure (bwd_flops) counts five."""
+    f = 14.0 * B * H * N * N * d
+    return f / 2 if causal else f
+
+
 def visible_pairs(Nq: int, Nk: int, causal: bool) -> float:
     """(query, key) pairs the product covers per head: Nq * Nk, or, causal with the
     queries as the last Nq of the Nk tokens, Nq * Nk - Nq^2 / 2 (the same halving

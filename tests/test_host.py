@@ -25,6 +25,9 @@ def test_flop_convention():
     assert traffic.fwd_flops(1, 1, 2, 3, False) == 4 * 4 * 3
     assert traffic.fwd_flops(2, 16, 8192, 128, True) == 2 * 2 * 16 * 8192 ** 2 * 128
     assert traffic.bwd_flops(2, 16, 8192, 128, True) == 5 * 2 * 16 * 8192 ** 2 * 128
+    # the split backward executes 7 products of 2*N^2*d per head (4 in dK/dV, 3 in dQ)
+    assert traffic.bwd_executed_flops(2, 16, 8192, 128, True) == 7 * 2 * 16 * 8192 ** 2 * 128
+    assert traffic.bwd_executed_flops(1, 1, 4, 2, False) == 7 * 2 * 4 ** 2 * 2
 
 
 def test_flops_with_fewer_queries_than_keys():
