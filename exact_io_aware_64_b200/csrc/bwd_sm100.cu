@@ -24,8 +24,10 @@
 //      stream past through separate rings (3 slots for K, which the last product of a
 //      tile still reads, 2 for V):  S = Q_i K_j^T, dP = dO_i V_j^T, P, dS as above,
 //      dQ_i += dS K_j.
-//      TMEM: dQ | S | dP | dS.  dS has its own region, so S(j+1) and dP(j+1) are issued
-//      as soon as the element-wise warps have read S(j) and dP(j), ahead of dQ(j).
+//      TMEM: dQ | S | dP (dS over it) | Q_i | dO_i.  The element-wise warps copy the
+//      unit's Q_i and dO_i into tensor memory once, so the S and dP products read only
+//      K_j or V_j from shared memory: one SS product alone already uses the whole
+//      shared-memory bandwidth, and the TMA writes of the incoming tiles share it.
 //
 // Both tensor-core kernels are persistent (one CTA per SM) with 384 threads: warps 0-7
 // are two element-wise warpgroups that split every 128 x 128 tile by columns (group g
@@ -35,7 +37,7 @@
 // each other's TMEM, and the MMA reads the bf16 operand as two 32-column pieces.  The MMA order is chosen so the
 // tensor core works on one product while the element-wise warps build the next operand
 // (dK/dV: S^T(i) dP^T(i) | dV(i) S^T(i+1) | dK(i) dP^T(i+1) | ...;
-//  dQ: S(j) dP(j) | S(j+1) dP(j+1) | dQ(j) | S(j+2) dP(j+2) | dQ(j+1) ...).
+//  dQ: S(j) dP(j) | S(j+1) dQ(j) dP(j+1) | S(j+2) dQ(j+1) dP(j+2) | ...).
 // Causal work units are ordered heaviest first.
 #include <cstdint>
 
@@ -629,7 +631,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ------------------------------------------------------------------ 3. dQ
 template <int D>
 struct DqLayout {
-  // Q_i and dO_i stay for the whole unit; K_j and V_j stream through separate rings.
+  // Q_i and dO_i arrive once per unit and are copied into tensor memory, where the S and
+  // dP products read them (so those products read only K_j or V_j from shared memory);
+  // their shared-memory slot is then free for the next unit's tiles.  K_j and V_j stream
+  // through separate rings.
   // K_j is read until the dQ product of its tile, V_j only by the dP product, so K gets
   // one more slot: both are then loaded a tile and a half before they are needed.
   static constexpr int kTileBytes = kTile * D * 2;
@@ -653,9 +658,8 @@ struct DqLayout {
   static constexpr int kBarAccFull = kBarSFull + 4;
   static constexpr int kBarAccFree = kBarSFull + 5;
   static constexpr int kBarDrain = kBarSFull + 6;
-  static constexpr int kBarDPFree = kBarSFull + 7;   // element-wise warps have read dP
-  static constexpr int kBarDQDone = kBarSFull + 8;   // the dQ product has read dS
-  static constexpr int kNumBars = kBarDQDone + 1;
+  static constexpr int kBarQTmem = kBarSFull + 7;   // this unit's Q, dO are in TMEM
+  static constexpr int kNumBars = kBarQTmem + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kAlloc = kMisc + 16 + 1024;
   static_assert(kAlloc <= 232448, "shared memory over the 227 KB per-block limit");
@@ -692,7 +696,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     mbar_init(bar(L::kBarQFull), 1);
-    mbar_init(bar(L::kBarQEmpty), 1);
+    mbar_init(bar(L::kBarQEmpty), kEw / 32);  // the element-wise warps, once copied
     for (int s = 0; s < L::kKStages; ++s) {
       mbar_init(bar(L::kBarKFull + s), 1);
       mbar_init(bar(L::kBarKEmpty + s), 1);
@@ -708,8 +712,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(L::kBarAccFull), 1);
     mbar_init(bar(L::kBarAccFree), kEw / 32);
     mbar_init(bar(L::kBarDrain), 1);
-    mbar_init(bar(L::kBarDPFree), kEw / 32);
-    mbar_init(bar(L::kBarDQDone), 1);
+    mbar_init(bar(L::kBarQTmem), kEw / 32);
     fence_mbar_init();
   }
   if (warp == kWarpMMA) {
@@ -720,9 +723,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // dS has a region of its own (rather than overwriting dP), so the next tile's S and
-  // dP products can start as soon as the element-wise warps have read this tile's.
-  const uint32_t tdQ = tmem, tS = tmem + 128, tdP = tmem + 256, tdS = tmem + 384;
+  // dQ | S | dP (dS written over the columns each group has read, as bf16) | Q | dO.
+  // Q and dO (bf16, one 32-bit column per pair of elements) are the A operands of the
+  // S and dP products for the whole unit.
+  const uint32_t tdQ = tmem, tS = tmem + 128, tdP = tmem + 256, tQt = tmem + 384,
+                 tdOt = tmem + 384 + D / 2;
 
   // unit w: query tile i of head bh, meeting key tiles 0 .. m - 1 of its sequence
   // (m = 0: the tile lies past the sequence's queries, or the sequence has no keys)
@@ -808,22 +813,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the whole warp runs the loop so descriptors stay warp-uniform; one elected lane
     // issues each tcgen05 instruction
     {
-      constexpr uint32_t idSS = idesc_bf16_f32(kTile, false);
+      constexpr uint32_t idS = idesc_bf16_f32(kTile, false);  // B K-major, N = 128 keys
       constexpr uint32_t idTS = idesc_bf16_f32(D, true);
-      const uint64_t dQd = desc_kmajor(base + L::kQ);
-      const uint64_t ddO = desc_kmajor(base + L::kDO);
       int kc = 0, vc = 0, units = 0, sfree_cnt = 0, ds_cnt = 0;
       uint32_t kcph = 0, vcph = 0;
       bool ok = true;
       auto kslot = [&](int s) { return base + L::kK0 + s * L::kTileBytes; };
       auto vslot = [&](int s) { return base + L::kV0 + s * L::kTileBytes; };
-      // S = Q K^T or dP = dO V^T: both operands K-major, K extent = D
-      auto issue_ss = [&](uint32_t dtm, uint64_t da, uint32_t b_saddr, uint32_t done_bar) {
+      // S = Q K^T or dP = dO V^T: A (this unit's Q or dO, K extent = D) from tensor
+      // memory, B (K_j or V_j) K-major from shared memory
+      auto issue_qk = [&](uint32_t dtm, uint32_t a_tmem, uint32_t b_saddr, uint32_t done_bar) {
         const uint64_t db = desc_kmajor(b_saddr);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = ((kk / 4) * L::kBoxBytes + (kk % 4) * 32) >> 4;
-          mma_ss_elect(dtm, da + off, db + off, idSS, kk > 0 ? 1u : 0u);
+          mma_ts_elect(dtm, a_tmem + kk * 8, db + off, idS, kk > 0 ? 1u : 0u);
         }
         mma_commit_elect(done_bar);
       };
@@ -831,12 +835,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_dp = [&]() -> bool {
         if (!wait_warp(bar(L::kBarVFull + vc), vcph)) return false;
         tc_fence_after();
-        issue_ss(tdP, ddO, vslot(vc), bar(L::kBarDPFull));
+        issue_qk(tdP, tdOt, vslot(vc), bar(L::kBarDPFull));
         mma_commit_elect(bar(L::kBarVEmpty + vc));
         if (++vc == L::kVStages) vc = 0, vcph ^= 1;
         return true;
       };
-      int dpfree_cnt = 0;
       int live = 0;
       for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
          w = snake_unit(++r), units += live) {
@@ -844,15 +847,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         unit(w, bh, i, m, lq, lk, off, tq0, tk0);
         live = m > 0;
         if (!live) continue;
-        ok = wait_warp(bar(L::kBarQFull), units & 1);
+        ok = wait_warp(bar(L::kBarQTmem), units & 1);
         if (ok) ok = wait_warp(bar(L::kBarKFull + kc), kcph);
         if (!ok) break;
         tc_fence_after();
         int cur = kc;
         if (++kc == L::kKStages) kc = 0, kcph ^= 1;
-        issue_ss(tS, dQd, kslot(cur), bar(L::kBarSFull));
+        issue_qk(tS, tQt, kslot(cur), bar(L::kBarSFull));
         ok = issue_dp();
         if (!ok) break;
+        // per tile t: S(t+1) | dQ(t) | dP(t+1).  dS(t) lies over the dP region, so dP(t+1)
+        // is issued after the dQ(t) product that reads it (the tensor pipe executes
+        // products in issue order).
         for (int t = 0; t < m; ++t) {
           int nxt = -1;
           if (t + 1 < m) {
@@ -864,14 +870,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             nxt = kc;
             if (++kc == L::kKStages) kc = 0, kcph ^= 1;
             tc_fence_after();
-            issue_ss(tS, dQd, kslot(nxt), bar(L::kBarSFull));
-            // dP(t+1) once they hold dP(t)
-            ok = wait_warp(bar(L::kBarDPFree), dpfree_cnt & 1);
-            if (!ok) break;
-            ++dpfree_cnt;
-            tc_fence_after();
-            ok = issue_dp();
-            if (!ok) break;
+            issue_qk(tS, tQt, kslot(nxt), bar(L::kBarSFull));
           }
           ok = wait_warp(bar(L::kBarDSReady), ds_cnt & 1);
           if (ok && t == 0 && units > 0) ok = wait_warp(bar(L::kBarAccFree), (units - 1) & 1);
@@ -882,21 +881,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t db = desc_mnmajor(kslot(cur), L::kBoxBytes);
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
-            mma_ts_elect(tdQ, split_operand_col(tdS, kk), db + static_cast<uint64_t>((kk * 2048) >> 4),
+            mma_ts_elect(tdQ, split_operand_col(tdP, kk), db + static_cast<uint64_t>((kk * 2048) >> 4),
                          idTS, (t > 0 || kk > 0) ? 1u : 0u);
           mma_commit_elect(bar(L::kBarKEmpty + cur));
-          mma_commit_elect(bar(L::kBarDQDone));
+          if (t + 1 < m) {
+            ok = issue_dp();
+            if (!ok) break;
+          }
           if (nxt >= 0) cur = nxt;
         }
         if (!ok) break;
-        // the unit's last S and dP tiles were read by the element-wise warps: consume
-        // those signals before the next unit overwrites the regions
+        // the unit's last S tile was read by the element-wise warps: consume that signal
+        // before the next unit overwrites the region
         ok = wait_warp(bar(L::kBarSFree), sfree_cnt & 1);
-        if (ok) ok = wait_warp(bar(L::kBarDPFree), dpfree_cnt & 1);
         if (!ok) break;
         ++sfree_cnt;
-        ++dpfree_cnt;
-        mma_commit_elect(bar(L::kBarQEmpty));
         mma_commit_elect(bar(L::kBarAccFull));
       }
       mma_commit_elect(bar(L::kBarDrain));
@@ -908,7 +907,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int col0 = g * kCols;        // first tile column (key) of this group
     const int row = (warp % 4) * 32 + lane;  // query row within the tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp % 4) * 32) << 16;
-    int units = 0, s_cnt = 0, dp_cnt = 0, dq_cnt = 0;
+    int units = 0, s_cnt = 0, dp_cnt = 0;
     bool ok = true;
     int live = 0;
     for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
@@ -917,6 +916,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       unit(w, bh, i, m, lq, lk, off, tq0, tk0);
       live = m > 0;
       if (!live) continue;
+      // This unit's Q and dO rows into tensor memory: thread = query row = TMEM lane;
+      // group g copies the d-columns [g*D/2, (g+1)*D/2), one 32-bit column per pair of
+      // bf16 elements.  The tiles sit in shared memory as 64-column boxes with the
+      // 128-byte swizzle (16-byte chunk c of row r stored at chunk c ^ (r % 8)).  Every
+      // product of the previous unit has completed (its dQ accumulator was drained), so
+      // nothing still reads these TMEM columns.
+      ok = wait_warp(bar(L::kBarQFull), units & 1);
+      if (!ok) break;
+      {
+        constexpr int kChunks = D / 16;  // 16-byte chunks per group
+        uint32_t vq[D / 4], vo[D / 4];
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) {
+          const int J = g * kChunks + c;  // chunk of the whole row
+          const uint32_t at = (J / 8) * L::kBoxBytes + row * 128 + (((J % 8) ^ (row & 7)) * 16);
+          const uint4 a = *reinterpret_cast<const uint4*>(smem + L::kQ + at);
+          const uint4 b = *reinterpret_cast<const uint4*>(smem + L::kDO + at);
+          vq[4 * c] = a.x, vq[4 * c + 1] = a.y, vq[4 * c + 2] = a.z, vq[4 * c + 3] = a.w;
+          vo[4 * c] = b.x, vo[4 * c + 1] = b.y, vo[4 * c + 2] = b.z, vo[4 * c + 3] = b.w;
+        }
+        if constexpr (D == 128) {
+          tmem_st32(tQt + lane_off + g * 32, vq);
+          tmem_st32(tdOt + lane_off + g * 32, vo);
+        } else {
+          tmem_st16(tQt + lane_off + g * 16, vq);
+          tmem_st16(tdOt + lane_off + g * 16, vo);
+        }
+        tmem_wait_st();
+      }
+      warp_arrive(bar(L::kBarQTmem));   // the S and dP products may read them
+      warp_arrive(bar(L::kBarQEmpty));  // the next unit's tiles may be loaded
       const int q_row = i * kTile + row;
       const size_t prow = static_cast<size_t>(bh) * args.Npad + q_row;  // q_row < Npad
       const float nl2row = args.L2pad[prow];   // -LSE * log2(e) of this query row
@@ -964,7 +994,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < kCols / 32; ++c) tmem_ld32(tdP + lane_off + col0 + c * 32, &dpv[c * 32]);
         tmem_wait_ld();
-        warp_arrive(bar(L::kBarDPFree));  // dP(t+1) may now be written over it
         uint32_t pk[kCols / 2];
         const uint64_t nd2 = f32x2(ndrow, ndrow);
 #pragma unroll
@@ -976,14 +1005,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                       ds0, ds1);
           pk[k] = pack_bf16x2(ds0, ds1);
         }
-        // the previous tile's dQ product must have read the dS region before it is reused
-        if (dq_cnt > 0) {
-          ok = wait_warp(bar(L::kBarDQDone), (dq_cnt - 1) & 1);
-          if (!ok) break;
-        }
-        ++dq_cnt;
-        tc_fence_after();
-        tmem_st32(tdS + lane_off + col0, pk);  // this group's 32-column piece of dS
+        // this group's 32-column piece of dS, over dP columns it has just read
+        tmem_st32(tdP + lane_off + col0, pk);
         tmem_wait_st();
         warp_arrive(bar(L::kBarDSReady));
       }
