@@ -95,6 +95,21 @@ def recorded_traffic(kernel: str):
     return e.get("bytes_per_launch")
 
 
+def add_rates(kernels: dict) -> dict:
+    """Per-kernel rates from mean launch times: TFLOP/s for kernels credited with FLOPs
+    (and executed TFLOP/s where the executed work differs), GB/s for the ones credited
+    with bytes."""
+    for kinfo in kernels.values():
+        sec = kinfo["ms"] * 1e-3
+        if "flops" in kinfo:
+            kinfo["tflops"] = kinfo["flops"] / sec / 1e12
+        else:
+            kinfo["gbs"] = kinfo["bytes"] / sec / 1e9
+        if "executed_flops" in kinfo:
+            kinfo["executed_tflops"] = kinfo["executed_flops"] / sec / 1e12
+    return kernels
+
+
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -300,13 +315,7 @@ def run_gpu(args, w):
         # credited: the dQ product; executed: the S and dP recomputes as well
         kernels[kn[3]] = {"ms": span(4, 5), "flops": 2.0 * B * H * N * N * d * half,
                           "executed_flops": 6.0 * B * H * N * N * d * half}
-    for kinfo in kernels.values():
-        if "flops" in kinfo:
-            kinfo["tflops"] = kinfo["flops"] / (kinfo["ms"] * 1e-3) / 1e12
-        if "executed_flops" in kinfo:
-            kinfo["executed_tflops"] = kinfo["executed_flops"] / (kinfo["ms"] * 1e-3) / 1e12
-        else:
-            kinfo["gbs"] = kinfo["bytes"] / (kinfo["ms"] * 1e-3) / 1e9
+    add_rates(kernels)
     value = fa_dist.aggregate_throughput(f_fwd + f_bwd, ms * 1e-3, info) / 1e12
 
     # ---- end to end through the public API with host buffers

@@ -30,3 +30,19 @@ def test_reference_arm_under_torchrun():
     assert line["impl"] == "reference" and line["unit"] == "TFLOP/s"
     assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
     assert line["config"]["workload"] == "n4096_d64"
+
+
+def test_per_kernel_rates():
+    """The bench line's per-kernel figures: TFLOP/s for FLOP-credited kernels, GB/s for
+    the bandwidth-bound preparation, executed TFLOP/s beside the credited figure."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    k = bench.add_rates({"fwd": {"ms": 0.5, "flops": 1e12},
+                         "prep": {"ms": 0.04, "bytes": 1.4e8},
+                         "dq": {"ms": 0.8, "flops": 2.75e11, "executed_flops": 8.25e11}})
+    assert abs(k["fwd"]["tflops"] - 2000.0) < 1e-9 and "gbs" not in k["fwd"]
+    assert abs(k["prep"]["gbs"] - 3500.0) < 1e-9 and "tflops" not in k["prep"]
+    assert abs(k["dq"]["tflops"] - 343.75) < 1e-9
+    assert abs(k["dq"]["executed_tflops"] - 1031.25) < 1e-9
