@@ -20,8 +20,9 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libfa.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
 
-SOURCES = ["fa_api.cu", "fwd_sm100.cu", "fwd_f32.cu", "bwd_sm100.cu", "bwd_f32.cu", "merge.cu", "selftest.cu"]
-HEADERS = ["sm100.cuh", "internal.h"]
+SOURCES = ["fa_api.cu", "fwd_sm100.cu", "fwd_f32.cu", "bwd_sm100.cu", "bwd_f32.cu", "merge.cu", "selftest.cu",
+           "zero_rows.cu"]
+HEADERS = ["sm100.cuh", "internal.h", "f32_seq.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [

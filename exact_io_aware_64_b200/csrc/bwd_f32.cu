@@ -101,12 +101,22 @@ __global__ void __launch_bounds__(F32Shape<D>::kThreads)
   const int bh = blockIdx.x / tiles;
   const int tile = blockIdx.x % tiles;
   const F32Seq sq = f32_seq(p, bh, D, threadIdx.x == 0);
-  // past the sequence's keys, or no queries (then its key rows are not written either)
-  if (tile * kRows >= sq.lk || sq.lq == 0) return;
+  if (tile * kRows >= sq.lk) return;  // past the sequence's keys
   const int r = threadIdx.x / TPR;
   const int part = threadIdx.x % TPR;
   const int key = tile * kRows + r;
   const bool valid = key < sq.lk;
+  if (sq.lq == 0) {
+    // keys without queries: no query sees them, so their gradients are exactly zero
+    if (valid)
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const size_t at = sq.k0 + static_cast<size_t>(key) * sq.rs + TPR * e + part;
+        dK[at] = 0.f;
+        dV[at] = 0.f;
+      }
+    return;
+  }
 
   float k[E], v[E], dk[E], dv[E];
 #pragma unroll

@@ -159,6 +159,10 @@ bool overlaps(const void* a, size_t a_bytes, const void* b, size_t b_bytes) {
   return x < y + b_bytes && y < x + a_bytes;
 }
 
+// Longest sequence any call accepts: every length rounded up to whole 256-row units
+// still fits a 32-bit int.
+constexpr int kMaxRows = 0x7fffffff - 255;
+
 // Checks shared by every call: Nq query rows and Nk key rows per head (Nk == Nq for
 // the entry points without the _qk suffix).  Sets *noop when there is nothing to
 // compute.
@@ -173,10 +177,15 @@ fa_status check_common(int B, int H, int Nq, int Nk, int d, float scale, int cau
     return fail(FA_ERR_INVALID_ARG, "scale must be finite and positive");
   if (causal != 0 && causal != 1) return fail(FA_ERR_INVALID_ARG, "causal must be 0 or 1");
   const long long bh = static_cast<long long>(B) * H;
-  // work units and row indices are 32-bit on the device
-  for (const int n : {Nq, Nk})
-    if (bh > 0 && n > 0 && (bh > (1ll << 31) / ((n + 255) / 256) || bh * n >= (1ll << 31)))
+  // work units and row indices are 32-bit on the device, and lengths are rounded up to
+  // whole 256-row units in 32-bit arithmetic there
+  for (const int n : {Nq, Nk}) {
+    if (n > kMaxRows)
+      return fail(FA_ERR_INVALID_ARG, "N = %d rows is too large (at most %d)", n, kMaxRows);
+    const long long units = (static_cast<long long>(n) + 255) / 256;
+    if (bh > 0 && n > 0 && (bh > (1ll << 31) / units || bh * n >= (1ll << 31)))
       return fail(FA_ERR_INVALID_ARG, "B*H*N = %lld rows is too large", bh * n);
+  }
   *noop = (bh == 0 || Nq == 0);
   if (*noop) return FA_OK;
   if (Nk == 0) return fail(FA_ERR_INVALID_ARG, "queries need at least one key (Nk=0)");
@@ -296,6 +305,26 @@ fa_status check_seqlens(const int* seqlens_q, const int* seqlens_k) {
   return FA_OK;
 }
 
+// A backward call with keys but no query rows (Nq == 0, or no query tokens in the
+// packed layout): no query sees any key, so dK and dV are exactly zero in every key row
+// of every sequence; rows past a sequence's key length stay unwritten as elsewhere.
+// Its arguments are checked (check_key_grads) before the device is queried.
+fa_status check_key_grads(const void* dK, const void* dV, size_t key_bytes) {
+  FA_TRY(check_ptr(dK, "dK"));
+  FA_TRY(check_ptr(dV, "dV"));
+  if (overlaps(dK, key_bytes, dV, key_bytes))
+    return fail(FA_ERR_INVALID_ARG, "gradients overlap each other");
+  return FA_OK;
+}
+
+fa_status zero_key_grads(void* dK, void* dV, const fa::Problem& p, size_t elem,
+                         const DeviceInfo& dev, cudaStream_t stream) {
+  cudaError_t e = fa::launch_zero_key_rows(dK, dV, p, static_cast<int>(elem), dev.num_sms,
+                                           stream);
+  if (e != cudaSuccess) return cuda_fail(e, "launching the key-gradient zero fill");
+  return FA_OK;
+}
+
 fa_status fwd_impl(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
                    int H, int Nq, int Nk, int d, float scale, int causal, cudaStream_t stream,
                    const int* seqlens_q = nullptr, const int* seqlens_k = nullptr) {
@@ -326,7 +355,17 @@ fa_status bwd_impl(const void* Q, const void* K, const void* V, const void* O, c
   bool noop = false;
   FA_TRY(check_bwd_args(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, Nq, Nk, d, scale, causal,
                         workspace, workspace_bytes, 2, &noop));
-  if (noop) return FA_OK;  // empty problem: the pointers are never used (may be NULL)
+  if (noop) {
+    // no work, and then no pointer is used (they may be NULL) -- unless there are keys
+    // without queries, whose gradients are zeros to be written
+    if (static_cast<long long>(B) * H == 0 || Nk == 0) return FA_OK;
+    FA_TRY(check_key_grads(dK, dV, static_cast<size_t>(B) * H * Nk * d * 2));
+    DeviceInfo dev;
+    FA_TRY(device_info(&dev));
+    const fa::Problem p = make_problem(B, H, Nq, Nk, d, scale, causal, dev, seqlens_q,
+                                       seqlens_k);
+    return zero_key_grads(dK, dV, p, 2, dev, stream);
+  }
   DeviceInfo dev;
   FA_TRY(device_info(&dev));
   FA_TRY(require_sm100(dev));
@@ -336,7 +375,7 @@ fa_status bwd_impl(const void* Q, const void* K, const void* V, const void* O, c
   FA_TRY(make_tmap(&tmK, K, BH, Nk, d));
   FA_TRY(make_tmap(&tmV, V, BH, Nk, d));
   FA_TRY(make_tmap(&tmdO, dO, BH, Nq, d));
-  const int Npad = fa::bwd_padded_rows(Nq);
+  const int Npad = static_cast<int>(fa::bwd_padded_rows(Nq));  // Nq <= kMaxRows
   float* ws = static_cast<float*>(workspace);
   FA_TRY(make_row_tmap(&tmD, ws, BH, Npad));
   FA_TRY(make_row_tmap(&tmL2, ws + static_cast<size_t>(BH) * Npad, BH, Npad));
@@ -344,6 +383,15 @@ fa_status bwd_impl(const void* Q, const void* K, const void* V, const void* O, c
   cudaError_t e = fa::launch_bwd_sm100(tmQ, tmK, tmV, tmdO, tmL2, tmD, O, dO, LSE, dQ, dK, dV,
                                        ws, p, dev.num_sms, stream);
   if (e != cudaSuccess) return cuda_fail(e, "launching the backward kernels");
+  return FA_OK;
+}
+
+// The start-token arrays of the packed-layout calls: both given, 4-byte aligned.
+fa_status check_cu(const int* cu_q, const int* cu_k) {
+  if (cu_q == nullptr || cu_k == nullptr)
+    return fail(FA_ERR_INVALID_ARG, "cu_seqlens_q and cu_seqlens_k are required");
+  if ((reinterpret_cast<uintptr_t>(cu_q) | reinterpret_cast<uintptr_t>(cu_k)) & 3u)
+    return fail(FA_ERR_INVALID_ARG, "cu_seqlens_q and cu_seqlens_k must be 4-byte aligned");
   return FA_OK;
 }
 
@@ -360,11 +408,7 @@ fa_status check_packed(const int* cu_q, const int* cu_k, int B, int H, int max_q
     *noop = true;
     return FA_OK;
   }
-  if (cu_q == nullptr || cu_k == nullptr)
-    return fail(FA_ERR_INVALID_ARG, "cu_seqlens_q and cu_seqlens_k are required");
-  if ((reinterpret_cast<uintptr_t>(cu_q) | reinterpret_cast<uintptr_t>(cu_k)) & 3u)
-    return fail(FA_ERR_INVALID_ARG, "cu_seqlens_q and cu_seqlens_k must be 4-byte aligned");
-  return FA_OK;
+  return check_cu(cu_q, cu_k);
 }
 
 // Pointer and overlap checks of the packed-layout forward calls (elem = bytes per
@@ -451,7 +495,16 @@ fa_status bwd_f32_impl(const float* Q, const float* K, const float* V, const flo
   bool noop = false;
   FA_TRY(check_bwd_args(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, Nq, Nk, d, scale, causal,
                         workspace, workspace_bytes, 4, &noop));
-  if (noop) return FA_OK;  // empty problem: the pointers are never used (may be NULL)
+  if (noop) {
+    // as in bwd_impl: keys without queries get zero gradients
+    if (static_cast<long long>(B) * H == 0 || Nk == 0) return FA_OK;
+    FA_TRY(check_key_grads(dK, dV, static_cast<size_t>(B) * H * Nk * d * 4));
+    DeviceInfo dev;
+    FA_TRY(device_info(&dev));
+    const fa::Problem p = make_problem(B, H, Nq, Nk, d, scale, causal, dev, seqlens_q,
+                                       seqlens_k);
+    return zero_key_grads(dK, dV, p, 4, dev, stream);
+  }
   DeviceInfo dev;
   FA_TRY(device_info(&dev));
   const fa::Problem p = make_problem(B, H, Nq, Nk, d, scale, causal, dev, seqlens_q, seqlens_k);
@@ -545,7 +598,18 @@ fa_status fa_bwd_packed(const void* Q, const void* K, const void* V, const void*
   bool noop = false;
   FA_TRY(check_packed(cu_seqlens_q, cu_seqlens_k, B, H, max_seqlen_q, max_seqlen_k, total_q,
                       total_k, d, scale, causal, &noop));
-  if (noop) return FA_OK;
+  if (noop) {
+    // keys without queries get zero gradients (see bwd_impl)
+    if (static_cast<long long>(B) * H == 0 || total_k == 0 || max_seqlen_k == 0) return FA_OK;
+    FA_TRY(check_cu(cu_seqlens_q, cu_seqlens_k));
+    FA_TRY(check_key_grads(dK, dV, static_cast<size_t>(total_k) * H * d * 2));
+    DeviceInfo dev;
+    FA_TRY(device_info(&dev));
+    const fa::Problem p = make_problem(B, H, max_seqlen_q, max_seqlen_k, d, scale, causal, dev,
+                                       nullptr, nullptr, cu_seqlens_q, cu_seqlens_k, total_q,
+                                       total_k);
+    return zero_key_grads(dK, dV, p, 2, dev, stream);
+  }
   const size_t need = fa_bwd_workspace_bytes(B, H, max_seqlen_q, d);
   FA_TRY(check_packed_bwd_ptrs(Q, K, V, O, dO, LSE, dQ, dK, dV, H, d, total_q, total_k,
                                workspace, need, workspace_bytes, 2));
@@ -558,7 +622,7 @@ fa_status fa_bwd_packed(const void* Q, const void* K, const void* V, const void*
   FA_TRY(make_tmap_packed(&tmK, K, total_k, H, d));
   FA_TRY(make_tmap_packed(&tmV, V, total_k, H, d));
   FA_TRY(make_tmap_packed(&tmdO, dO, total_q, H, d));
-  const int Npad = fa::bwd_padded_rows(max_seqlen_q);
+  const int Npad = static_cast<int>(fa::bwd_padded_rows(max_seqlen_q));
   float* ws = static_cast<float*>(workspace);
   FA_TRY(make_row_tmap(&tmD, ws, BH, Npad));
   FA_TRY(make_row_tmap(&tmL2, ws + static_cast<size_t>(BH) * Npad, BH, Npad));
@@ -618,7 +682,8 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
   (void)d;
   if (B <= 0 || H <= 0 || N <= 0) return 0;
   // D and LSE*log2(e), one float each per query row, rows padded to whole 128-row tiles
-  const size_t raw = 2 * static_cast<size_t>(B) * H * fa::bwd_padded_rows(N) * sizeof(float);
+  const size_t raw = 2 * static_cast<size_t>(B) * H *
+                    static_cast<size_t>(fa::bwd_padded_rows(N)) * sizeof(float);
   return (raw + 255) / 256 * 256;
 }
 
@@ -644,7 +709,7 @@ fa_status fa_bwd_varlen(const void* Q, const void* K, const void* V, const void*
                         int Nk, int d, float scale, int causal, void* workspace,
                         size_t workspace_bytes, cudaStream_t stream) {
   g_last_error[0] = '\0';
-  if (B > 0 && H > 0 && Nq > 0) FA_TRY(check_seqlens(seqlens_q, seqlens_k));
+  if (B > 0 && H > 0 && (Nq > 0 || Nk > 0)) FA_TRY(check_seqlens(seqlens_q, seqlens_k));
   return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, Nq, Nk, d, scale, causal, workspace,
                   workspace_bytes, stream, seqlens_q, seqlens_k);
 }
@@ -671,7 +736,7 @@ fa_status fa_bwd_f32_varlen(const float* Q, const float* K, const float* V, cons
                             int H, int Nq, int Nk, int d, float scale, int causal,
                             void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   g_last_error[0] = '\0';
-  if (B > 0 && H > 0 && Nq > 0) FA_TRY(check_seqlens(seqlens_q, seqlens_k));
+  if (B > 0 && H > 0 && (Nq > 0 || Nk > 0)) FA_TRY(check_seqlens(seqlens_q, seqlens_k));
   return bwd_f32_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, Nq, Nk, d, scale, causal,
                       workspace, workspace_bytes, stream, seqlens_q, seqlens_k);
 }
@@ -686,7 +751,18 @@ fa_status fa_bwd_f32_packed(const float* Q, const float* K, const float* V, cons
   bool noop = false;
   FA_TRY(check_packed(cu_seqlens_q, cu_seqlens_k, B, H, max_seqlen_q, max_seqlen_k, total_q,
                       total_k, d, scale, causal, &noop));
-  if (noop) return FA_OK;
+  if (noop) {
+    // keys without queries get zero gradients (see bwd_impl)
+    if (static_cast<long long>(B) * H == 0 || total_k == 0 || max_seqlen_k == 0) return FA_OK;
+    FA_TRY(check_cu(cu_seqlens_q, cu_seqlens_k));
+    FA_TRY(check_key_grads(dK, dV, static_cast<size_t>(total_k) * H * d * 4));
+    DeviceInfo dev;
+    FA_TRY(device_info(&dev));
+    const fa::Problem p = make_problem(B, H, max_seqlen_q, max_seqlen_k, d, scale, causal, dev,
+                                       nullptr, nullptr, cu_seqlens_q, cu_seqlens_k, total_q,
+                                       total_k);
+    return zero_key_grads(dK, dV, p, 4, dev, stream);
+  }
   const size_t need = fa_bwd_workspace_bytes(B, H, max_seqlen_q, d);
   FA_TRY(check_packed_bwd_ptrs(Q, K, V, O, dO, LSE, dQ, dK, dV, H, d, total_q, total_k,
                                workspace, need, workspace_bytes, 4));
@@ -848,19 +924,18 @@ fa_status fa_bwd_noalloc(const void* Q, const void* K, const void* V, const void
                          int B, int H, int N, int d, float scale, int causal,
                          cudaStream_t stream) {
   g_last_error[0] = '\0';
-  if (B > 0 && H > 0 && N > 0) {
-    const size_t need = fa_bwd_workspace_bytes(B, H, N, d);
-    if (need > kNoAllocScratchBytes)
-      return fail(FA_ERR_INVALID_ARG,
-                  "fa_bwd_noalloc: B=%d H=%d N=%d needs %zu bytes of scratch, more than the "
-                  "library's fixed %zu (B*H*ceil(N/128)*128 must be at most %zu); use fa_bwd "
-                  "with a workspace",
-                  B, H, N, need, kNoAllocScratchBytes, kNoAllocScratchBytes / 8);
-  }
   void* scratch = nullptr;
   bool noop = false;
+  // sizes first: the scratch arithmetic below assumes validated sizes
   fa_status st = check_common(B, H, N, N, d, scale, causal, &noop);
   if (st != FA_OK || noop) return st;
+  const size_t need = fa_bwd_workspace_bytes(B, H, N, d);
+  if (need > kNoAllocScratchBytes)
+    return fail(FA_ERR_INVALID_ARG,
+                "fa_bwd_noalloc: B=%d H=%d N=%d needs %zu bytes of scratch, more than the "
+                "library's fixed %zu (B*H*ceil(N/128)*128 must be at most %zu); use fa_bwd "
+                "with a workspace",
+                B, H, N, need, kNoAllocScratchBytes, kNoAllocScratchBytes / 8);
   st = noalloc_scratch(&scratch);
   if (st != FA_OK) return st;
   return fa_bwd(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, scale, causal, scratch,

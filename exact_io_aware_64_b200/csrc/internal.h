@@ -57,7 +57,7 @@ cudaError_t launch_fwd_f32(const float* Q, const float* K, const float* V, float
 // then dK/dV, then dQ.  Workspace layout: -D as [BH][Npad] float, then -L2 as [BH][Npad]
 // float, Npad = bwd_padded_rows(N).  tmL2 / tmD describe those two arrays as 3-D
 // [1][BH][Npad] float tensors with 128 x 1 x 1 boxes.
-int bwd_padded_rows(int N);
+long long bwd_padded_rows(long long N);
 cudaError_t launch_bwd_sm100(const CUtensorMap& tmQ, const CUtensorMap& tmK,
                              const CUtensorMap& tmV, const CUtensorMap& tmdO,
                              const CUtensorMap& tmL2, const CUtensorMap& tmD, const void* O,
@@ -70,6 +70,12 @@ cudaError_t launch_bwd_sm100(const CUtensorMap& tmQ, const CUtensorMap& tmK,
 cudaError_t launch_bwd_f32(const float* Q, const float* K, const float* V, const float* O,
                            const float* dO, const float* LSE, float* dQ, float* dK, float* dV,
                            float* workspace, const Problem& p, cudaStream_t stream);
+
+// Zeros in rows [0, lk) of dK and dV for every sequence with no queries (lq == 0);
+// elem_bytes is 2 (bf16) or 4 (float32).  For calls with keys and no query rows at all,
+// where the backward kernels have nothing to run over.
+cudaError_t launch_zero_key_rows(void* dK, void* dV, const Problem& p, int elem_bytes,
+                                 int num_sms, cudaStream_t stream);
 
 // Merge of a partial attention result (O_part bf16, LSE_part) into a float32 accumulator
 // (O_acc, LSE_acc), optionally writing the merged O as bf16 to O_out; [BH][N] rows.

@@ -50,7 +50,9 @@
  *   the calling thread's most recent failed call.
  *
  * N == 0 (or B*H == 0) is valid and does nothing; the pointers are then not checked
- * (empty tensors may have NULL data pointers).
+ * (empty tensors may have NULL data pointers).  The one exception is a backward call
+ * with keys but no queries, which writes zero key gradients (see fa_bwd_qk).
+ * Lengths above 2^31 - 256 rows are rejected.
  */
 #ifndef FA_H
 #define FA_H
@@ -207,7 +209,9 @@ FA_API fa_status fa_bwd(const void* Q, const void* K, const void* V, const void*
  *   LSE      in : [B,H,Nq] float32 from fa_fwd_qk with the same scale and causal
  *   dQ       out: [B,H,Nq,d] bf16;   dK, dV out: [B,H,Nk,d] bf16
  *   workspace   : fa_bwd_workspace_bytes(B,H,Nq,d) bytes (two floats per query row)
- * Same kernels, rules and errors as fa_bwd (causal needs Nq <= Nk).
+ * Same kernels, rules and errors as fa_bwd (causal needs Nq <= Nk).  With Nq == 0 and
+ * Nk > 0 no query sees any key: dK and dV are set to zero (dK and dV must then be valid,
+ * 16-byte aligned and not overlap; the other pointers are not used and may be NULL).
  */
 FA_API fa_status fa_bwd_qk(const void* Q, const void* K, const void* V, const void* O,
                            const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
@@ -219,8 +223,11 @@ FA_API fa_status fa_bwd_qk(const void* Q, const void* K, const void* V, const vo
  *   Q, O, dO, dQ [B,H,Nq,d] bf16;  K, V, dK, dV [B,H,Nk,d] bf16;  LSE [B,H,Nq] float32
  *   workspace: fa_bwd_workspace_bytes(B,H,Nq,d) bytes
  * Rows past a sequence's lengths (dQ past seqlens_q[b], dK and dV past seqlens_k[b]) are
- * not written.  Padding rows of Q, K, V, O and dO must hold finite values.  Lengths as
- * for fa_fwd_varlen; otherwise as fa_bwd_qk.
+ * not written.  A sequence with keys but no queries (seqlens_q[b] == 0) gets zeros in its
+ * dK and dV rows below seqlens_k[b] (no query sees those keys), also when Nq == 0 (then
+ * only dK, dV and the length arrays are used).  A sequence with queries but no keys is
+ * skipped.  Padding rows of Q, K, V, O and dO must hold finite values.  Lengths as for
+ * fa_fwd_varlen; otherwise as fa_bwd_qk.
  */
 FA_API fa_status fa_bwd_varlen(const void* Q, const void* K, const void* V, const void* O,
                                const void* dO, const float* LSE, void* dQ, void* dK,
@@ -234,7 +241,9 @@ FA_API fa_status fa_bwd_varlen(const void* Q, const void* K, const void* V, cons
  *   Q, O, dO, dQ [total_q, H, d] bf16;  K, V, dK, dV [total_k, H, d] bf16;
  *   LSE [H, total_q] float32
  *   workspace: fa_bwd_workspace_bytes(B, H, max_seqlen_q, d) bytes
- * Otherwise as fa_bwd_varlen.
+ * A sequence with keys but no queries gets zeros in its dK and dV rows, also when the
+ * call has no query tokens at all (total_q == 0 or max_seqlen_q == 0; then only dK, dV
+ * and the start arrays are used).  Otherwise as fa_bwd_varlen.
  */
 FA_API fa_status fa_bwd_packed(const void* Q, const void* K, const void* V, const void* O,
                                const void* dO, const float* LSE, void* dQ, void* dK,
@@ -265,7 +274,8 @@ FA_API fa_status fa_bwd_f32(const float* Q, const float* K, const float* V, cons
  * fa_fwd_f32_packed, with the arguments, layouts, workspace sizes and rules of
  * fa_bwd_qk, fa_bwd_varlen and fa_bwd_packed and float32 tensors.  D goes to the first
  * 4*B*H*Nq (packed: 4*B*H*max_seqlen_q) bytes of the workspace.  Rows past a sequence's
- * lengths are not written.  Otherwise as fa_bwd_f32.
+ * lengths are not written; keys without queries get zero gradients, as in the bf16
+ * calls.  Otherwise as fa_bwd_f32.
  */
 FA_API fa_status fa_bwd_f32_qk(const float* Q, const float* K, const float* V, const float* O,
                                const float* dO, const float* LSE, float* dQ, float* dK,

@@ -170,7 +170,11 @@ def test_qk_validation(lib):
         return lib.fa_bwd_qk(A, B_, C, D_, E, F, G, dk, I, 1, 2, Nq, Nk, 64, 0.1, causal, J,
                              ws_bytes, None)
 
-    assert bwd(0, 3) == binding.FA_OK
+    assert bwd(0, 0) == binding.FA_OK
+    # keys without queries: dK and dV get zeros, so they are checked before the device is
+    assert bwd(0, 3, dk=0) == binding.FA_ERR_INVALID_ARG
+    assert "dK" in lib.fa_last_error_message().decode()
+    assert bwd(0, 3, dk=H_ + 8) == binding.FA_ERR_INVALID_ARG
     assert bwd(5, 3) == binding.FA_ERR_INVALID_ARG
     assert bwd(3, 0) == binding.FA_ERR_INVALID_ARG
     # the workspace is sized by the query rows
