@@ -88,7 +88,7 @@ def test_blockwise_backward_every_rank(causal):
     """The emulated 4-rank ring's backward: block backwards with the global O and LSE,
     accumulated in float32 in the ring's order, give the gradients of attention over the
     whole sequence (with D formed from the bf16 output, as fa_bwd does)."""
-    from parity import assert_bf16_close_scaled
+    from parity import assert_bf16_close_scaled, assert_bwd_exact
     W, B, H, L, d = 4, 1, 2, 384, 128
     ins = inputs.make_inputs(B, H, W * L, d, seed=64, with_dO=True)
     q, k, v, do = (ins[n].cuda() for n in ("Q", "K", "V", "dO"))
@@ -101,14 +101,17 @@ def test_blockwise_backward_every_rank(causal):
     binding.check_device_error()
     O_full = torch.cat(Os, dim=2)
     for h in range(H):
-        ref = oracle.attention_bwd_head(to64(ins["Q"][0, h]), to64(ins["K"][0, h]),
-                                        to64(ins["V"][0, h]), to64(ins["dO"][0, h]), scale,
-                                        causal, O_given=to64(O_full[0, h]))
-        for r in range(W):
-            sl = slice(r * L, (r + 1) * L)
-            for got, rf, name in ((dQs[r], ref[0], "dQ"), (dKs[r], ref[1], "dK"),
-                                  (dVs[r], ref[2], "dV")):
-                assert_bf16_close_scaled(to64(got[0, h]), rf[sl], f"rank {r} {name} h={h}")
+        args = [to64(ins[n][0, h]) for n in ("Q", "K", "V", "dO")]
+        ref = oracle.attention_bwd_head(*args, scale, causal, O_given=to64(O_full[0, h]))
+        exact = oracle.attention_bwd_head(*args, scale, causal)
+        for k_, name, got in ((0, "dQ", dQs), (1, "dK", dKs), (2, "dV", dVs)):
+            for r in range(W):
+                sl = slice(r * L, (r + 1) * L)
+                assert_bf16_close_scaled(to64(got[r][0, h]), ref[k_][sl],
+                                         f"rank {r} {name} h={h}")
+            # the whole sequence (1536 rows) against the exact gradient
+            whole = np.concatenate([to64(got[r][0, h]) for r in range(W)])
+            assert_bwd_exact(whole, exact[k_], f"ring {name} h={h} causal={causal}")
 
 
 def test_accumulate():

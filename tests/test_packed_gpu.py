@@ -8,7 +8,8 @@ import torch
 
 import oracle
 from exact_io_aware_64_b200 import binding, inputs
-from parity import (assert_bf16_close_scaled, assert_lse_close, bf16_max_abs_bound, errors,
+from parity import (EXACT_MIN_ROWS, assert_bf16_close_scaled, assert_bwd_exact,
+                    assert_lse_close, bf16_max_abs_bound, errors,
                     to64)
 
 pytestmark = pytest.mark.gpu
@@ -63,6 +64,8 @@ def test_packed_forward_backward(case, d, causal):
             assert bool((O[qs] == SENTINEL).all()) and bool((dQ[qs] == SENTINEL).all())
             continue
         if nq == 0:
+            # keys no query sees: their gradients are exactly zero
+            assert bool((dK[ks] == 0).all()) and bool((dV[ks] == 0).all()), f"seq {s}"
             continue
         pos = oracle.chunk_positions(nq, nk) if causal else None
         for h in range(H):
@@ -77,6 +80,9 @@ def test_packed_forward_backward(case, d, causal):
             exact = oracle.attention_bwd_head(Qh, Kh, Vh, Gh, scale, causal, q_index=pos)
             for k_, name, got, sl in ((0, "dQ", dQ, qs), (1, "dK", dK, ks), (2, "dV", dV, ks)):
                 g = to64(got[sl, h])
+                if min(nq, nk) >= EXACT_MIN_ROWS:
+                    assert_bwd_exact(g, exact[k_], f"{name} {what}")
+                    continue
                 assert_bf16_close_scaled(g, given[k_], f"{name} {what}")
                 max_abs, _ = errors(g, exact[k_])
                 assert max_abs <= bf16_max_abs_bound(exact[k_]), f"{name} vs exact {what}"

@@ -11,7 +11,8 @@ import torch
 
 import oracle
 from exact_io_aware_64_b200 import binding, inputs
-from parity import (assert_bf16_close_scaled, assert_lse_close, bf16_max_abs_bound, errors,
+from parity import (EXACT_MIN_ROWS, assert_bf16_close_scaled, assert_bwd_exact,
+                    assert_lse_close, bf16_max_abs_bound, errors,
                     to64)
 
 pytestmark = pytest.mark.gpu
@@ -56,6 +57,10 @@ def _check(ins, lq, lk, d, causal, O, LSE, grads):
                 assert bool((grads[0][b, h, nq:] == SENTINEL).all()), f"dQ padding b={b}"
                 assert bool((grads[1][b, h, nk:] == SENTINEL).all()), f"dK padding b={b}"
                 assert bool((grads[2][b, h, nk:] == SENTINEL).all()), f"dV padding b={b}"
+            if grads is not None and nq == 0 and nk > 0:
+                # keys no query sees: their gradients are exactly zero
+                assert bool((grads[1][b, h, :nk] == 0).all()), f"dK of keys without queries b={b}"
+                assert bool((grads[2][b, h, :nk] == 0).all()), f"dV of keys without queries b={b}"
             if nq == 0 or nk == 0:
                 continue
             Q = to64(ins["Q"][b, h, :nq])
@@ -74,6 +79,9 @@ def _check(ins, lq, lk, d, causal, O, LSE, grads):
             exact = oracle.attention_bwd_head(Q, K, V, dO, scale, causal, q_index=pos)
             for k_, name, n in ((0, "dQ", nq), (1, "dK", nk), (2, "dV", nk)):
                 got = to64(grads[k_][b, h, :n])
+                if min(nq, nk) >= EXACT_MIN_ROWS:
+                    assert_bwd_exact(got, exact[k_], f"{name} {what}")
+                    continue
                 assert_bf16_close_scaled(got, given[k_], f"{name} {what}")
                 max_abs, _ = errors(got, exact[k_])
                 assert max_abs <= bf16_max_abs_bound(exact[k_]), f"{name} vs exact {what}"
