@@ -169,6 +169,15 @@ class ClockSampler:
                 "power_w_max": max(power) if power else None}
 
 
+def config_dict(w, with_bwd: bool, world: int) -> dict:
+    """The workload as both arms name it in their JSON line."""
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+            "step": "fa_fwd + fa_bwd" if with_bwd else "fa_fwd",
+            "l2": "inputs larger than L2 (no flush)" if w.B * w.H * w.N * w.d * 2 > (126 << 20)
+            else "inputs smaller than L2 (resident between steps)",
+            "parallelism": f"replicas x{world} (independent heads per GPU)"}
+
+
 def step_flops(w) -> float:
     return traffic.fwd_flops(w.B, w.H, w.N, w.d, w.causal) + \
         traffic.bwd_flops(w.B, w.H, w.N, w.d, w.causal)
@@ -207,6 +216,97 @@ def time_oracle(w, max_seconds: float = 20.0):
     return flops / el / 1e12, int(threads), sample, el
 
 
+# The checked subset of each named workload (the oracle is O(N^2 d) per head in fp64):
+# whole heads, and seeded rows of every head (each output row needs only its own query
+# and the head's keys and values; the backward's dQ rows likewise).
+CHECK_PLAN = {
+    "tiny_f32": {"full_heads": ((0, 0),), "rows": 0},
+    "n4096_d64": {"full_heads": ((0, 0),), "rows": 256},
+    "n4096_d64_causal": {"full_heads": ((0, 0),), "rows": 256},
+    "n10000_d128_causal": {"full_heads": ((0, 31),), "rows": 512},
+    "n32768_d128_causal_sigma3": {"full_heads": (), "rows": 512, "extra_rows": 128},
+    "n8192_d128_causal_bwd": {"full_heads": ((0, 3), (1, 7)), "rows": 256},
+}
+
+
+def parity_check(w, ins, outs, with_bwd):
+    """Errors of the timed run's outputs against the fp64 oracle on the workload's checked
+    subset (CHECK_PLAN), and the oracle's time for that subset on this host, with its
+    extrapolation to the whole problem (by the oracle's executed products).  ins and outs
+    are the device tensors of the run (inputs Q, K, V, dO; outputs O, LSE, dQ, dK, dV)."""
+    import numpy as np
+    import oracle
+    plan = CHECK_PLAN[w.name]
+    f64 = lambda t: t.detach().to("cpu", torch.float64).numpy()  # noqa: E731
+    rows = sorted(set(fa_inputs.sample_rows(w.N, plan["rows"], seed=1234)) |
+                  set(range(min(plan.get("extra_rows", 0), w.N)))) if plan["rows"] else []
+    rows = np.array(rows, dtype=np.int64)
+    got = {n: [] for n in ("O", "LSE", "dQ", "dK", "dV")}
+    ref = {n: [] for n in got}
+    t_or, units = 0.0, 0.0  # oracle seconds; its products in units of N*d multiply-adds
+    for b in range(w.B):
+        for h in range(w.H):
+            full = (b, h) in plan["full_heads"]
+            if not full and rows.size == 0:
+                continue
+            Q, K, V = (f64(ins[n][b, h]) for n in ("Q", "K", "V"))
+            dO = f64(ins["dO"][b, h]) if with_bwd else None
+            O64, L64 = f64(outs["O"][b, h]), f64(outs["LSE"][b, h])
+            t0 = time.perf_counter()
+            if full:
+                rO, rL, _ = oracle.attention_head(Q, K, V, w.scale, w.causal)
+                units += 2 * w.N
+                if with_bwd:
+                    rg = oracle.attention_bwd_head(Q, K, V, dO, w.scale, w.causal)
+                    units += 6 * w.N
+            else:
+                rO, rL, _ = oracle.attention_head(Q[rows], K, V, w.scale, w.causal,
+                                                  q_index=rows)
+                units += 2 * rows.size
+                if with_bwd:
+                    rdq, _ = oracle.attention_bwd_dq_rows(Q[rows], K, V, dO[rows], w.scale,
+                                                          w.causal, rows)
+                    units += 4 * rows.size
+            t_or += time.perf_counter() - t0
+            sel = slice(None) if full else rows
+            got["O"].append(O64[sel].ravel())
+            ref["O"].append(rO.ravel())
+            got["LSE"].append(L64[sel].ravel())
+            ref["LSE"].append(rL.ravel())
+            if with_bwd:
+                gq = f64(outs["dQ"][b, h])
+                if full:
+                    for k_, n in enumerate(("dQ", "dK", "dV")):
+                        got[n].append(f64(outs[n][b, h]).ravel())
+                        ref[n].append(rg[k_].ravel())
+                else:
+                    got["dQ"].append(gq[rows].ravel())
+                    ref["dQ"].append(rdq.ravel())
+    res = {}
+    for n in got:
+        if not got[n]:
+            continue
+        g, r = np.concatenate(got[n]), np.concatenate(ref[n])
+        diff = g - r
+        res[n] = {"max_abs": float(np.abs(diff).max()),
+                  "rel_l2": float(np.linalg.norm(diff) / np.linalg.norm(r)),
+                  "values": int(g.size)}
+    full_units = w.B * w.H * (2 + (6 if with_bwd else 0)) * w.N
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((i.get("num_threads", 1) for i in threadpool_info()
+                       if i.get("user_api") == "blas"), default=1)
+    except Exception:
+        threads = os.cpu_count() or 1
+    res["subset"] = (f"whole heads {list(plan['full_heads'])}; "
+                     f"{rows.size} seeded rows of every head" if rows.size else
+                     f"whole heads {list(plan['full_heads'])}")
+    res["oracle_s"] = t_or
+    res["oracle_threads"] = int(threads)
+    res["oracle_est_full_s"] = t_or * full_units / units if units else None
+    return res
+
+
 def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -224,10 +324,11 @@ def run_reference(args, w):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
-                   "causal": w.causal, "parallelism": "host cores"},
+        "config": config_dict(w, not args.fwd_only, args.gpus),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads,
-                         "kind": "oracle", "sample": sample},
+                         "kind": "oracle",
+                         "sample": sample + "; run on the host cores (rank 0 only), each "
+                         "step one bounded sample of the workload"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -466,10 +567,7 @@ def run_gpu(args, w):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32" if f32 else "bf16",
         "data": "synthetic",
-        "config": {"workload": w.name, "B": B, "H": H, "N": N, "d": d, "causal": w.causal,
-                   "step": "fa_fwd + fa_bwd" if with_bwd else "fa_fwd",
-                   "l2": "inputs larger than L2 (no flush)",
-                   "parallelism": f"replicas x{world} (independent heads per GPU)"},
+        "config": config_dict(w, with_bwd, world),
         "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "step_ms_percentiles": step_pct,
         "fwd_tflops": f_fwd / (fwd_ms * 1e-3) / 1e12,
         "bwd_tflops": (f_bwd / (bwd_ms * 1e-3) / 1e12) if with_bwd else None,
@@ -478,7 +576,11 @@ def run_gpu(args, w):
                                 / (bwd_ms * 1e-3) / 1e12) if with_bwd else None,
         "roofline": {"kernel": dom_name, "bound": bound, "achieved": achieved,
                      "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                     "peak_source": peak_source, "traffic": recorded_traffic(dom_name)},
+                     "peak_source": peak_source, "traffic": recorded_traffic(dom_name),
+                     **({} if f32 else {
+                         "peak_sustained": peaks.get("bf16_tflops_sustained"),
+                         "frac_sustained": achieved / peaks["bf16_tflops_sustained"]
+                         if peaks.get("bf16_tflops_sustained") else None})},
         "kernels": kernels,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
@@ -488,6 +590,9 @@ def run_gpu(args, w):
         "gpu_launches": args.steps * (1 + (3 if with_bwd else 0)),
         "clocks": clocks.summary(),
     }
+    if args.check and world == 1:
+        line["parity"] = parity_check(
+            w, ins, {"O": O, "LSE": LSE, "dQ": dQ, "dK": dK, "dV": dV}, with_bwd)
     if world == 1 and not args.no_cpu_baseline:
         v_cpu, threads, sample, _ = time_oracle(w, max_seconds=args.ref_seconds)
         line["cpu_baseline"] = {"value": v_cpu, "unit": "TFLOP/s", "cores": threads,
@@ -615,6 +720,9 @@ def main():
     ap.add_argument("--sustained-peak", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=20.0)
+    ap.add_argument("--check", action="store_true",
+                    help="after timing, compare the outputs with the fp64 oracle on the "
+                    "workload's checked subset and time the oracle on it")
     ap.add_argument("--sweep", action="store_true",
                     help="print TFLOP/s of fa_fwd and fa_bwd against N instead of the step")
     args = ap.parse_args()

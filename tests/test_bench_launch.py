@@ -30,6 +30,13 @@ def test_reference_arm_under_torchrun():
     assert line["impl"] == "reference" and line["unit"] == "TFLOP/s"
     assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
     assert line["config"]["workload"] == "n4096_d64"
+    # the same config dict as the GPU arm of the same command line
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_cfg", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    from exact_io_aware_64_b200 import inputs
+    assert line["config"] == bench.config_dict(inputs.WORKLOADS["n4096_d64"], True, 2)
 
 
 def test_per_kernel_rates():
