@@ -72,15 +72,6 @@ __device__ __forceinline__ uint32_t split_operand_col(uint32_t base, int kk) {
 }
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
-// Every PolyEvery<D>-th pair of exponentials of a row may be computed on the FMA pipe
-// (exp2_poly_x2) instead of the MUFU unit; masked entries are zeroed after the
-// exponential either way; 0 keeps all of them on MUFU.
-template <int D>
-struct PolyEvery {
-  static constexpr int value = 0;
-};
-
-__host__ __device__ constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
 struct BwdArgs {
   unsigned int* err;
@@ -335,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // unit w: key tile j of head bh, meeting query tiles i0 .. i0 + m - 1 of its sequence
   // (m = 0: the tile lies past the sequence's keys, or the sequence has no queries)
   auto unit = [&](int w, int& bh, int& j, int& i0, int& m, int& lk, int& off, int& tq0,
-                  int& tk0) {
+                  int& tk0, int& lq) {
     if (args.causal) {
       j = w / args.BH;  // key tile 0 meets every query tile: heaviest first
       bh = w % args.BH;
@@ -343,7 +334,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       bh = w / args.n_kt;
       j = w % args.n_kt;
     }
-    int lq;
     seq_info(args, bh, lq, lk, tq0, tk0);
     off = lk - lq;  // position of query row 0 among the keys
     i0 = 0;
@@ -369,8 +359,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int live = 0;  // 1 when the unit just processed had work: units counts only those
     for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
          w = snake_unit(++r), units += live) {
-      int bh, j, i0, m, lk, off, tq0, tk0;
-      unit(w, bh, j, i0, m, lk, off, tq0, tk0);
+      int bh, j, i0, m, lk, off, tq0, tk0, lq;
+      unit(w, bh, j, i0, m, lk, off, tq0, tk0, lq);
       live = m > 0;
       if (!live) continue;
       if (units > 0) ok = wait_warp(bar(L::kBarKVEmpty), (units - 1) & 1);
@@ -466,8 +456,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int live = 0;
     for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
          w = snake_unit(++r), units += live) {
-      int bh, j, i0, m, lk, off, tq0, tk0;
-      unit(w, bh, j, i0, m, lk, off, tq0, tk0);
+      int bh, j, i0, m, lk, off, tq0, tk0, lq;
+      unit(w, bh, j, i0, m, lk, off, tq0, tk0, lq);
       live = m > 0;
       if (!live) continue;
       ok = wait_warp(bar(L::kBarKVFull), units & 1);
@@ -519,10 +509,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     int live = 0;
     for (int r = 0, w = snake_unit(0); ok && w < args.total_units;
          w = snake_unit(++r), units += live) {
-      int bh, j, i0, m, lk, off, tq0, tk0;
-      unit(w, bh, j, i0, m, lk, off, tq0, tk0);
+      int bh, j, i0, m, lk, off, tq0, tk0, lq;
+      unit(w, bh, j, i0, m, lk, off, tq0, tk0, lq);
       live = m > 0;
-      if (!live) continue;
+      if (!live) {
+        // a sequence with keys but no queries: no query sees these keys, so their
+        // gradients are exactly zero (group g writes its half of each row)
+        const int kv_row = j * kTile + row;
+        if (lq == 0 && kv_row < lk) {
+          const size_t orow = k_row_offset(args, bh, tk0, kv_row, D) + g * (D / 2);
+          uint4* zk = reinterpret_cast<uint4*>(args.dK + orow);
+          uint4* zv = reinterpret_cast<uint4*>(args.dV + orow);
+#pragma unroll
+          for (int c = 0; c < D / 16; ++c) {
+            zk[c] = make_uint4(0u, 0u, 0u, 0u);
+            zv[c] = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+        continue;
+      }
       for (int i = i0; i < i0 + m; ++i) {
         // this tile's L2 and D rows sit in its dO slot
         const uint8_t* sb = smem + L::kDO0 + stage * L::kDOSlotBytes;
@@ -533,7 +538,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         ++s_cnt;
         tc_fence_after();
-        constexpr int kStride = PolyEvery<D>::value > 0 ? PolyEvery<D>::value : 1;
         float p[kCols];
         {
           uint32_t r[kCols];
@@ -551,9 +555,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t nl = *reinterpret_cast<const uint64_t*>(sL + c);
             const uint64_t x2 =
                 fma_x2(f32x2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), scale2, nl);
-            const bool poly = PolyEvery<D>::value > 0 && (c / 2) % kStride == kStride - 1;
             float e0, e1;
-            exp2_pair(x2, poly, e0, e1);
+            exp2_pair(x2, e0, e1);
             if (diag && col0 + c < row + delta) e0 = 0.f;
             if (diag && col0 + c + 1 < row + delta) e1 = 0.f;
             p[c] = e0;
@@ -956,7 +959,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         ++s_cnt;
         tc_fence_after();
-        constexpr int kStride = PolyEvery<D>::value > 0 ? PolyEvery<D>::value : 1;
         float p[kCols];
         {
           uint32_t r[kCols];
@@ -977,9 +979,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < kCols; c += 2) {
             const uint64_t x2 =
                 fma_x2(f32x2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), scale2, nl2);
-            const bool poly = PolyEvery<D>::value > 0 && (c / 2) % kStride == kStride - 1;
             float e0, e1;
-            exp2_pair(x2, poly, e0, e1);
+            exp2_pair(x2, e0, e1);
             if (need_mask && kv0 + c >= lim) e0 = 0.f;
             if (need_mask && kv0 + c + 1 >= lim) e1 = 0.f;
             p[c] = e0;
@@ -1109,7 +1110,7 @@ cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUten
 
 }  // namespace
 
-int bwd_padded_rows(int N) { return round_up(N, kTile); }
+long long bwd_padded_rows(long long N) { return (N + kTile - 1) / kTile * kTile; }
 
 cudaError_t launch_bwd_sm100(const CUtensorMap& tmQ, const CUtensorMap& tmK,
                              const CUtensorMap& tmV, const CUtensorMap& tmdO,

@@ -68,13 +68,18 @@ static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kThreads * kRegsLau
 constexpr int kWarpTMA = 8;
 constexpr int kWarpMMA = 9;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-// Every PolyEvery<D>-th pair of exponentials (unmasked tiles only) may be computed on
-// the FMA pipe with exp2_poly_x2 instead of MUFU; 0 keeps all of them on MUFU.
-template <int D>
-struct PolyEvery {
-  static constexpr int value = 0;
-};
 constexpr uint32_t kTmemCols = 512;
+// At d = 64 the S0 | S1 | O0 | O1 regions fill 384 of the 512 TMEM columns, which leaves
+// room for the probabilities in regions of their own (P0 | P1, 64 columns each) instead
+// of over their score tile.  S_t(j+1) can then be computed while the softmax of S_t(j)
+// is still running: the tile's score product no longer waits for the P V product that
+// reads the probabilities, and the softmax warps, which bound the kernel at d = 64
+// (a 128 x 128 tile costs as many exponentials as at d = 128 for half the tensor work),
+// find their next tile ready.
+template <int D>
+struct SeparateP {
+  static constexpr bool value = (D == 64);
+};
 
 template <int D>
 struct FwdLayout {
@@ -95,7 +100,8 @@ struct FwdLayout {
   static constexpr int kBarODone = 8 + 2 * kStages;   // [2]
   static constexpr int kBarOFree = 10 + 2 * kStages;  // [2]
   static constexpr int kBarDrain = 12 + 2 * kStages;  // [1]
-  static constexpr int kNumBars = 13 + 2 * kStages;
+  static constexpr int kBarSFree = 13 + 2 * kStages;  // [2] (separate-P layout only)
+  static constexpr int kNumBars = 15 + 2 * kStages;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024 bytes
@@ -220,6 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(L::kBarPReady + t), kBM / 32);  // one arrival per softmax warp
       mbar_init(bar(L::kBarODone + t), 1);
       mbar_init(bar(L::kBarOFree + t), kBM / 32);
+      mbar_init(bar(L::kBarSFree + t), kBM / 32);
     }
     mbar_init(bar(L::kBarDrain), 1);
     fence_mbar_init();
@@ -237,8 +244,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  constexpr bool kSepP = SeparateP<D>::value;
   const uint32_t tS[2] = {tmem, tmem + 128};
   const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
+  // where the bf16 probabilities of tile t go: their own region, or over S_t
+  const uint32_t tP[2] = {kSepP ? tmem + 256 + 2 * D : tS[0],
+                          kSepP ? tmem + 256 + 2 * D + 64 : tS[1]};
 
   if (warp >= 8) regs_dec<kRegsControl>();
   if (warp == kWarpTMA) {
@@ -336,11 +347,99 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t db = dRingV + static_cast<uint64_t>((vslot * L::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
-          mma_ts_elect(tO[t], tS[t] + kk * 8, db + static_cast<uint64_t>((kk * 2048) >> 4), idPV,
+          mma_ts_elect(tO[t], tP[t] + kk * 8, db + static_cast<uint64_t>((kk * 2048) >> 4), idPV,
                  (accumulate || kk > 0) ? 1u : 0u);
         }
         mma_commit_elect(bar(L::kBarODone + t));
       };
+      // warp-uniform non-blocking test of a barrier phase
+      auto test_warp = [&](uint32_t b, uint32_t parity) -> bool {
+        return __shfl_sync(0xffffffffu, mbar_test(b, parity) ? 1 : 0, 0) != 0;
+      };
+      if constexpr (kSepP) {
+        // Separate P regions: the four products of a key tile j (S_t(j) for t = 0, 1 and
+        // P_t V_j) are issued in whatever order their inputs become ready -- S_t(j) once
+        // K_j has landed and the softmax warps hold S_t(j-1) in registers, P_t V_j once
+        // they have written P_t(j) and V_j has landed.  K_j and V_j are released when
+        // both tiles have issued their product with it.  The TMA warp loads the unit's
+        // tiles in the order K_0 V_0 K_1 V_1 ..., so K_j sits at ring position
+        // ring + 2j and V_j at ring + 2j + 1.
+        int ring = 0;
+        int s_tot[2] = {0, 0};
+        for (int r = 0, w = snake_unit(0); ok && w < args.total_units; w = snake_unit(++r)) {
+          const UnitInfo ui = unit_info(w, args);
+          if (ui.n0 == 0) continue;  // no query rows in this unit
+          const int nt[2] = {ui.n0, ui.n1};
+          const int n = max(ui.n0, ui.n1);
+          for (int t = 0; t < 2 && ok; ++t)
+            if (nt[t] > 0) ok = wait_warp(bar(L::kBarQFull + t), uses[t] & 1);
+          if (!ok) break;
+          int sI[2] = {0, 0}, pI[2] = {0, 0};
+          long long t0 = clock64();
+          uint32_t idle = 0;
+          while (sI[0] < nt[0] || sI[1] < nt[1] || pI[0] < nt[0] || pI[1] < nt[1]) {
+            bool progress = false;
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              const int o = 1 - t;
+              if (sI[t] < nt[t]) {
+                const int j = sI[t];
+                const int pos = ring + 2 * j;
+                const int st = pos % L::kStages;
+                if ((s_tot[t] == 0 || test_warp(bar(L::kBarSFree + t), (s_tot[t] - 1) & 1)) &&
+                    test_warp(bar(L::kBarKVFull + st), (pos / L::kStages) & 1)) {
+                  tc_fence_after();
+                  issue_s(t, st);
+                  if (j + 1 == nt[t]) mma_commit_elect(bar(L::kBarQEmpty + t));
+                  ++s_tot[t];
+                  ++sI[t];
+                  if (nt[o] <= j || sI[o] > j) mma_commit_elect(bar(L::kBarKVEmpty + st));
+                  progress = true;
+                }
+              }
+              if (pI[t] < nt[t]) {
+                const int j = pI[t];
+                const int pos = ring + 2 * j + 1;
+                const int st = pos % L::kStages;
+                if (test_warp(bar(L::kBarPReady + t), p_count[t] & 1) &&
+                    (j > 0 || uses[t] == 0 ||
+                     test_warp(bar(L::kBarOFree + t), (uses[t] - 1) & 1)) &&
+                    test_warp(bar(L::kBarKVFull + st), (pos / L::kStages) & 1)) {
+                  tc_fence_after();
+                  issue_pv(t, st, j > 0);
+                  ++p_count[t];
+                  ++pI[t];
+                  if (nt[o] <= j || pI[o] > j) mma_commit_elect(bar(L::kBarKVEmpty + st));
+                  progress = true;
+                }
+              }
+            }
+            if (progress) {
+              idle = 0;
+              continue;
+            }
+            // nothing was ready: give up after the same limit as every other wait
+            if (++idle == 1) t0 = clock64();
+            if (idle % kSpinCheck == 0) {
+              int code = 0;  // 1: another warp aborted, 2: this wait timed out
+              if (lane == 0)
+                code = *abort_flag ? 1 : (clock64() - t0 > kWaitLimitCycles ? 2 : 0);
+              code = __shfl_sync(0xffffffffu, code, 0);
+              if (code == 2 && lane == 0) {
+                atomicOr(args.err, kErrWaitTimeout);
+                *abort_flag = 1;
+              }
+              if (code != 0) {
+                ok = false;
+                break;
+              }
+            }
+          }
+          ring += 2 * n;
+          for (int t = 0; t < 2; ++t)
+            if (nt[t] > 0) ++uses[t];
+        }
+      } else {
       for (int r = 0, w = snake_unit(0); ok && w < args.total_units; w = snake_unit(++r)) {
         const UnitInfo ui = unit_info(w, args);
         if (ui.n0 == 0) continue;  // no query rows in this unit
@@ -389,6 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < 2; ++t)
           if (nt[t] > 0) ++uses[t];
       }
+      }
       // drain: every MMA issued has completed before TMEM is released
       mma_commit_elect(bar(L::kBarDrain));
       mbar_wait_drain(bar(L::kBarDrain), 0, args.err);
@@ -401,6 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>((warp % 4) * 32) << 16;
     const uint32_t tSrow = tS[t] + lane_off;
     const uint32_t tOrow = tO[t] + lane_off;
+    const uint32_t tProw = tP[t] + lane_off;
     int s_count = 0, o_count = 0;
     bool ok = true;
     for (int r = 0, w = snake_unit(0); ok && w < args.total_units; w = snake_unit(++r)) {
@@ -420,6 +521,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < kBN / 32; ++c) tmem_ld32(tSrow + c * 32, &sr[c * 32]);
         tmem_wait_ld();
+        // with P in its own region, S_t's columns are free as soon as they are read
+        if constexpr (kSepP) warp_arrive(bar(L::kBarSFree + t));
         float s[kBN];
 #pragma unroll
         for (int c = 0; c < kBN; ++c) s[c] = __uint_as_float(sr[c]);
@@ -452,12 +555,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           m = m_new;
           rescale = true;
         }
-        if (__any_sync(0xffffffffu, rescale && j > 0)) {
-          // O_t holds the sum through key tile j-1: wait for that product, then scale
-          ok = wait_warp(bar(L::kBarODone + t), (o_count + j - 1) & 1);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-          tc_fence_after();
+        // O_t holds the sum through key tile j-1 once that P V product completes; then it
+        // is scaled by alpha (only when some row's reference max moved)
+        auto rescale_o = [&]() {
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             uint32_t v[32];
@@ -468,6 +568,13 @@ __global__ void __launch_bounds__(kThreads, 1)
               v[k] = __float_as_uint(__uint_as_float(v[k]) * alpha);
             tmem_st32(tOrow + c * 32, v);
           }
+        };
+        if (!kSepP && __any_sync(0xffffffffu, rescale && j > 0)) {
+          ok = wait_warp(bar(L::kBarODone + t), (o_count + j - 1) & 1);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+          rescale_o();
         }
         l *= alpha;
         const float mref = (m == -INFINITY) ? 0.f : m;
@@ -477,16 +584,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t scale2 = f32x2(args.scale_log2, args.scale_log2);
         const uint64_t negm2 = f32x2(-mref, -mref);
         uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};
-        constexpr int kEvery = PolyEvery<D>::value;
-        constexpr int kStride = kEvery > 0 ? kEvery : 1;
 #pragma unroll
         for (int c = 0; c < kBN / 2; ++c) {
           const uint64_t x2 = fma_x2(f32x2(s[2 * c], s[2 * c + 1]), scale2, negm2);
-          // every kEvery-th pair may go to the FMA pipe (never on masked tiles, so masked
-          // entries stay exactly 0)
-          const bool poly = kEvery > 0 && !need_mask && c % kStride == kStride - 1;
           float p0, p1;
-          exp2_pair(x2, poly, p0, p1);
+          exp2_pair(x2, p0, p1);
           ls2[c % 4] = add_x2(ls2[c % 4], f32x2(p0, p1));
           pk[c] = pack_bf16x2(p0, p1);
         }
@@ -494,8 +596,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int k = 0; k < 4; ++k) f32x2_split(ls2[k], ls[2 * k], ls[2 * k + 1]);
         l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-        tmem_st32(tSrow, &pk[0]);
-        tmem_st32(tSrow + 32, &pk[32]);
+        if constexpr (kSepP) {
+          // P_t's region is free, and O_t complete through key tile j-1, once P_t V_{j-1}
+          // has completed; by now it normally has (it was issued a whole tile ago)
+          if (j > 0) {
+            ok = wait_warp(bar(L::kBarODone + t), (o_count + j - 1) & 1);
+            if (!ok) break;
+            tc_fence_after();
+            if (__any_sync(0xffffffffu, rescale)) rescale_o();
+          }
+        }
+        tmem_st32(tProw, &pk[0]);
+        tmem_st32(tProw + 32, &pk[32]);
         tmem_wait_st();
         warp_arrive(bar(L::kBarPReady + t));
       }

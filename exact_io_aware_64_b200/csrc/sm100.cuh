@@ -59,6 +59,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test: has the phase with the given parity completed?
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Upper bound on any single pipeline wait, in SM clock cycles (4 s at 2 GHz, longer at
 // lower clocks).  Every wait in these kernels is on work that the same CTA has already
 // issued or will issue within microseconds; a wait this long means the pipeline is
@@ -403,43 +416,12 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   return d;
 }
 
-// 2^x on the FMA and integer pipes instead of the MUFU unit, for x >= -126 (smaller x
-// is clamped; the result is then below 2^-126).  Cody-Waite style range reduction
-// x = n + f with n = round(x) taken by adding 1.5 * 2^23 (its low mantissa bits then hold
-// n), f in [-1/2, 1/2]; 2^f by a cubic fitted with the Remez exchange algorithm on the
-// relative error (gen_exp2_poly.py: max relative error 7.5e-5, well below bf16
-// rounding); 2^n applied by adding n to the exponent field.
-// Two values at once: the additions and the polynomial run on packed float pairs;
-// x - round(x) is formed as fma(round(x), -1, x), which is exact.
-__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x2) {
-  constexpr float kC0 = 0.99992806f, kC1 = 0.69326097f, kC2 = 0.24261113f, kC3 = 0.05517167f;
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+// 2^x of a packed pair on the MUFU unit (ex2.approx, flush-to-zero).
+__device__ __forceinline__ void exp2_pair(uint64_t x2, float& e0, float& e1) {
   float x0, x1;
   f32x2_split(x2, x0, x1);
-  const uint64_t x = f32x2(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
-  const uint64_t t = add_x2(x, f32x2(kRound, kRound));
-  const uint64_t n = add_x2(t, f32x2(-kRound, -kRound));
-  const uint64_t f = fma_x2(n, f32x2(-1.0f, -1.0f), x);
-  uint64_t p = fma_x2(f32x2(kC3, kC3), f, f32x2(kC2, kC2));
-  p = fma_x2(p, f, f32x2(kC1, kC1));
-  p = fma_x2(p, f, f32x2(kC0, kC0));
-  float p0, p1, t0, t1;
-  f32x2_split(p, p0, p1);
-  f32x2_split(t, t0, t1);
-  return f32x2(__int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23)),
-               __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23)));
-}
-
-// 2^x of a packed pair, on MUFU (ex2.approx) or, when `poly`, on the FMA pipe.
-__device__ __forceinline__ void exp2_pair(uint64_t x2, bool poly, float& e0, float& e1) {
-  if (poly) {
-    f32x2_split(exp2_poly_x2(x2), e0, e1);
-  } else {
-    float x0, x1;
-    f32x2_split(x2, x0, x1);
-    e0 = ex2_approx(x0);
-    e1 = ex2_approx(x1);
-  }
+  e0 = ex2_approx(x0);
+  e1 = ex2_approx(x1);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -116,13 +116,17 @@ def test_f32_varlen(case, d, causal):
         for h in range(H):
             what = f"f32 varlen b={bi} h={h} lq={nq} lk={nk} d={d} causal={causal}"
             skipped = nq == 0 or nk == 0
-            q_end = 0 if skipped else nq  # a skipped sequence writes no row at all
-            k_end = 0 if skipped else nk
+            q_end = 0 if skipped else nq  # a skipped sequence writes no query row
+            # keys without queries get zero gradients; a sequence without keys, none
+            k_end = 0 if nk == 0 else nk
             assert bool((O[bi, h, q_end:] == SENTINEL).all()), "O past the rows " + what
             assert bool((LSE[bi, h, q_end:] == SENTINEL).all()), "LSE past the rows " + what
             assert bool((grads[0][bi, h, q_end:] == SENTINEL).all()), "dQ past " + what
             assert bool((grads[1][bi, h, k_end:] == SENTINEL).all()), "dK past " + what
             assert bool((grads[2][bi, h, k_end:] == SENTINEL).all()), "dV past " + what
+            if nq == 0:
+                assert bool((grads[1][bi, h, :nk] == 0).all()), "dK of unseen keys " + what
+                assert bool((grads[2][bi, h, :nk] == 0).all()), "dV of unseen keys " + what
             if skipped:
                 continue
             _check_head(to64(a["Q"][bi, h, :nq]), to64(b["K"][bi, h, :nk]),
@@ -174,7 +178,8 @@ def test_f32_packed(case, d, causal):
         qs, ks = slice(q0s[s], q0s[s] + nq), slice(k0s[s], k0s[s] + nk)
         if nk == 0 or nq == 0:
             assert bool((O[qs] == SENTINEL).all()) and bool((dQ[qs] == SENTINEL).all())
-            assert bool((dK[ks] == SENTINEL).all()) and bool((dV[ks] == SENTINEL).all())
+            # keys no query sees: exactly zero gradients
+            assert bool((dK[ks] == 0).all()) and bool((dV[ks] == 0).all())
             continue
         for h in range(H):
             _check_head(to64(a["Q"][qs, h]), to64(b["K"][ks, h]), to64(b["V"][ks, h]),

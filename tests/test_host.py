@@ -72,48 +72,3 @@ def test_workloads_have_expected_shapes():
     assert w["n10000_d128_causal"].N % 128 != 0
     assert w["n32768_d128_causal_sigma3"].sigma_qk == 3.0
     assert w["n8192_d128_causal_bwd"].backward
-
-
-def _exp2_poly_coefficients():
-    import re
-    src = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
-                            "exact_io_aware_64_b200", "csrc", "sm100.cuh")).read()
-    m = re.search(r"kC0 = ([0-9.]+)f, kC1 = ([0-9.]+)f, kC2 = ([0-9.]+)f, kC3 = ([0-9.]+)f", src)
-    return [float(v) for v in m.groups()]
-
-
-def test_exp2_poly_matches_its_generator_and_error_bound():
-    """The kernels' FMA-pipe exp2 (exp2_poly_x2: range reduction + cubic): its
-    coefficients are the Remez fit that csrc/gen_exp2_poly.py produces, and the float32
-    arithmetic it performs (each step exactly rounded, x - round(x) exact) stays within
-    the fit's relative-error bound over the range it is used on."""
-    import importlib.util
-    import numpy as np
-    c = _exp2_poly_coefficients()
-    path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
-                        "exact_io_aware_64_b200", "csrc", "gen_exp2_poly.py")
-    spec = importlib.util.spec_from_file_location("gen_exp2_poly", path)
-    gen = importlib.util.module_from_spec(spec)
-    spec.loader.exec_module(gen)
-    fit, bound = gen.remez()
-    assert np.allclose(np.float32(fit), np.float32(c), rtol=0, atol=1e-7)
-    assert bound < 8e-5
-    f32 = np.float32
-    x = np.linspace(-125.0, 8.0, 3000001).astype(f32)
-    t = (x + f32(12582912.0)).astype(f32)
-    f = (x - (t - f32(12582912.0)).astype(f32)).astype(f32)
-    p = f32(c[3])
-    for k in (2, 1, 0):
-        p = (p * f + f32(c[k])).astype(f32)
-    r = (p.view(np.int32) + (t.view(np.int32) << 23)).view(f32)
-    rel = np.abs(r.astype(np.float64) / np.exp2(x.astype(np.float64)) - 1.0)
-    assert rel.max() < 8e-5
-    # the clamp keeps the exponent field valid for any very negative input
-    xc = np.maximum(np.array([-1e30, -200.0, -126.0], dtype=f32), f32(-126.0))
-    tc = (xc + f32(12582912.0)).astype(f32)
-    fc = (xc - (tc - f32(12582912.0)).astype(f32)).astype(f32)
-    pc = f32(c[3])
-    for k in (2, 1, 0):
-        pc = (pc * fc + f32(c[k])).astype(f32)
-    rc = (pc.view(np.int32) + (tc.view(np.int32) << 23)).view(f32)
-    assert np.all(rc >= 0) and np.all(rc < 2.0 ** -125)
