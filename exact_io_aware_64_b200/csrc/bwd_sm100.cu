@@ -36,7 +36,8 @@
 // dS over the first 32 columns of its own 64-column half, so the two groups never touch
 // each other's TMEM, and the MMA reads the bf16 operand as two 32-column pieces.  The MMA order is chosen so the
 // tensor core works on one product while the element-wise warps build the next operand
-// (dK/dV: S^T(i) dP^T(i) | dV(i) S^T(i+1) | dK(i) dP^T(i+1) | ...;
+// (dK/dV: S^T(i) dP^T(i) | dV(i) S^T(i+1) | dK(i) dP^T(i+1) | ..., with dV(i) issued in
+// two halves as the two halves of each group's P^T(i) are written;
 //  dQ: S(j) dP(j) | S(j+1) dQ(j) dP(j+1) | S(j+2) dQ(j+1) dP(j+2) | ...).
 // Causal work units are ordered heaviest first.
 #include <cstdint>
@@ -257,7 +258,8 @@ struct DkdvLayout {
   static constexpr int kBarAccFull = kBarSFull + 4;
   static constexpr int kBarAccFree = kBarSFull + 5;
   static constexpr int kBarDrain = kBarSFull + 6;
-  static constexpr int kNumBars = kBarDrain + 1;
+  static constexpr int kBarPReadyB = kBarSFull + 7;  // second half of each group's P^T
+  static constexpr int kNumBars = kBarPReadyB + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kAlloc = kMisc + 16;
   static_assert(kAlloc <= 232448, "shared memory over the 227 KB per-block limit");
@@ -307,6 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(L::kBarSFull), 1);
     mbar_init(bar(L::kBarDPFull), 1);
     mbar_init(bar(L::kBarPReady), kEw / 32);
+    mbar_init(bar(L::kBarPReadyB), kEw / 32);
     mbar_init(bar(L::kBarDSReady), kEw / 32);
     mbar_init(bar(L::kBarAccFull), 1);
     mbar_init(bar(L::kBarAccFree), kEw / 32);
@@ -435,6 +438,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_ts_elect(acc, split_operand_col(a_tmem, kk), db + static_cast<uint64_t>((kk * 2048) >> 4),
                      idTS, (accumulate || kk > 0) ? 1u : 0u);
     };
+    // the same product over the K steps whose 16 queries lie in half h of each group's
+    // 64 columns (h = 0: K steps 0, 1, 4, 5; h = 1: 2, 3, 6, 7); half 0 comes first, so the
+    // product's first K step, which starts the accumulation of a unit, is in it
+    auto issue_ts_half = [&](uint32_t acc, uint32_t a_tmem, uint32_t b_saddr, bool accumulate,
+                             int h) {
+      const uint64_t db = desc_mnmajor(b_saddr, L::kBoxBytes);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int kk = (q / 2) * 4 + h * 2 + (q % 2);
+        mma_ts_elect(acc, split_operand_col(a_tmem, kk), db + static_cast<uint64_t>((kk * 2048) >> 4),
+                     idTS, (accumulate || kk > 0) ? 1u : 0u);
+      }
+    };
     // S^T(next query tile) from the next Q slot
     auto next_s = [&](int& slot) -> bool {
       if (!wait_warp(bar(L::kBarQFull + qc), qcph)) return false;
@@ -469,9 +485,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = wait_warp(bar(L::kBarPReady), p_cnt & 1);
         if (ok && t == 0 && units > 0) ok = wait_warp(bar(L::kBarAccFree), (units - 1) & 1);
         if (!ok) break;
-        ++p_cnt;
         tc_fence_after();
-        issue_ts(tdV, tS, doslot(curd), t > 0);  // dV += P^T dO
+        // dV += P^T dO over the first half of every group's queries while the
+        // element-wise warps still compute the second half (the dV product reads P^T;
+        // starting it early shortens the S^T -> exponentials -> dV -> next S^T loop that
+        // paces the kernel), then over the second half
+        issue_ts_half(tdV, tS, doslot(curd), t > 0, 0);
+        ok = wait_warp(bar(L::kBarPReadyB), p_cnt & 1);
+        if (!ok) break;
+        tc_fence_after();
+        issue_ts_half(tdV, tS, doslot(curd), t > 0, 1);
+        ++p_cnt;
         mma_commit_elect(bar(L::kBarDOEmpty + curd));
         int nq = -1, nd = -1;
         if (t + 1 < m) {
@@ -549,28 +573,32 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int delta = (j - i) * kTile - off;
           const bool diag = args.causal && delta > -kTile;
           const uint64_t scale2 = f32x2(args.scale_log2, args.scale_log2);
+          // the group's 64 columns in two halves of 32; each half's bf16 P^T is stored and
+          // announced as soon as it is made
 #pragma unroll
-          for (int c = 0; c < kCols; c += 2) {
-            // x = S^T * scale * log2e - L2 for two query columns in one packed FMA
-            const uint64_t nl = *reinterpret_cast<const uint64_t*>(sL + c);
-            const uint64_t x2 =
-                fma_x2(f32x2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), scale2, nl);
-            float e0, e1;
-            exp2_pair(x2, e0, e1);
-            if (diag && col0 + c < row + delta) e0 = 0.f;
-            if (diag && col0 + c + 1 < row + delta) e1 = 0.f;
-            p[c] = e0;
-            p[c + 1] = e1;
+          for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll
+            for (int c = hf * (kCols / 2); c < (hf + 1) * (kCols / 2); c += 2) {
+              // x = S^T * scale * log2e - L2 for two query columns in one packed FMA
+              const uint64_t nl = *reinterpret_cast<const uint64_t*>(sL + c);
+              const uint64_t x2 =
+                  fma_x2(f32x2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), scale2, nl);
+              float e0, e1;
+              exp2_pair(x2, e0, e1);
+              if (diag && col0 + c < row + delta) e0 = 0.f;
+              if (diag && col0 + c + 1 < row + delta) e1 = 0.f;
+              p[c] = e0;
+              p[c + 1] = e1;
+            }
+            uint32_t pk[kCols / 4];
+#pragma unroll
+            for (int c = 0; c < kCols / 4; ++c)
+              pk[c] = pack_bf16x2(p[hf * (kCols / 2) + 2 * c], p[hf * (kCols / 2) + 2 * c + 1]);
+            tmem_st16(tS + lane_off + col0 + hf * (kCols / 4), pk);
+            tmem_wait_st();
+            warp_arrive(bar(hf == 0 ? L::kBarPReady : L::kBarPReadyB));
           }
         }
-        {
-          uint32_t pk[kCols / 2];
-#pragma unroll
-          for (int c = 0; c < kCols / 2; ++c) pk[c] = pack_bf16x2(p[2 * c], p[2 * c + 1]);
-          tmem_st32(tS + lane_off + col0, pk);
-        }
-        tmem_wait_st();
-        warp_arrive(bar(L::kBarPReady));
         ok = wait_warp(bar(L::kBarDPFull), dp_cnt & 1);
         if (!ok) break;
         ++dp_cnt;
