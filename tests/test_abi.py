@@ -89,6 +89,16 @@ def test_fwd_validation(lib):
     assert "d=96" in msg
     huge = _fwd(lib, B=1 << 15, H=1 << 15, N=1 << 12)
     assert huge[0] == binding.FA_ERR_INVALID_ARG
+    # lengths near INT_MAX: rounded up to whole 256-row units they would overflow a
+    # 32-bit int, so they are rejected before any arithmetic on them
+    for n in ((1 << 31) - 1, (1 << 31) - 255):
+        st, msg = _fwd(lib, N=n)
+        assert st == binding.FA_ERR_INVALID_ARG and "too large" in msg, msg
+    assert lib.fa_fwd_qk(A, B_, C, D_, E, 1, 1, 16, (1 << 31) - 1, 64, 0.1, 0,
+                         None) == binding.FA_ERR_INVALID_ARG
+    # the workspace size of such a length is computed without overflow
+    n = (1 << 31) - 1
+    assert binding.workspace_bytes(1, 1, n, 64) == 2 * ((n + 127) // 128 * 128) * 4
 
 
 def test_empty_problems_are_noops(lib):
