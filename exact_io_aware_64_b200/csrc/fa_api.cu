@@ -94,17 +94,18 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [BH][N][d] bf16 viewed as a 3-D tensor; boxes of 64 elements x 128 rows x 1 head with
-// the 128-byte swizzle that the tensor-core shared-memory descriptors expect.  Rows
-// past N inside a head read as zeros.
-fa_status make_tmap(CUtensorMap* tm, const void* ptr, int BH, int N, int d) {
+// [BH][N][d] bf16 viewed as a 3-D tensor; boxes of 64 elements x `rows` rows x 1 head
+// with the 128-byte swizzle that the tensor-core shared-memory descriptors expect (128
+// rows for the operand tiles, 32 for the forward's per-warp output stores).  Rows past N
+// inside a head read as zeros.
+fa_status make_tmap(CUtensorMap* tm, const void* ptr, int BH, int N, int d, int rows = 128) {
   auto fn = encode_fn();
   if (!fn) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
                         static_cast<cuuint64_t>(BH)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
                            static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -114,17 +115,17 @@ fa_status make_tmap(CUtensorMap* tm, const void* ptr, int BH, int N, int d) {
 }
 
 // Packed [tokens][H][d] bf16 viewed as a 3-D tensor {d, H, tokens}; boxes of 64
-// elements x 1 head x 128 tokens, which land in shared memory exactly like the 64 x 128
-// boxes above (128 rows of 128 bytes, 128-byte swizzle).  Tokens past the end read as
-// zeros.
-fa_status make_tmap_packed(CUtensorMap* tm, const void* ptr, int tokens, int H, int d) {
+// elements x 1 head x `rows` tokens, which land in shared memory exactly like the boxes
+// above (`rows` rows of 128 bytes, 128-byte swizzle).  Tokens past the end read as zeros.
+fa_status make_tmap_packed(CUtensorMap* tm, const void* ptr, int tokens, int H, int d,
+                           int rows = 128) {
   auto fn = encode_fn();
   if (!fn) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
                         static_cast<cuuint64_t>(tokens)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
                            static_cast<cuuint64_t>(H) * static_cast<cuuint64_t>(d) * 2};
-  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(rows)};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -336,12 +337,13 @@ fa_status fwd_impl(const void* Q, const void* K, const void* V, void* O, float* 
   FA_TRY(device_info(&dev));
   FA_TRY(require_sm100(dev));
   const int BH = B * H;
-  CUtensorMap tmQ, tmK, tmV;
+  CUtensorMap tmQ, tmK, tmV, tmO;
   FA_TRY(make_tmap(&tmQ, Q, BH, Nq, d));
   FA_TRY(make_tmap(&tmK, K, BH, Nk, d));
   FA_TRY(make_tmap(&tmV, V, BH, Nk, d));
+  FA_TRY(make_tmap(&tmO, O, BH, Nq, d, 32));
   const fa::Problem p = make_problem(B, H, Nq, Nk, d, scale, causal, dev, seqlens_q, seqlens_k);
-  cudaError_t e = fa::launch_fwd_sm100(tmQ, tmK, tmV, O, LSE, p, dev.num_sms, stream);
+  cudaError_t e = fa::launch_fwd_sm100(tmQ, tmK, tmV, tmO, O, LSE, p, dev.num_sms, stream);
   if (e != cudaSuccess) return cuda_fail(e, "launching the forward kernel");
   return FA_OK;
 }
@@ -576,14 +578,15 @@ fa_status fa_fwd_packed(const void* Q, const void* K, const void* V, void* O, fl
   DeviceInfo dev;
   FA_TRY(device_info(&dev));
   FA_TRY(require_sm100(dev));
-  CUtensorMap tmQ, tmK, tmV;
+  CUtensorMap tmQ, tmK, tmV, tmO;
   FA_TRY(make_tmap_packed(&tmQ, Q, total_q, H, d));
   FA_TRY(make_tmap_packed(&tmK, K, total_k, H, d));
   FA_TRY(make_tmap_packed(&tmV, V, total_k, H, d));
+  FA_TRY(make_tmap_packed(&tmO, O, total_q, H, d, 32));
   const fa::Problem p = make_problem(B, H, max_seqlen_q, max_seqlen_k, d, scale, causal, dev,
                                      nullptr, nullptr, cu_seqlens_q, cu_seqlens_k, total_q,
                                      total_k);
-  cudaError_t e = fa::launch_fwd_sm100(tmQ, tmK, tmV, O, LSE, p, dev.num_sms, stream);
+  cudaError_t e = fa::launch_fwd_sm100(tmQ, tmK, tmV, tmO, O, LSE, p, dev.num_sms, stream);
   if (e != cudaSuccess) return cuda_fail(e, "launching the forward kernel");
   return FA_OK;
 }

@@ -31,6 +31,12 @@
 //     the same reference, and keeps every exponential below 2^8.
 //   * K/V tiles stream through a ring of shared-memory slots guarded by mbarriers
 //     (full: TMA transaction bytes; empty: tcgen05.commit from the MMA thread).
+//   * O leaves through shared memory: each softmax warp writes its 32 rows, 64 columns
+//     at a time, into a 4 KB staging box and its lane 0 issues a bulk tensor store of the
+//     box, so HBM sees whole 128-byte lines and the warp goes on to its next unit while
+//     the store drains.  A store of a row per lane would touch 32 lines per instruction;
+//     at short sequences, where a unit is only a few key tiles long, those stores took
+//     about a third of each unit.
 //   * Queries and keys may differ in number (Nq <= Nk when causal): the queries are then
 //     the last Nq tokens of the sequence, query row r at position r + Nk - Nq, and a
 //     causal row sees keys up to its position (bottom-right alignment; Nq == Nk gives
@@ -89,7 +95,10 @@ struct FwdLayout {
   static constexpr int kQ0 = 0;
   static constexpr int kQ1 = kTileBytes;
   static constexpr int kRing = 2 * kTileBytes;
-  static constexpr int kBar = kRing + kStages * kTileBytes;
+  // O staging for the bulk tensor stores of the epilogue: per softmax warp, one box of
+  // its 32 rows x 64 columns (4 KB)
+  static constexpr int kOst = kRing + kStages * kTileBytes;
+  static constexpr int kBar = kOst + 2 * kBoxBytes;
   // barrier indices
   static constexpr int kBarQFull = 0;                 // [2]
   static constexpr int kBarQEmpty = 2;                // [2]
@@ -186,7 +195,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                      const __grid_constant__ CUtensorMap tmK,
-                     const __grid_constant__ CUtensorMap tmV, const FwdArgs args) {
+                     const __grid_constant__ CUtensorMap tmV,
+                     const __grid_constant__ CUtensorMap tmO, const FwdArgs args) {
   using L = FwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -235,6 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmO);
   }
   if (warp == kWarpMMA) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -503,6 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tOrow = tO[t] + lane_off;
     const uint32_t tProw = tP[t] + lane_off;
     int s_count = 0, o_count = 0;
+    bool st_used = false;  // this warp's O staging box has been handed to a bulk store
     bool ok = true;
     for (int r = 0, w = snake_unit(0); ok && w < args.total_units; w = snake_unit(++r)) {
       const UnitInfo ui = unit_info(w, args);
@@ -630,7 +642,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < D / 32; ++c) tmem_ld32(tOrow + c * 32, &ov[c * 32]);
       tmem_wait_ld();
       warp_arrive(bar(L::kBarOFree + t));
-      if (q_row < ui.lq) {
+      if ((qt * kBM + (warp % 4) * 32 + 32) <= ui.lq) {
+        // all 32 rows of this warp are valid: each row goes, 64 columns at a time, into
+        // the warp's staging box in the 128-byte-swizzled layout of the tensor map (row
+        // r's 16-byte chunk k at r * 128 + ((k ^ (r % 8)) * 16), so the warp writes all
+        // 32 banks four times over), and one bulk tensor store per box writes it to HBM
+        // in whole lines.  The warp's lane 0 issues the stores and, before the box is
+        // written again, waits until the previous store has read it.
+        const uint32_t stg_a = base + L::kOst + (t * 4 + warp % 4) * (32 * 128);
+        uint8_t* stg = smem + (stg_a - base);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          if (st_used) {
+            if (lane == 0) bulk_wait_group_read0();
+            __syncwarp();
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t* o8 = &ov[c * 64 + 8 * k];
+            *reinterpret_cast<uint4*>(stg + lane * 128 + ((k ^ (lane & 7)) << 4)) = make_uint4(
+                pack_bf16x2(__uint_as_float(o8[0]) * inv_l, __uint_as_float(o8[1]) * inv_l),
+                pack_bf16x2(__uint_as_float(o8[2]) * inv_l, __uint_as_float(o8[3]) * inv_l),
+                pack_bf16x2(__uint_as_float(o8[4]) * inv_l, __uint_as_float(o8[5]) * inv_l),
+                pack_bf16x2(__uint_as_float(o8[6]) * inv_l, __uint_as_float(o8[7]) * inv_l));
+          }
+          fence_proxy_async_shared();
+          __syncwarp();
+          if (lane == 0) {
+            const int r0 = qt * kBM + (warp % 4) * 32;
+            tma_store_3d(&tmO, stg_a, c * 64, tma_y(ui, r0), tma_z(ui, ui.tq0, r0));
+            bulk_commit_group();
+          }
+          st_used = true;
+        }
+      } else if (q_row < ui.lq) {
+        // some of the warp's rows belong to no query (or, packed, to the next sequence):
+        // row by row, valid rows only
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t pk[16];
@@ -649,6 +696,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         : static_cast<size_t>(bh) * args.Nq + q_row] =
             (m + __log2f(l)) * 0.69314718055994531f;
     }
+    // the bulk stores this thread issued have completed before the CTA (and its shared
+    // memory) goes away
+    if (lane == 0) bulk_wait_group0();
   }
 
   __syncwarp();
@@ -662,7 +712,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D>
 cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                     void* O, float* LSE, const Problem& p, int num_sms, cudaStream_t stream) {
+                     const CUtensorMap& tmO, void* O, float* LSE, const Problem& p, int num_sms,
+                     cudaStream_t stream) {
   using L = FwdLayout<D>;
   FwdArgs a;
   a.err = p.err;
@@ -693,7 +744,7 @@ cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUten
   if (e != cudaSuccess) return e;
   const int grid = a.total_units < num_sms ? a.total_units : num_sms;
   if ((e = trace_mark(p, 0, stream)) != cudaSuccess) return e;
-  fwd_sm100_kernel<D><<<grid, kThreads, L::kAlloc, stream>>>(tmQ, tmK, tmV, a);
+  fwd_sm100_kernel<D><<<grid, kThreads, L::kAlloc, stream>>>(tmQ, tmK, tmV, tmO, a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   return trace_mark(p, 1, stream);
 }
@@ -701,10 +752,10 @@ cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUten
 }  // namespace
 
 cudaError_t launch_fwd_sm100(const CUtensorMap& tmQ, const CUtensorMap& tmK,
-                             const CUtensorMap& tmV, void* O, float* LSE, const Problem& p,
-                             int num_sms, cudaStream_t stream) {
-  if (p.d == 64) return launch_d<64>(tmQ, tmK, tmV, O, LSE, p, num_sms, stream);
-  return launch_d<128>(tmQ, tmK, tmV, O, LSE, p, num_sms, stream);
+                             const CUtensorMap& tmV, const CUtensorMap& tmO, void* O, float* LSE,
+                             const Problem& p, int num_sms, cudaStream_t stream) {
+  if (p.d == 64) return launch_d<64>(tmQ, tmK, tmV, tmO, O, LSE, p, num_sms, stream);
+  return launch_d<128>(tmQ, tmK, tmV, tmO, O, LSE, p, num_sms, stream);
 }
 
 }  // namespace fa

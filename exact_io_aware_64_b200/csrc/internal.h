@@ -43,11 +43,13 @@ inline cudaError_t trace_mark(const Problem& p, int k, cudaStream_t stream) {
   return cudaEventRecord(p.trace[k], stream);
 }
 
-// Forward, bf16, tcgen05.  Tensor maps describe Q, K, V as 3-D [BH][N][d] bf16 with
-// 64 x 128 x 1 boxes and the 128-byte swizzle.
+// Forward, bf16, tcgen05.  Tensor maps describe Q, K, V and O as 3-D [BH][N][d] bf16
+// (or packed [tokens][H][d]) with the 128-byte swizzle, boxes of 64 x 128 x 1 for Q, K
+// and V and 64 x 32 x 1 for O, which is written through it (bulk tensor stores of 32
+// valid rows at a time) and row by row where a warp's rows are ragged.
 cudaError_t launch_fwd_sm100(const CUtensorMap& tmQ, const CUtensorMap& tmK,
-                             const CUtensorMap& tmV, void* O, float* LSE, const Problem& p,
-                             int num_sms, cudaStream_t stream);
+                             const CUtensorMap& tmV, const CUtensorMap& tmO, void* O, float* LSE,
+                             const Problem& p, int num_sms, cudaStream_t stream);
 
 // Forward, float32 on the CUDA cores.
 cudaError_t launch_fwd_f32(const float* Q, const float* K, const float* V, float* O,
