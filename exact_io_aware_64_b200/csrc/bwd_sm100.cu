@@ -481,6 +481,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) ok = next_s(curq);
       if (ok) ok = next_dp(curd);
       if (!ok) break;
+      // K_j and V_j are read only by the S^T and dP^T products: once the unit's last
+      // dP^T is issued, their slot is released (when it completes) and the next unit's
+      // K and V load while this unit's last dV and dK products and the element-wise work
+      // still run, instead of after them
+      if (m == 1) mma_commit_elect(bar(L::kBarKVEmpty));
       for (int t = 0; t < m; ++t) {
         ok = wait_warp(bar(L::kBarPReady), p_cnt & 1);
         if (ok && t == 0 && units > 0) ok = wait_warp(bar(L::kBarAccFree), (units - 1) & 1);
@@ -511,12 +516,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (t + 1 < m) {
           ok = next_dp(nd);
           if (!ok) break;
+          if (t + 2 == m) mma_commit_elect(bar(L::kBarKVEmpty));
           curq = nq;
           curd = nd;
         }
       }
       if (!ok) break;
-      mma_commit_elect(bar(L::kBarKVEmpty));
       mma_commit_elect(bar(L::kBarAccFull));
     }
     mma_commit_elect(bar(L::kBarDrain));
