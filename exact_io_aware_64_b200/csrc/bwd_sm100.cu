@@ -20,6 +20,11 @@
 //          dS^T = P^T * (dP^T - D_i)
 //          dV_j += P^T dO_i,  dK_j += dS^T Q_i             (TS MMAs, P^T/dS^T from TMEM)
 //      TMEM: dV | dK | S^T (P^T over its first 64 columns) | dP^T (dS^T likewise).
+//      K_j and V_j are released after the unit's last dP^T product, so the next unit's
+//      load overlaps this unit's last products.  At the end of a unit the element-wise
+//      warps of group 0 write dV and those of group 1 write dK, each warp its 32 rows,
+//      through a 4 KB shared-memory staging box and a bulk tensor store (whole lines
+//      instead of a row per lane).
 //   3. bwd_dq: one work unit per (batch*head, 128-row query tile i); key and value tiles
 //      stream past through separate rings (3 slots for K, which the last product of a
 //      tile still reads, 2 for V):  S = Q_i K_j^T, dP = dO_i V_j^T, P, dS as above,
@@ -227,16 +232,17 @@ __device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t* 
 template <int D>
 struct DkdvLayout {
   // K_j and V_j stay for the whole unit.  Query tiles stream through two rings: Q_i
-  // (3 slots; its last reader is the dK product) and dO_i together with the tile's
+  // (2 slots; its last reader is the dK product) and dO_i together with the tile's
   // LSE*log2(e) and D rows (2 slots; read by dP^T, dV and the element-wise warps).
-  // With 3 Q slots the next query tile is loaded a full tile ahead of the S^T product
-  // that needs it.  The layout uses 231.6 KB of the 227 KB (232448 B) a CTA may have,
+  // (A third Q slot measured no faster; its 32 KB hold the epilogue's staging boxes
+  // instead: 4 KB per element-wise warp, through which dK and dV leave by bulk tensor
+  // stores.)  At d = 128 the layout uses 226 KB of the 227 KB (232448 B) a CTA may have,
   // so it leaves no slack for aligning the base: the kernel checks that the dynamic
   // shared memory starts on a 1024-byte boundary (the 128-byte swizzle atoms need it)
   // and reports kErrSmemAlign instead of running if it does not.
   static constexpr int kTileBytes = kTile * D * 2;
   static constexpr int kBoxBytes = 128 * 128;
-  static constexpr int kQStages = 3;
+  static constexpr int kQStages = 2;
   static constexpr int kDOStages = 2;
   static constexpr int kK = 0;
   static constexpr int kV = kTileBytes;
@@ -245,7 +251,8 @@ struct DkdvLayout {
   static constexpr int kDOSlotBytes = kTileBytes + 1024;  // dO tile, L2 row, D row
   static constexpr int kSlotL = kTileBytes;
   static constexpr int kSlotD = kTileBytes + 512;
-  static constexpr int kBar = kDO0 + kDOStages * kDOSlotBytes;
+  static constexpr int kOst = kDO0 + kDOStages * kDOSlotBytes;  // [kEw / 32] x 4 KB
+  static constexpr int kBar = kOst + (kEw / 32) * 4096;
   static constexpr int kBarKVFull = 0, kBarKVEmpty = 1;
   static constexpr int kBarQFull = 2;                            // [kQStages]
   static constexpr int kBarQEmpty = kBarQFull + kQStages;        // [kQStages]
@@ -270,6 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                     const __grid_constant__ CUtensorMap tmL2, const __grid_constant__ CUtensorMap tmD,
+                    const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
                     const BwdArgs args) {
   using L = DkdvLayout<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -533,6 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = (warp % 4) * 32 + lane;  // key row within the tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp % 4) * 32) << 16;
     int stage = 0, units = 0, s_cnt = 0, dp_cnt = 0;
+    bool st_used = false;  // this warp's staging box has been handed to a bulk store
     uint32_t phase = 0;
     bool ok = true;
     int live = 0;
@@ -634,25 +643,62 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (++stage == L::kDOStages) stage = 0, phase ^= 1;
       }
       if (!ok) break;
-      // epilogue: dV and scale * dK for this key row; group g writes columns of its half
+      // epilogue: group 0 writes dV, group 1 scale * dK, each warp its 32 key rows.  A
+      // warp whose rows all lie inside the sequence puts them, 64 columns at a time, into
+      // its staging box in the 128-byte-swizzled layout (row r's 16-byte chunk k at
+      // r * 128 + ((k ^ (r % 8)) * 16): 32 rows cover the 32 banks four times over) and
+      // its lane 0 writes the box out with a bulk tensor store, whole lines at a time;
+      // otherwise the valid rows are stored one per lane.
       ok = wait_warp(bar(L::kBarAccFull), units & 1);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const int kv_row = j * kTile + row;
-      const size_t orow = k_row_offset(args, bh, tk0, kv_row, D);
+      const uint32_t tacc = g == 0 ? tdV : tdK;
+      const float mul = g == 0 ? 1.f : args.scale;
+      const int r0 = j * kTile + (warp % 4) * 32;  // the warp's first key row
+      const bool whole = r0 + 32 <= lk;
+      const uint32_t stg_a = base + L::kOst + warp * 4096;
+      uint8_t* stg = smem + L::kOst + warp * 4096;
+      __nv_bfloat16* grad = g == 0 ? args.dV : args.dK;
+      const size_t orow = k_row_offset(args, bh, tk0, j * kTile + row, D);
 #pragma unroll 1
-      for (int c = g * (D / 64); c < (g + 1) * (D / 64); ++c) {
-        uint32_t v[32];
-        tmem_ld32(tdV + lane_off + c * 32, v);
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t v[64];
+        tmem_ld32(tacc + lane_off + c * 64, v);
+        tmem_ld32(tacc + lane_off + c * 64 + 32, v + 32);
         tmem_wait_ld();
-        if (kv_row < lk) store_row32(args.dV + orow + c * 32, v, 1.f);
-        tmem_ld32(tdK + lane_off + c * 32, v);
-        tmem_wait_ld();
-        if (kv_row < lk) store_row32(args.dK + orow + c * 32, v, args.scale);
+        // the accumulators may be zeroed by the next unit once every warp has read them
+        if (c == D / 64 - 1) warp_arrive(bar(L::kBarAccFree));
+        if (whole) {
+          if (st_used) {
+            if (lane == 0) bulk_wait_group_read0();
+            __syncwarp();
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t* v8 = &v[8 * k];
+            *reinterpret_cast<uint4*>(stg + lane * 128 + ((k ^ (lane & 7)) << 4)) = make_uint4(
+                pack_bf16x2(__uint_as_float(v8[0]) * mul, __uint_as_float(v8[1]) * mul),
+                pack_bf16x2(__uint_as_float(v8[2]) * mul, __uint_as_float(v8[3]) * mul),
+                pack_bf16x2(__uint_as_float(v8[4]) * mul, __uint_as_float(v8[5]) * mul),
+                pack_bf16x2(__uint_as_float(v8[6]) * mul, __uint_as_float(v8[7]) * mul));
+          }
+          fence_proxy_async_shared();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(g == 0 ? &tmdV : &tmdK, stg_a, c * 64, tma_y(bh, r0), tma_z(bh, tk0, r0));
+            bulk_commit_group();
+          }
+          st_used = true;
+        } else if (j * kTile + row < lk) {
+          store_row32(grad + orow + c * 64, v, mul);
+          store_row32(grad + orow + c * 64 + 32, v + 32, mul);
+        }
       }
-      warp_arrive(bar(L::kBarAccFree));
     }
+    // the bulk stores this thread issued have completed before the CTA (and its shared
+    // memory) goes away
+    if (lane == 0) bulk_wait_group0();
   }
 
   __syncwarp();
@@ -1074,7 +1120,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D>
 cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                      const CUtensorMap& tmdO, const CUtensorMap& tmL2, const CUtensorMap& tmD,
-                     const void* O, const void* dO, const float* LSE, void* dQ, void* dK,
+                     const CUtensorMap& tmdK, const CUtensorMap& tmdV, const void* O, const void* dO, const float* LSE, void* dQ, void* dK,
                      void* dV, float* ws, const Problem& p, int num_sms, cudaStream_t stream) {
   BwdArgs a;
   a.err = p.err;
@@ -1129,8 +1175,8 @@ cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUten
   e = cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            DkdvLayout<D>::kAlloc);
   if (e != cudaSuccess) return e;
-  bwd_dkdv_kernel<D><<<grid_kv, kThreads, DkdvLayout<D>::kAlloc, stream>>>(tmQ, tmK, tmV, tmdO,
-                                                                            tmL2, tmD, a_kv);
+  bwd_dkdv_kernel<D><<<grid_kv, kThreads, DkdvLayout<D>::kAlloc, stream>>>(
+      tmQ, tmK, tmV, tmdO, tmL2, tmD, tmdK, tmdV, a_kv);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if ((e = trace_mark(p, 2, stream)) != cudaSuccess) return e;
   e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1147,15 +1193,16 @@ long long bwd_padded_rows(long long N) { return (N + kTile - 1) / kTile * kTile;
 
 cudaError_t launch_bwd_sm100(const CUtensorMap& tmQ, const CUtensorMap& tmK,
                              const CUtensorMap& tmV, const CUtensorMap& tmdO,
-                             const CUtensorMap& tmL2, const CUtensorMap& tmD, const void* O,
+                             const CUtensorMap& tmL2, const CUtensorMap& tmD,
+                             const CUtensorMap& tmdK, const CUtensorMap& tmdV, const void* O,
                              const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
                              float* workspace, const Problem& p, int num_sms,
                              cudaStream_t stream) {
   if (p.d == 64)
-    return launch_d<64>(tmQ, tmK, tmV, tmdO, tmL2, tmD, O, dO, LSE, dQ, dK, dV, workspace, p,
-                        num_sms, stream);
-  return launch_d<128>(tmQ, tmK, tmV, tmdO, tmL2, tmD, O, dO, LSE, dQ, dK, dV, workspace, p,
-                       num_sms, stream);
+    return launch_d<64>(tmQ, tmK, tmV, tmdO, tmL2, tmD, tmdK, tmdV, O, dO, LSE, dQ, dK, dV,
+                        workspace, p, num_sms, stream);
+  return launch_d<128>(tmQ, tmK, tmV, tmdO, tmL2, tmD, tmdK, tmdV, O, dO, LSE, dQ, dK, dV,
+                       workspace, p, num_sms, stream);
 }
 
 }  // namespace fa

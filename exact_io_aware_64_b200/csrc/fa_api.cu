@@ -372,18 +372,20 @@ fa_status bwd_impl(const void* Q, const void* K, const void* V, const void* O, c
   FA_TRY(device_info(&dev));
   FA_TRY(require_sm100(dev));
   const int BH = B * H;
-  CUtensorMap tmQ, tmK, tmV, tmdO, tmL2, tmD;
+  CUtensorMap tmQ, tmK, tmV, tmdO, tmL2, tmD, tmdK, tmdV;
   FA_TRY(make_tmap(&tmQ, Q, BH, Nq, d));
   FA_TRY(make_tmap(&tmK, K, BH, Nk, d));
   FA_TRY(make_tmap(&tmV, V, BH, Nk, d));
   FA_TRY(make_tmap(&tmdO, dO, BH, Nq, d));
+  FA_TRY(make_tmap(&tmdK, dK, BH, Nk, d, 32));
+  FA_TRY(make_tmap(&tmdV, dV, BH, Nk, d, 32));
   const int Npad = static_cast<int>(fa::bwd_padded_rows(Nq));  // Nq <= kMaxRows
   float* ws = static_cast<float*>(workspace);
   FA_TRY(make_row_tmap(&tmD, ws, BH, Npad));
   FA_TRY(make_row_tmap(&tmL2, ws + static_cast<size_t>(BH) * Npad, BH, Npad));
   const fa::Problem p = make_problem(B, H, Nq, Nk, d, scale, causal, dev, seqlens_q, seqlens_k);
-  cudaError_t e = fa::launch_bwd_sm100(tmQ, tmK, tmV, tmdO, tmL2, tmD, O, dO, LSE, dQ, dK, dV,
-                                       ws, p, dev.num_sms, stream);
+  cudaError_t e = fa::launch_bwd_sm100(tmQ, tmK, tmV, tmdO, tmL2, tmD, tmdK, tmdV, O, dO, LSE,
+                                       dQ, dK, dV, ws, p, dev.num_sms, stream);
   if (e != cudaSuccess) return cuda_fail(e, "launching the backward kernels");
   return FA_OK;
 }
@@ -620,11 +622,13 @@ fa_status fa_bwd_packed(const void* Q, const void* K, const void* V, const void*
   FA_TRY(device_info(&dev));
   FA_TRY(require_sm100(dev));
   const int BH = B * H;
-  CUtensorMap tmQ, tmK, tmV, tmdO, tmL2, tmD;
+  CUtensorMap tmQ, tmK, tmV, tmdO, tmL2, tmD, tmdK, tmdV;
   FA_TRY(make_tmap_packed(&tmQ, Q, total_q, H, d));
   FA_TRY(make_tmap_packed(&tmK, K, total_k, H, d));
   FA_TRY(make_tmap_packed(&tmV, V, total_k, H, d));
   FA_TRY(make_tmap_packed(&tmdO, dO, total_q, H, d));
+  FA_TRY(make_tmap_packed(&tmdK, dK, total_k, H, d, 32));
+  FA_TRY(make_tmap_packed(&tmdV, dV, total_k, H, d, 32));
   const int Npad = static_cast<int>(fa::bwd_padded_rows(max_seqlen_q));
   float* ws = static_cast<float*>(workspace);
   FA_TRY(make_row_tmap(&tmD, ws, BH, Npad));
@@ -632,8 +636,8 @@ fa_status fa_bwd_packed(const void* Q, const void* K, const void* V, const void*
   const fa::Problem p = make_problem(B, H, max_seqlen_q, max_seqlen_k, d, scale, causal, dev,
                                      nullptr, nullptr, cu_seqlens_q, cu_seqlens_k, total_q,
                                      total_k);
-  cudaError_t e = fa::launch_bwd_sm100(tmQ, tmK, tmV, tmdO, tmL2, tmD, O, dO, LSE, dQ, dK, dV,
-                                       ws, p, dev.num_sms, stream);
+  cudaError_t e = fa::launch_bwd_sm100(tmQ, tmK, tmV, tmdO, tmL2, tmD, tmdK, tmdV, O, dO, LSE,
+                                       dQ, dK, dV, ws, p, dev.num_sms, stream);
   if (e != cudaSuccess) return cuda_fail(e, "launching the backward kernels");
   return FA_OK;
 }

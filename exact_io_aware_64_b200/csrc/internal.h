@@ -58,11 +58,13 @@ cudaError_t launch_fwd_f32(const float* Q, const float* K, const float* V, float
 // Backward, bf16: -D = -rowsum(dO * O) and -L2 = -LSE * log2(e) into the workspace,
 // then dK/dV, then dQ.  Workspace layout: -D as [BH][Npad] float, then -L2 as [BH][Npad]
 // float, Npad = bwd_padded_rows(N).  tmL2 / tmD describe those two arrays as 3-D
-// [1][BH][Npad] float tensors with 128 x 1 x 1 boxes.
+// [1][BH][Npad] float tensors with 128 x 1 x 1 boxes.  tmdK / tmdV describe dK and dV
+// like K and V but with 64 x 32 x 1 boxes: the dK/dV kernel writes them through these.
 long long bwd_padded_rows(long long N);
 cudaError_t launch_bwd_sm100(const CUtensorMap& tmQ, const CUtensorMap& tmK,
                              const CUtensorMap& tmV, const CUtensorMap& tmdO,
-                             const CUtensorMap& tmL2, const CUtensorMap& tmD, const void* O,
+                             const CUtensorMap& tmL2, const CUtensorMap& tmD,
+                             const CUtensorMap& tmdK, const CUtensorMap& tmdV, const void* O,
                              const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
                              float* workspace, const Problem& p, int num_sms,
                              cudaStream_t stream);
