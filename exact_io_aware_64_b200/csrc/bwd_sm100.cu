@@ -101,6 +101,7 @@ struct BwdArgs {
   int n_kt;         // ceil(Nk / 128)
   int total_units;  // this kernel's units: BH * n_kt (dK/dV) or BH * n_qt (dQ)
   int causal;
+  int dq_aligned32;  // dQ starts on a 32-byte boundary (its rows then allow 32-byte stores)
   float scale;
   float scale_log2;
 };
@@ -226,6 +227,20 @@ __device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t* 
   uint4* d = reinterpret_cast<uint4*>(dst);
 #pragma unroll
   for (int k = 0; k < 4; ++k) d[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+}
+
+// The same for 64 columns with 32-byte stores (dst 32-byte aligned).
+__device__ __forceinline__ void store_row64_v8(__nv_bfloat16* dst, const uint32_t* v, float mul) {
+  uint32_t pk[32];
+#pragma unroll
+  for (int k = 0; k < 32; ++k)
+    pk[k] = pack_bf16x2(__uint_as_float(v[2 * k]) * mul, __uint_as_float(v[2 * k + 1]) * mul);
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst + 16 * k),
+                 "r"(pk[8 * k]), "r"(pk[8 * k + 1]), "r"(pk[8 * k + 2]), "r"(pk[8 * k + 3]),
+                 "r"(pk[8 * k + 4]), "r"(pk[8 * k + 5]), "r"(pk[8 * k + 6]), "r"(pk[8 * k + 7])
+                 : "memory");
 }
 
 // ------------------------------------------------------------------ 2. dK, dV
@@ -1095,15 +1110,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const size_t orow = q_row_offset(args, bh, tq0, q_row, D);
-#pragma unroll 1
-      for (int c = g * (D / 64); c < (g + 1) * (D / 64); ++c) {
-        uint32_t v[32];
-        tmem_ld32(tdQ + lane_off + c * 32, v);
-        tmem_wait_ld();
-        if (q_row < lq) store_row32(args.dQ + orow + c * 32, v, args.scale);
-      }
+      const size_t orow = q_row_offset(args, bh, tq0, q_row, D) + g * (D / 2);
+      // this group's half of the row: read whole, release the accumulator (the next
+      // unit's first dQ product may start), then store it, 32 bytes per store where dQ
+      // is aligned for that (half as many store instructions, each still touching a
+      // line per row)
+      uint32_t v[D / 2];
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) tmem_ld32(tdQ + lane_off + g * (D / 2) + c * 32, v + c * 32);
+      tmem_wait_ld();
       warp_arrive(bar(L::kBarAccFree));
+      if (q_row < lq) {
+        if (D == 128 && args.dq_aligned32) {
+          store_row64_v8(args.dQ + orow, v, args.scale);
+        } else {
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) store_row32(args.dQ + orow + c * 32, v + c * 32, args.scale);
+        }
+      }
     }
   }
 
@@ -1141,6 +1165,7 @@ cudaError_t launch_d(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUten
   a.n_kt = (p.Nk + kTile - 1) / kTile;
   a.Npad = a.n_qt * kTile;
   a.causal = p.causal;
+  a.dq_aligned32 = (reinterpret_cast<uintptr_t>(dQ) & 31u) == 0;
   a.scale = p.scale;
   a.scale_log2 = p.scale * kLog2e;
   float* Dpad = ws;

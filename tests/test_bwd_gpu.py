@@ -119,6 +119,29 @@ def test_bwd_deterministic_and_in_bounds():
     assert bool((wsbuf[:guard] == 0xAB).all()) and bool((wsbuf[-guard:] == 0xAB).all())
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_outputs_at_16_byte_offsets(d):
+    """Outputs that start 16 bytes past a 32-byte boundary (the least alignment the calls
+    accept) get the same bits as outputs at aligned addresses: O, dQ, dK and dV, whose
+    stores use wider or bulk forms where the address allows."""
+    B, H, N = 1, 3, 300
+    ins = inputs.make_inputs(B, H, N, d, seed=21, with_dO=True)
+    q, k, v, do = (ins[n].cuda() for n in ("Q", "K", "V", "dO"))
+    O, LSE = binding.fwd(q, k, v, causal=True)
+    dQ, dK, dV = binding.bwd(q, k, v, O, do, LSE, causal=True)
+    n = B * H * N * d
+    bufs = [torch.full((n + 64,), 3.0, device="cuda", dtype=torch.bfloat16) for _ in range(4)]
+    views = [b[8:8 + n].view(B, H, N, d) for b in bufs]  # 16 bytes past the allocation
+    assert all(t.data_ptr() % 32 == 16 for t in views)
+    O2, _ = binding.fwd(q, k, v, causal=True, O=views[0])
+    binding.bwd(q, k, v, O, do, LSE, causal=True, dQ=views[1], dK=views[2], dV=views[3])
+    binding.check_device_error()
+    for got, want in zip(views, (O, dQ, dK, dV)):
+        assert torch.equal(got, want)
+    for b in bufs:
+        assert bool((b[:8] == 3.0).all()) and bool((b[8 + n:] == 3.0).all())
+
+
 def test_bwd_rejects_small_workspace():
     ins = inputs.make_inputs(1, 2, 256, 64, seed=1, with_dO=True)
     q, k, v, do = (ins[n].cuda() for n in ("Q", "K", "V", "dO"))
