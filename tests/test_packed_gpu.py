@@ -31,6 +31,10 @@ def _cu(lengths):
 CASES = [
     ([300, 1, 129, 0, 77, 256], [300, 1, 129, 5, 200, 256]),
     ([256, 100, 1, 200, 0], [640, 100, 33, 513, 0]),
+    # lengths around the 32-row groups the output stores work in: a group of rows that
+    # ends inside a sequence is written whole, one that crosses its end row by row (the
+    # rows after it belong to the next sequence)
+    ([31, 32, 33, 95, 96, 97, 160], [31, 32, 33, 95, 96, 97, 160]),
 ]
 
 
