@@ -159,9 +159,11 @@ __device__ __forceinline__ size_t lse_index(const BwdArgs& a, int bh, int t0, in
 // ------------------------------------------------------------------ 1. preparation
 // Stores the negated row statistics the element-wise steps add:
 //   ND[bh][r] = -sum_k dO[bh][r][k] * O[bh][r][k],   NL2[bh][r] = -LSE[bh][r] * log2(e).
-// Padded rows r in [N, Npad): ND = 0, NL2 = -inf (their probabilities are exactly 0).  Bandwidth bound: each thread reads 16
-// bytes of O and of dO for kRowsPerThread rows (independent loads in flight), the
-// D / 8 threads of a row combine their partial sums with shuffles.
+// Padded rows r in [N, Npad): ND = 0, NL2 = -inf (their probabilities are exactly 0).
+// Bandwidth bound: each thread issues its 16-byte loads of O and dO for all of its
+// kPrepRowsPerThread rows before using any (all in flight together), the D / 8 threads
+// of a row combine their partial sums with shuffles, and a block's rows lie in one head
+// (no per-row division).
 constexpr int kPrepThreads = 256;
 constexpr int kPrepRowsPerThread = 4;
 
@@ -170,49 +172,51 @@ __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(
     const __nv_bfloat16* __restrict__ O, const __nv_bfloat16* __restrict__ dO,
     const float* __restrict__ LSE, float* __restrict__ Dout, float* __restrict__ L2out,
     const BwdArgs a) {
-  const int BH = a.BH, Npad = a.Npad;
+  const int Npad = a.Npad;
   constexpr int kPer = D / 8;                         // threads per row (8 bf16 each)
   constexpr int kRowsPerPass = kPrepThreads / kPer;   // rows covered by one pass
+  constexpr int kRowsPerBlock = kRowsPerPass * kPrepRowsPerThread;
+  static_assert(128 % kRowsPerBlock == 0, "a block's rows must lie in one head");
   const int part = threadIdx.x % kPer;
-  const long long total = static_cast<long long>(BH) * Npad;
-  const long long row0 = (static_cast<long long>(blockIdx.x) * kPrepRowsPerThread) * kRowsPerPass +
-                         threadIdx.x / kPer;
-  float acc[kPrepRowsPerThread];
+  // Npad is a multiple of 128, so a block's rows lie in one head
+  const long long blk_row0 = static_cast<long long>(blockIdx.x) * kRowsPerBlock;
+  const int bh = static_cast<int>(blk_row0 / Npad);
+  if (bh >= a.BH) return;
+  const int rb = static_cast<int>(blk_row0 - static_cast<long long>(bh) * Npad) + threadIdx.x / kPer;
+  int lq, lk, tq0, tk0;
+  seq_info(a, bh, lq, lk, tq0, tk0);
+  // every load of the thread's rows first, so that they are all in flight together
+  uint4 va[kPrepRowsPerThread], vb[kPrepRowsPerThread];
 #pragma unroll
   for (int k = 0; k < kPrepRowsPerThread; ++k) {
-    acc[k] = 0.f;
-    const long long row = row0 + static_cast<long long>(k) * kRowsPerPass;
-    if (row >= total) continue;
-    const int bh = static_cast<int>(row / Npad);
-    const int r = static_cast<int>(row % Npad);
-    int lq, lk, tq0, tk0;
-    seq_info(a, bh, lq, lk, tq0, tk0);
+    const int r = rb + k * kRowsPerPass;
     if (r < lq) {
       const size_t off = q_row_offset(a, bh, tq0, r, D) + part * 8;
-      const uint4 a = *reinterpret_cast<const uint4*>(O + off);
-      const uint4 b = *reinterpret_cast<const uint4*>(dO + off);
-      const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
-      const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 fa = __bfloat1622float2(pa[e]);
-        const float2 fb = __bfloat1622float2(pb[e]);
-        acc[k] = fmaf(fa.x, fb.x, acc[k]);
-        acc[k] = fmaf(fa.y, fb.y, acc[k]);
-      }
+      va[k] = *reinterpret_cast<const uint4*>(O + off);
+      vb[k] = *reinterpret_cast<const uint4*>(dO + off);
+    } else {
+      va[k] = make_uint4(0u, 0u, 0u, 0u);
+      vb[k] = make_uint4(0u, 0u, 0u, 0u);
     }
   }
 #pragma unroll
   for (int k = 0; k < kPrepRowsPerThread; ++k) {
+    float acc = 0.f;
+    const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&va[k]);
+    const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&vb[k]);
 #pragma unroll
-    for (int o = kPer / 2; o > 0; o >>= 1) acc[k] += __shfl_xor_sync(0xffffffffu, acc[k], o);
-    const long long row = row0 + static_cast<long long>(k) * kRowsPerPass;
-    if (part == 0 && row < total) {
-      const int bh = static_cast<int>(row / Npad);
-      const int r = static_cast<int>(row % Npad);
-      int lq, lk, tq0, tk0;
-      seq_info(a, bh, lq, lk, tq0, tk0);
-      Dout[row] = -acc[k];
+    for (int e = 0; e < 4; ++e) {
+      const float2 fa = __bfloat1622float2(pa[e]);
+      const float2 fb = __bfloat1622float2(pb[e]);
+      acc = fmaf(fa.x, fb.x, acc);
+      acc = fmaf(fa.y, fb.y, acc);
+    }
+#pragma unroll
+    for (int o = kPer / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    const int r = rb + k * kRowsPerPass;
+    if (part == 0) {
+      const size_t row = static_cast<size_t>(bh) * Npad + r;
+      Dout[row] = -acc;
       L2out[row] = r < lq ? -LSE[lse_index(a, bh, tq0, r)] * kLog2e : -INFINITY;
     }
   }
