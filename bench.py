@@ -456,11 +456,14 @@ def run_gpu(args, w):
 
     # (b) pipelined, as a throughput-minded caller would run it: step i's inputs go up
     # on one stream while step i-1 computes and step i-2's results come down on a third
-    # (PCIe carries both directions at once).  Two sets of device buffers take turns;
-    # events order each copy after the step that last used its buffers.  Every step still
-    # moves all its inputs in and all its results out inside the timed region.
+    # (PCIe carries both directions at once).  Three sets of device buffers take turns
+    # (one more than the three stages strictly need, so that a slow copy in one direction
+    # does not stall the other); events order each copy after the step that last used
+    # its buffers.  Every step still moves all its inputs in and all its results out
+    # inside the timed region.
+    n_sets = 3
     sets = []
-    for _ in range(2):
+    for _ in range(n_sets):
         di = {n: torch.empty_like(t) for n, t in (("q", q), ("k", k), ("v", v), ("do", do))}
         do_ = {"O": torch.empty_like(O), "LSE": torch.empty_like(LSE)}
         if with_bwd:
@@ -473,19 +476,19 @@ def run_gpu(args, w):
     def pipelined(n_steps):
         computed, downloaded = [], []
         for i in range(n_steps):
-            di, dout, ho = sets[i % 2]
+            di, dout, ho = sets[i % n_sets]
             up = torch.cuda.Event()
             with torch.cuda.stream(s_up):
-                if i >= 2:
-                    s_up.wait_event(computed[i - 2])
+                if i >= n_sets:
+                    s_up.wait_event(computed[i - n_sets])
                 for n, t in di.items():
                     t.copy_(hin[n], non_blocking=True)
                 up.record(s_up)
             cmp_done = torch.cuda.Event()
             with torch.cuda.stream(s_cmp):
                 s_cmp.wait_event(up)
-                if i >= 2:
-                    s_cmp.wait_event(downloaded[i - 2])
+                if i >= n_sets:
+                    s_cmp.wait_event(downloaded[i - n_sets])
                 binding.fwd(di["q"], di["k"], di["v"], scale=w.scale, causal=w.causal,
                             O=dout["O"], LSE=dout["LSE"], stream=s_cmp)
                 if with_bwd:
@@ -502,7 +505,7 @@ def run_gpu(args, w):
                 dn.record(s_down)
             downloaded.append(dn)
 
-    pipelined(3)
+    pipelined(n_sets + 1)
     torch.cuda.synchronize()
     fa_dist.barrier(info)
     p0, p1 = ev(), ev()
