@@ -261,8 +261,9 @@ struct DkdvLayout {
   // and reports kErrSmemAlign instead of running if it does not.
   static constexpr int kTileBytes = kTile * D * 2;
   static constexpr int kBoxBytes = 128 * 128;
-  static constexpr int kQStages = 2;
-  static constexpr int kDOStages = 2;
+  // (d = 64 tiles are half the size: three slots in each ring there)
+  static constexpr int kQStages = (D == 64) ? 3 : 2;
+  static constexpr int kDOStages = (D == 64) ? 3 : 2;
   static constexpr int kK = 0;
   static constexpr int kV = kTileBytes;
   static constexpr int kQ0 = 2 * kTileBytes;
